@@ -1,0 +1,28 @@
+"""B200-native paged GQA decode attention.
+
+Single-token decode attention read straight through a paged KV cache's block
+table, where G = H_q / H_kv query heads share each KV head: a split-S kernel
+whose chunks produce partial softmax states, an exact merge, a compact work
+queue and a calibrated policy that picks no-split, split-S or work-queue per
+batch.  Every step runs in the C-ABI library `libpkv.so` (CUDA for sm_100a plus
+host C++); this package only marshals arguments to it.
+
+The CUDA library is loaded on first use of anything but `workloads`; if it is
+missing or cannot find a GPU, the call raises instead of falling back.
+"""
+from . import workloads  # noqa: F401  (inputs only; no CUDA needed)
+
+_LAZY = {
+    "lib", "paged_decode", "plan_decode", "DecodePlan", "Shape", "Plan", "Rule",
+    "select_policy", "build_work_queue", "workspace_bytes", "plan_counters",
+    "load_rules", "default_rules", "decode_host", "PkvError",
+    "NO_SPLIT", "SPLIT_S", "WORK_QUEUE", "FLAG_SEPARATE_MERGE",
+}
+
+
+def __getattr__(name):
+    if name in _LAZY:
+        from . import binding
+
+        return getattr(binding, name)
+    raise AttributeError(name)

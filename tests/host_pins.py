@@ -1,0 +1,195 @@
+"""Pins for the oracle's host scheduling pieces (work queue, policy, counters).
+
+Each check takes the oracle module `O`, so the same checks run against the
+real oracle and against copies with a planted mistake.
+
+  queue_closed_form   n_items = H_kv * sum_i max(1, ceil(ceil(N_i / P) / C))
+  queue_cover         per (row, head), items tile [0, N_i) in order, without
+                      gaps or overlap, every item non-empty and page aligned
+  queue_bruteforce    enumerate-and-filter over a rectangular (i, h, c) grid
+  policy_paper        the page's decisions at B = 1 / 4 / 8 (tests/golden/paper_policy.txt)
+  policy_semantics    first match wins, ranges are half-open, S' and C closed forms
+  launch_fanout       16 bucket launches vs 2 queue launches at B = 8
+                      (tests/golden/launch_fanout_b8.txt)
+  merge_state_closed  queue merge traffic = 2*G*(D+2)*4 * H_kv * (slots of
+                      multi-chunk pairs); rectangular = the same over B*H_kv*S slots
+"""
+from __future__ import annotations
+
+import itertools
+import os
+import random
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+PKG = os.path.join(os.path.dirname(HERE), "paged_kv_gqa_17_b200")
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+CASES = [
+    ([512], 1, 16, 4),
+    ([32768], 8, 16, 64),
+    ([0, 1, 15, 16, 17, 255, 256, 257], 2, 16, 1),
+    ([0, 1, 15, 16, 17, 255, 256, 257], 3, 16, 5),
+    ([4097, 16384, 9000, 5001], 8, 16, 16),
+    ([0, 0], 4, 16, 2),
+    ([], 8, 16, 8),
+]
+
+
+def _random_cases(seed=7, n=40):
+    rng = random.Random(seed)
+    for _ in range(n):
+        B = rng.randint(1, 9)
+        lens = [rng.choice([0, rng.randint(1, 40), rng.randint(1, 5000)]) for _ in range(B)]
+        yield lens, rng.randint(1, 8), rng.choice([8, 16, 32]), rng.randint(1, 70)
+
+
+def queue_closed_form(O):
+    for lens, H_kv, P, C in itertools.chain(CASES, _random_cases()):
+        items, indptr = O.build_work_queue(lens, H_kv, P, C)
+        want = H_kv * sum(max(1, _cdiv(_cdiv(n, P), C)) for n in lens)
+        assert len(items) == want, ("queue_closed_form", lens, H_kv, P, C)
+        assert len(indptr) == len(lens) * H_kv + 1 and indptr[-1] == len(items)
+
+
+def queue_cover(O):
+    for lens, H_kv, P, C in itertools.chain(CASES, _random_cases(8)):
+        items, indptr = O.build_work_queue(lens, H_kv, P, C)
+        for i, n in enumerate(lens):
+            for h in range(H_kv):
+                pair = items[indptr[i * H_kv + h]:indptr[i * H_kv + h + 1]]
+                assert all(it[0] == i and it[1] == h for it in pair), "queue_cover: wrong pair"
+                if n == 0:
+                    assert pair == [(i, h, 0, 0)], "queue_cover: empty row"
+                    continue
+                pos = 0
+                for (_, _, b, e) in pair:
+                    assert b == pos and e > b and b % (C * P) == 0, ("queue_cover", lens, i, h, pair)
+                    assert e - b <= C * P
+                    pos = e
+                assert pos == n, ("queue_cover: gap at end", lens, i, h)
+
+
+def queue_bruteforce(O):
+    for lens, H_kv, P, C in itertools.chain(CASES, _random_cases(9)):
+        items, indptr = O.build_work_queue(lens, H_kv, P, C)
+        n_max = max(lens, default=0)
+        grid = []
+        for i, h, c in itertools.product(range(len(lens)), range(H_kv), range(max(1, _cdiv(n_max, C * P)))):
+            n = lens[i]
+            if n == 0 and c == 0:
+                grid.append((i, h, 0, 0))
+            elif c * C * P < n:
+                grid.append((i, h, c * C * P, min(n, (c + 1) * C * P)))
+        assert items == grid, ("queue_bruteforce", lens, H_kv, P, C)
+        ptr = [0]
+        for i, h in itertools.product(range(len(lens)), range(H_kv)):
+            ptr.append(ptr[-1] + sum(1 for it in grid if it[0] == i and it[1] == h))
+        assert indptr == ptr
+
+
+def read_golden(name):
+    rows = []
+    with open(os.path.join(HERE, "golden", name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def policy_paper(O):
+    rules = O.load_rules(os.path.join(PKG, "policy_paper_rule.json"))
+    names = {"NO_SPLIT": O.NO_SPLIT, "SPLIT_S": O.SPLIT_S, "WORK_QUEUE": O.WORK_QUEUE}
+    for B, n_max, mode in read_golden("paper_policy.txt"):
+        B, n_max = int(B), int(n_max)
+        lens = [n_max] + [max(1, n_max // 3)] * (B - 1)
+        plan = O.select_policy(lens, 16, rules)
+        assert plan[0] == names[mode], ("policy_paper", B, n_max, plan)
+
+
+def policy_semantics(O):
+    R = O.Rule
+    rules = [R(1, 2, 4096, O.INT32_MAX, O.SPLIT_S, num_splits=37),
+             R(1, 2, 0, 4096, O.NO_SPLIT, flags=1),
+             R(2, 8, 0, O.INT32_MAX, O.WORK_QUEUE, chunk_pages=24, flags=1),
+             R(0, O.INT32_MAX, 0, O.INT32_MAX, O.WORK_QUEUE, chunk_pages=8)]
+    P = 16
+    # B = 1, N_max = 32768: S = 37 -> C = ceil(2048 / 37) = 56, S' = ceil(2048 / 56) = 37
+    assert O.select_policy([32768], P, rules) == (O.SPLIT_S, 37, 56, 0)
+    # boundary of a half-open range: 4096 belongs to the first rule, 4095 to the second;
+    # 256 pages, S = 37 -> C = ceil(256 / 37) = 7, S' = ceil(256 / 7) = 37
+    assert O.select_policy([4096], P, rules) == (O.SPLIT_S, 37, 7, 0)
+    # 100 pages, S = 37 -> C = 3, S' = ceil(100 / 3) = 34: the tight split count
+    assert O.select_policy([1600], P, [R(1, 2, 0, O.INT32_MAX, O.SPLIT_S, num_splits=37)]) == (O.SPLIT_S, 34, 3, 0)
+    assert O.select_policy([4095], P, rules) == (O.NO_SPLIT, 1, 0, 1)
+    # B = 8 misses [2, 8) and falls to the catch-all
+    assert O.select_policy([100] * 8, P, rules) == (O.WORK_QUEUE, 1, 8, 0)
+    assert O.select_policy([1000, 5] * 2, P, rules) == (O.WORK_QUEUE, 3, 24, 1)
+    # no rule matches -> single kernel; empty batch and all-empty rows -> single kernel
+    assert O.select_policy([10], P, rules[:1]) == (O.NO_SPLIT, 1, 0, 0)
+    assert O.select_policy([], P, rules) == (O.NO_SPLIT, 1, 0, 0)
+    assert O.select_policy([0, 0], P, rules) == (O.NO_SPLIT, 1, 0, 0)
+    for bad in ([R(0, 9, 0, 9, 7)], [R(0, 9, 0, 9, O.SPLIT_S, num_splits=0)],
+                [R(0, 9, 0, 9, O.WORK_QUEUE, chunk_pages=0)]):
+        try:
+            O.select_policy([5], P, bad)
+        except ValueError:
+            continue
+        raise AssertionError("policy_semantics: invalid table accepted")
+    try:
+        O.select_policy([-1], P, rules)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("policy_semantics: negative length accepted")
+
+
+def launch_fanout(O):
+    g = {k: int(v) for k, v in read_golden("launch_fanout_b8.txt")}
+    rng = random.Random(5)
+    lens = sorted(rng.sample(range(600, 40000), g["distinct_lengths"]))
+    assert len(lens) == g["batch"]
+    plan = (O.WORK_QUEUE, 0, 32, O.FLAG_SEPARATE_MERGE)
+    plan = (plan[0], _cdiv(_cdiv(max(lens), 16), 32), 32, plan[3])
+    c = O.counters(lens, 32, 8, 128, 16, plan)
+    assert c.bucket_launches == g["bucket_launches_per_step"], ("launch_fanout", c)
+    assert c.launches == g["queue_launches_per_step"], ("launch_fanout", c)
+    # exact-length bucketing launches one (split, merge) pair per distinct
+    # non-empty length, however many rows share it
+    rep = [700, 700, 5000, 700, 5000, 0, 123, 123]
+    c = O.counters(rep, 32, 8, 128, 16, plan)
+    assert c.bucket_launches == 2 * 3, ("launch_fanout", c)
+
+
+def merge_state_closed(O):
+    for lens, H_kv, P, C in itertools.chain(CASES, _random_cases(10)):
+        if not lens:
+            continue
+        H_q, D = H_kv * 4, 64
+        state = 4 * (D + 2) * 4
+        S = max(1, _cdiv(_cdiv(max(lens), P), C))
+        wq = O.counters(lens, H_q, H_kv, D, P, (O.WORK_QUEUE, S, C, 0))
+        rect = O.counters(lens, H_q, H_kv, D, P, (O.SPLIT_S, S, C, 0))
+        slots = sum(k for k in (max(1, _cdiv(_cdiv(n, P), C)) for n in lens) if k > 1)
+        assert wq.merge_state_bytes == 2 * state * H_kv * slots, ("merge_state_closed", lens)
+        assert rect.merge_state_bytes == (2 * state * len(lens) * H_kv * S if S > 1 else 0)
+        assert wq.work_items + rect.empty_items == rect.work_items + H_kv * sum(1 for n in lens if n == 0)
+        assert wq.kv_bytes == rect.kv_bytes == sum(lens) * H_kv * 4 * D
+
+
+HOST_PINS = (queue_closed_form, queue_cover, queue_bruteforce, policy_paper, policy_semantics,
+             launch_fanout, merge_state_closed)
+
+
+def run_all(O):
+    failed = []
+    for pin in HOST_PINS:
+        try:
+            pin(O)
+        except (AssertionError, ValueError, IndexError, TypeError) as e:
+            failed.append(f"{pin.__name__}: {e}")
+    return failed
