@@ -1,0 +1,258 @@
+/*
+ * pkv.h - C ABI of the B200 paged GQA decode-attention library (libpkv.so).
+ *
+ * One decode step: every sequence ("row") i of a batch has one new query
+ * token with H_q query heads and N_i cached tokens whose keys and values live
+ * in a paged pool.  G = H_q / H_kv query heads share each KV head; query head
+ * hq reads KV head floor(hq / G).  For each (row, query head):
+ *
+ *     out = softmax(scale * q . K^T) V     over the row's N_i cached tokens,
+ *
+ * with K and V read straight through the block table, never repacked:
+ * token t of row i is slot t mod P of physical page block_table[i][t / P].
+ * Sources: "PersistentKV: Page-Aware Decode Scheduling for Long-Context LLM
+ * Serving on Commodity GPUs" (gist.science explainer, "PKV" below), Technical
+ * summary > Methodology > 1 "Native block-table decode engine" (GQA grouping,
+ * layout without repacking); "Chapter 8 - Next-generation KV cache management"
+ * (actionbridge.io), section 8.1 (block table = logical block -> physical block).
+ *
+ * Conventions for every function:
+ *  - The return value is a pkv_status; nothing else reports errors.
+ *  - Device memory is allocated by the caller (e.g. PyTorch) and owned by the
+ *    caller; the library allocates no device memory and keeps no pointer
+ *    after a call returns.  Host functions are pure and thread-safe.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Device work is queued on it asynchronously unless stated.
+ *  - Sizes are element counts unless the name ends in _bytes.
+ *  - The fast path supports bf16 q/K/V/out, page_size 16, head_dim 64 or 128,
+ *    1 <= G <= 16, pools 16-byte aligned with head_dim contiguous and token,
+ *    head and page strides that are multiples of 8 elements.  Anything else
+ *    returns PKV_ERR_UNSUPPORTED.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+/* Status codes. */
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID = -1,      /* an argument is malformed (null pointer, negative size, bad table) */
+    PKV_ERR_UNSUPPORTED = -2,  /* well formed but outside the fast path (see above) */
+    PKV_ERR_CAPACITY = -3,     /* a caller buffer (items, workspace, staging) is too small */
+    PKV_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
+    PKV_ERR_TIMEOUT = -5,      /* a device-side wait gave up (reported by pkv_workspace_status) */
+    PKV_ERR_DEVICE_INPUT = -6  /* the kernel met an out-of-range seq_len, page id or work item
+                                  (reported by pkv_workspace_status); it clamped and went on */
+} pkv_status;
+
+/* Execution paths [PKV, Methodology 2 "Calibrated adaptive policy"]. */
+typedef enum {
+    PKV_NO_SPLIT = 0,   /* one block per (row, KV head) covers the whole row; no merge */
+    PKV_SPLIT_S = 1,    /* rectangular grid (row, KV head, split); empty splits write the neutral state */
+    PKV_WORK_QUEUE = 2  /* 1D grid over the compact queue of non-empty (row, KV head, chunk) items */
+} pkv_mode;
+
+/* pkv_plan.flags / pkv_policy_rule.flags */
+#define PKV_FLAG_SEPARATE_MERGE 1 /* merge partial states in a second kernel instead of in the
+                                     last block that finishes a (row, KV head) */
+
+/* Problem shape and pool layout.  Pool element (page, kv_head, slot, d) of
+ * k_pool / v_pool lives at  page*kv_stride_page + kv_head*kv_stride_head +
+ * slot*kv_stride_token + d  (elements).  The default "HND" pool
+ * [num_pool_pages][H_kv][page_size][head_dim] has strides
+ * (H_kv*P*D, P*D, D); an "NHD" pool [pages][P][H_kv][D] has (P*H_kv*D, D, H_kv*D). */
+typedef struct {
+    int32_t B;                  /* rows (sequences) in the batch, >= 0 */
+    int32_t H_q;                /* query heads, a multiple of H_kv */
+    int32_t H_kv;               /* KV heads */
+    int32_t head_dim;           /* D */
+    int32_t page_size;          /* P, tokens per page */
+    int32_t max_pages_per_seq;  /* columns of block_table; every N_i <= max_pages_per_seq * P */
+    int32_t num_pool_pages;     /* pages in each pool; block-table entries lie in [0, num_pool_pages) */
+    int32_t reserved;           /* 0 */
+    int64_t kv_stride_page;
+    int64_t kv_stride_head;
+    int64_t kv_stride_token;
+} pkv_shape;
+
+/* The chosen execution plan (16 bytes, compared bit-exactly by the tests).
+ *   NO_SPLIT:    {0, 1, 0, flags}
+ *   SPLIT_S:     {1, S', C, flags}  C = ceil(pages_max / S), S' = ceil(pages_max / C)
+ *   WORK_QUEUE:  {2, S', C, flags}  C from the rule,        S' = ceil(pages_max / C)
+ * where pages_max = ceil(N_max / P).  S' is the most chunks any row needs. */
+typedef struct {
+    int32_t mode;
+    int32_t num_splits;
+    int32_t chunk_pages;
+    int32_t flags;
+} pkv_plan;
+
+/* One work item: tokens [tok_begin, tok_end) of (row, kv_head).  tok_begin is
+ * a multiple of the page size; an item with tok_begin == tok_end exists only
+ * for a row with N_i = 0 (it writes that row's zero output). */
+typedef struct {
+    int32_t row;
+    int32_t kv_head;
+    int32_t tok_begin;
+    int32_t tok_end;
+} pkv_work_item;
+
+/* One row of a policy table: batches with b_lo <= B < b_hi and
+ * nmax_lo <= N_max < nmax_hi take this rule's plan.  The first matching rule
+ * wins; no match means NO_SPLIT.  Use INT32_MAX for an open upper end. */
+typedef struct {
+    int32_t b_lo, b_hi;
+    int32_t nmax_lo, nmax_hi;
+    int32_t mode;         /* pkv_mode */
+    int32_t num_splits;   /* SPLIT_S: requested S >= 1 */
+    int32_t chunk_pages;  /* WORK_QUEUE: chunk size C >= 1 in pages */
+    int32_t flags;        /* PKV_FLAG_* */
+} pkv_policy_rule;
+
+/* Scheduler workload counters of one step [PKV, Key contributions:
+ * "scheduler-induced workload counters"; Results: launch fan-out and
+ * merge-state traffic].  All in units of the name (bytes or counts). */
+typedef struct {
+    int64_t launches;           /* kernel launches of the step */
+    int64_t work_items;         /* blocks of the attention kernel */
+    int64_t empty_items;        /* blocks that only write a neutral state or a zero row */
+    int64_t merge_state_bytes;  /* partial states written and read back: 2*slots*G*(D+2)*4
+                                   over every (row, KV head) with more than one slot */
+    int64_t kv_bytes;           /* K+V of the valid tokens: sum_i N_i * H_kv * 2 * D * 2 */
+    int64_t kv_bytes_streamed;  /* K+V of whole pages: sum_i ceil(N_i/P) * P * H_kv * 2 * D * 2 */
+    int64_t q_bytes;            /* B * H_q * D * 2 */
+    int64_t out_bytes;          /* B * H_q * D * 2 */
+    int64_t queue_bytes;        /* WORK_QUEUE: 16 * items + 4 * (B*H_kv + 1) sent to the device */
+    int64_t bucket_launches;    /* exact-length bucketing: 2 * distinct non-zero N_i */
+} pkv_counters;
+
+/* Library version string (static storage). */
+PKV_API const char *pkv_version(void);
+
+/* Human-readable name of a status code (static storage). */
+PKV_API const char *pkv_status_string(int status);
+
+/* Copy the built-in policy table (calibrated on B200 with seed 20260622) into
+ * rules[0 .. capacity).  *n_rules receives its length; PKV_ERR_CAPACITY if
+ * capacity is smaller (rules may then be NULL to query the length). */
+PKV_API int pkv_default_policy(pkv_policy_rule *rules, int32_t capacity, int32_t *n_rules);
+
+/* Pick the plan for a batch from (B, N_max) [PKV, Methodology 2 "Calibrated
+ * adaptive policy": B = 1 long context -> split with length buckets, B >= 8
+ * -> compact work queue, otherwise the single kernel; Results, B = 4 boundary].
+ * seq_lens_host: host int32[shape->B]; rules: n_rules rows, or NULL for the
+ * built-in table.  Pure host function; writes *plan (see pkv_plan).
+ * PKV_ERR_INVALID on a negative length, a rule with an unknown mode,
+ * num_splits < 1 in a SPLIT_S rule or chunk_pages < 1 in a WORK_QUEUE rule. */
+PKV_API int pkv_select_policy(const int32_t *seq_lens_host, const pkv_shape *shape,
+                              const pkv_policy_rule *rules, int32_t n_rules, pkv_plan *plan);
+
+/* Number of items pkv_build_work_queue emits:
+ *   H_kv * sum_i max(1, ceil(ceil(N_i / P) / chunk_pages)). */
+PKV_API int pkv_work_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape,
+                                int32_t chunk_pages, int32_t *n_items);
+
+/* Build the compact work queue [PKV, Methodology 1 "Compact work queue" and
+ * "Row-local bounds"]: one item per (row, KV head, chunk) whose token range is
+ * non-empty, in lexicographic (row, kv_head, chunk) order; chunk c covers
+ * tokens [c*C*P, min((c+1)*C*P, N_i)) with C = chunk_pages, so bounds follow
+ * each row's real length.  indptr (host int32[B*H_kv + 1]) receives the first
+ * item of each (row, kv_head) pair, indptr[B*H_kv] = *n_items.  items: host
+ * array of `capacity` entries; PKV_ERR_CAPACITY (with *n_items set to the
+ * size needed) if it is too small.  Pure host function. */
+PKV_API int pkv_build_work_queue(const int32_t *seq_lens_host, const pkv_shape *shape,
+                                 int32_t chunk_pages, pkv_work_item *items, int32_t capacity,
+                                 int32_t *indptr, int32_t *n_items);
+
+/* Closed-form workload counters of `plan` on this batch (host, pure). */
+PKV_API int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape,
+                              const pkv_plan *plan, pkv_counters *counters);
+
+/* Device workspace that pkv_paged_decode needs for this shape and plan
+ * (n_items: WORK_QUEUE queue length, ignored otherwise).  The workspace holds
+ * a device error word, one completion counter per (row, KV head) pair and the
+ * fp32 partial states (m, l, acc) of every split. */
+PKV_API int pkv_workspace_bytes(const pkv_shape *shape, const pkv_plan *plan, int32_t n_items,
+                                size_t *bytes);
+
+/* Zero a workspace on `stream` (queued memset).  A workspace must be zeroed
+ * once before its first use; every successful decode leaves it zeroed again,
+ * so later calls need no memset.  Also clears a recorded device error. */
+PKV_API int pkv_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronize `stream`, then read the workspace's device error word:
+ * PKV_OK, PKV_ERR_TIMEOUT or PKV_ERR_DEVICE_INPUT (also stored in
+ * *device_error when not NULL, as the raw bit mask: 1 timeout, 2 seq_len out
+ * of range, 4 page id out of range, 8 malformed work item). */
+PKV_API int pkv_workspace_status(const void *workspace, void *stream, int32_t *device_error);
+
+/* One decode step on the GPU.  All pointers but `shape`, `plan` are device
+ * pointers:
+ *   q            bf16 [B][H_q][D], contiguous
+ *   k_pool       bf16 pool, layout from `shape` (never repacked, only read)
+ *   v_pool       bf16 pool, same layout as k_pool
+ *   block_table  int32 [B][max_pages_per_seq]; entries past a row's last page are never read
+ *   seq_lens     int32 [B]; N_i in [0, max_pages_per_seq * P]
+ *   out          bf16 [B][H_q][D], contiguous; fully overwritten (rows with N_i = 0 get zeros)
+ *   items,indptr WORK_QUEUE only: the queue from pkv_build_work_queue, copied to the device
+ *   workspace    >= pkv_workspace_bytes(), zeroed once (pkv_workspace_init)
+ * page_size must equal shape->page_size; scale multiplies the logits.
+ * The split kernel streams whole K/V pages through the block table into
+ * shared memory (TMA, multi-stage), computes each split's partial softmax
+ * state on the tensor cores, and the exact merge of the splits runs in the
+ * last block to finish each (row, KV head) [PKV, Methodology 1 "Sequence
+ * splitting": "a separate merge kernel combines the states exactly"] or,
+ * with PKV_FLAG_SEPARATE_MERGE, in a second kernel.  Results are
+ * deterministic: the merge order is fixed (ascending split index).
+ * Asynchronous on `stream`; a workspace must not be shared by calls that may
+ * run at the same time.  Returns PKV_ERR_CUDA if a launch fails; errors the
+ * kernels detect on device data are read back with pkv_workspace_status. */
+PKV_API int pkv_paged_decode(const void *q, const void *k_pool, const void *v_pool,
+                             const int32_t *block_table, const int32_t *seq_lens, int32_t page_size,
+                             float scale, void *out, const pkv_shape *shape, const pkv_plan *plan,
+                             const pkv_work_item *items, const int32_t *indptr, int32_t n_items,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Sizes of the caller buffers pkv_decode_host needs for this batch and
+ * policy table (rules NULL = built-in): *device_bytes of device memory and
+ * *host_bytes of host staging memory (page-locked memory makes the copies
+ * asynchronous; pageable memory also works). */
+PKV_API int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape *shape,
+                                  const pkv_policy_rule *rules, int32_t n_rules,
+                                  size_t *device_bytes, size_t *host_bytes);
+
+/* One synchronous decode step from host buffers, the way a serving loop
+ * calls it [PKV, Methodology 3 "Evaluation protocol": synchronized wall time
+ * including host planning]: pick the plan (pkv_select_policy), build the
+ * queue into host_staging (pkv_build_work_queue), copy q, block_table,
+ * seq_lens and the queue host->device into device_buffer, zero the
+ * completion counters, run pkv_paged_decode, copy out device->host and
+ * synchronize `stream`.  q_host, block_table_host, seq_lens_host, out_host
+ * are host pointers with the layouts of pkv_paged_decode; k_pool / v_pool
+ * are device pools (the cache stays resident on the device).  The plan used
+ * is written to *plan_out when not NULL.  Returns the device error status
+ * like pkv_workspace_status when the kernels ran. */
+PKV_API int pkv_decode_host(const void *q_host, const int32_t *block_table_host,
+                            const int32_t *seq_lens_host, void *out_host, const void *k_pool,
+                            const void *v_pool, float scale, const pkv_shape *shape,
+                            const pkv_policy_rule *rules, int32_t n_rules, void *device_buffer,
+                            size_t device_buffer_bytes, void *host_staging,
+                            size_t host_staging_bytes, void *stream, pkv_plan *plan_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

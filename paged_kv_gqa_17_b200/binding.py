@@ -1,0 +1,335 @@
+"""ctypes binding of libpkv.so (include/pkv.h): argument marshalling only.
+
+Every step of the decode path (policy, queue, kernels, merge) runs inside the
+C-ABI library; this module converts torch tensors to raw pointers, allocates
+caller-owned buffers with torch and passes torch's current CUDA stream.  If
+the library is missing or cannot be loaded, every call raises PkvError.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+import os
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpkv.so")
+
+NO_SPLIT, SPLIT_S, WORK_QUEUE = 0, 1, 2
+FLAG_SEPARATE_MERGE = 1
+INT32_MAX = 2**31 - 1
+_MODE_NAMES = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE}
+
+c_i32, c_i64, c_p, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = _lib.pkv_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{what}: {name} ({status})" if what else f"{name} ({status})")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", c_i32), ("H_q", c_i32), ("H_kv", c_i32), ("head_dim", c_i32), ("page_size", c_i32),
+                ("max_pages_per_seq", c_i32), ("num_pool_pages", c_i32), ("reserved", c_i32),
+                ("kv_stride_page", c_i64), ("kv_stride_head", c_i64), ("kv_stride_token", c_i64)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("mode", c_i32), ("num_splits", c_i32), ("chunk_pages", c_i32), ("flags", c_i32)]
+
+    def tuple(self):
+        return (self.mode, self.num_splits, self.chunk_pages, self.flags)
+
+    def __repr__(self):
+        return f"Plan{self.tuple()}"
+
+
+class WorkItem(ctypes.Structure):
+    _fields_ = [("row", c_i32), ("kv_head", c_i32), ("tok_begin", c_i32), ("tok_end", c_i32)]
+
+
+class Rule(ctypes.Structure):
+    _fields_ = [("b_lo", c_i32), ("b_hi", c_i32), ("nmax_lo", c_i32), ("nmax_hi", c_i32), ("mode", c_i32),
+                ("num_splits", c_i32), ("chunk_pages", c_i32), ("flags", c_i32)]
+
+    def tuple(self):
+        return tuple(getattr(self, f) for f, _ in self._fields_)
+
+
+class Counters(ctypes.Structure):
+    _fields_ = [(n, c_i64) for n in ("launches", "work_items", "empty_items", "merge_state_bytes", "kv_bytes",
+                                     "kv_bytes_streamed", "q_bytes", "out_bytes", "queue_bytes",
+                                     "bucket_launches")]
+
+    def as_dict(self):
+        return {f: int(getattr(self, f)) for f, _ in self._fields_}
+
+
+_lib = None
+
+# (name, restype, argtypes) of every function include/pkv.h declares
+SIGNATURES = [
+    ("pkv_version", ctypes.c_char_p, []),
+    ("pkv_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("pkv_default_policy", ctypes.c_int, [c_p, c_i32, c_p]),
+    ("pkv_select_policy", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_p]),
+    ("pkv_work_queue_size", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
+    ("pkv_build_work_queue", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p]),
+    ("pkv_plan_counters", ctypes.c_int, [c_p, c_p, c_p, c_p]),
+    ("pkv_workspace_bytes", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
+    ("pkv_workspace_init", ctypes.c_int, [c_p, c_sz, c_p]),
+    ("pkv_workspace_status", ctypes.c_int, [c_p, c_p, c_p]),
+    ("pkv_paged_decode", ctypes.c_int,
+     [c_p, c_p, c_p, c_p, c_p, c_i32, ctypes.c_float, c_p, c_p, c_p, c_p, c_p, c_i32, c_p, c_sz, c_p]),
+    ("pkv_decode_host_bytes", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_p, c_p]),
+    ("pkv_decode_host", ctypes.c_int,
+     [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p]),
+]
+
+
+def lib(path: Optional[str] = None):
+    """Load libpkv.so (built by paged_kv_gqa_17_b200.build); raise if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise PkvError(-4, f"{p} is missing; build it with `python -m paged_kv_gqa_17_b200.build`")
+    handle = ctypes.CDLL(p)
+    for name, res, args in SIGNATURES:
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = handle
+    return handle
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise PkvError(rc, what)
+
+
+def _ref(x):
+    return ctypes.byref(x) if x is not None else None
+
+
+def _lens_array(seq_lens) -> ctypes.Array:
+    if isinstance(seq_lens, torch.Tensor):
+        seq_lens = seq_lens.detach().cpu().tolist()
+    vals = [int(v) for v in seq_lens]
+    return (c_i32 * max(1, len(vals)))(*vals), len(vals)
+
+
+def make_shape(B: int, H_q: int, H_kv: int, head_dim: int, page_size: int, max_pages: int, num_pool_pages: int,
+               layout: str = "HND") -> Shape:
+    P, D = page_size, head_dim
+    if layout == "HND":
+        strides = (H_kv * P * D, P * D, D)
+    elif layout == "NHD":
+        strides = (P * H_kv * D, D, H_kv * D)
+    else:
+        raise ValueError(layout)
+    return Shape(B, H_q, H_kv, D, P, max_pages, num_pool_pages, 0, *strides)
+
+
+def shape_of(q: torch.Tensor, k_pool: torch.Tensor, block_table: torch.Tensor, layout: str = "HND") -> Shape:
+    """Shape of a decode step from q [B][H_q][D], a pool and block_table [B][max_pages]."""
+    B, H_q, D = (int(x) for x in q.shape)
+    if layout == "HND":
+        pages, H_kv, P, _ = (int(x) for x in k_pool.shape)
+    else:
+        pages, P, H_kv, _ = (int(x) for x in k_pool.shape)
+    return make_shape(B, H_q, H_kv, D, P, int(block_table.shape[1]), pages, layout)
+
+
+def rules_array(rules: Optional[Sequence]) -> tuple:
+    """(ctypes array or None, count) from Rule structs, tuples or dicts."""
+    if rules is None:
+        return None, 0
+    out = []
+    for r in rules:
+        if isinstance(r, Rule):
+            out.append(r)
+        elif isinstance(r, dict):
+            mode = _MODE_NAMES[r["mode"]] if isinstance(r["mode"], str) else int(r["mode"])
+            out.append(Rule(int(r["b_lo"]), int(r.get("b_hi", INT32_MAX)), int(r["nmax_lo"]),
+                            int(r.get("nmax_hi", INT32_MAX)), mode, int(r.get("num_splits", 1)),
+                            int(r.get("chunk_pages", 0)), int(r.get("flags", 0))))
+        else:
+            out.append(Rule(*[int(v) for v in r]))
+    return (Rule * max(1, len(out)))(*out), len(out)
+
+
+def load_rules(path: str) -> List[Rule]:
+    """Read a policy table JSON ({"rules": [...]}) into Rule structs."""
+    with open(path) as f:
+        doc = json.load(f)
+    arr, n = rules_array(doc["rules"])
+    return [arr[i] for i in range(n)]
+
+
+def default_rules() -> List[Rule]:
+    L = lib()
+    n = c_i32(0)
+    L.pkv_default_policy(None, 0, ctypes.byref(n))
+    arr = (Rule * max(1, n.value))()
+    _check(L.pkv_default_policy(arr, n.value, ctypes.byref(n)), "pkv_default_policy")
+    return [arr[i] for i in range(n.value)]
+
+
+def select_policy(seq_lens_host, shape: Shape, rules=None) -> Plan:
+    L = lib()
+    lens, _ = _lens_array(seq_lens_host)
+    arr, n = rules_array(rules)
+    plan = Plan()
+    _check(L.pkv_select_policy(lens, ctypes.byref(shape), arr, n, ctypes.byref(plan)), "pkv_select_policy")
+    return plan
+
+
+def build_work_queue(seq_lens_host, shape: Shape, chunk_pages: int):
+    """-> (items int32 tensor [n][4] on the CPU, indptr int32 tensor [B*H_kv + 1])."""
+    L = lib()
+    lens, _ = _lens_array(seq_lens_host)
+    n = c_i32(0)
+    _check(L.pkv_work_queue_size(lens, ctypes.byref(shape), chunk_pages, ctypes.byref(n)), "pkv_work_queue_size")
+    items = torch.zeros((max(1, n.value), 4), dtype=torch.int32)
+    indptr = torch.zeros(shape.B * shape.H_kv + 1, dtype=torch.int32)
+    _check(L.pkv_build_work_queue(lens, ctypes.byref(shape), chunk_pages, items.data_ptr(), n.value,
+                                  indptr.data_ptr(), ctypes.byref(n)), "pkv_build_work_queue")
+    return items[:n.value], indptr
+
+
+def plan_counters(seq_lens_host, shape: Shape, plan: Plan) -> dict:
+    L = lib()
+    lens, _ = _lens_array(seq_lens_host)
+    c = Counters()
+    _check(L.pkv_plan_counters(lens, ctypes.byref(shape), ctypes.byref(plan), ctypes.byref(c)), "pkv_plan_counters")
+    return c.as_dict()
+
+
+def workspace_bytes(shape: Shape, plan: Plan, n_items: int = 0) -> int:
+    L = lib()
+    b = c_sz(0)
+    _check(L.pkv_workspace_bytes(ctypes.byref(shape), ctypes.byref(plan), n_items, ctypes.byref(b)),
+           "pkv_workspace_bytes")
+    return int(b.value)
+
+
+def _stream_ptr(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+@dataclass
+class DecodePlan:
+    """Everything a decode step needs besides the tensors: the plan, the queue
+    on the device (WORK_QUEUE) and a zeroed workspace.  Reusable for every
+    step with the same sequence lengths and shape."""
+
+    shape: Shape
+    plan: Plan
+    items: Optional[torch.Tensor]
+    indptr: Optional[torch.Tensor]
+    n_items: int
+    workspace: torch.Tensor
+    counters: dict
+
+
+def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[Plan] = None) -> DecodePlan:
+    """Host planning for one batch: policy (unless `plan` is given), queue, workspace."""
+    if plan is None:
+        plan = select_policy(seq_lens_host, shape, rules)
+    items = indptr = None
+    n_items = 0
+    if plan.mode == WORK_QUEUE:
+        items_h, indptr_h = build_work_queue(seq_lens_host, shape, plan.chunk_pages)
+        n_items = int(items_h.shape[0])
+        items = items_h.to(device)
+        indptr = indptr_h.to(device)
+    ws = torch.zeros(workspace_bytes(shape, plan, n_items), dtype=torch.uint8, device=device)
+    return DecodePlan(shape, plan, items, indptr, n_items, ws, plan_counters(seq_lens_host, shape, plan))
+
+
+def paged_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, block_table: torch.Tensor,
+                 seq_lens: torch.Tensor, page_size: int, scale: float, *, plan: Optional[DecodePlan] = None,
+                 seq_lens_host=None, layout: str = "HND", rules=None, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """out = softmax(scale * q K^T) V per (row, query head), read through the block table.
+
+    q bf16 [B][H_q][D]; pools bf16 (layout "HND" [pages][H_kv][P][D] or "NHD"
+    [pages][P][H_kv][D]); block_table int32 [B][max_pages]; seq_lens int32 [B],
+    all on one CUDA device.  Without `plan`, the policy and queue are built from
+    `seq_lens_host` (or a host copy of seq_lens).
+    """
+    L = lib()
+    if plan is None:
+        shape = shape_of(q, k_pool, block_table, layout)
+        host = seq_lens_host if seq_lens_host is not None else seq_lens.detach().cpu()
+        plan = plan_decode(host, shape, q.device, rules)
+    shape = plan.shape
+    if out is None:
+        out = torch.empty_like(q)
+    rc = L.pkv_paged_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
+                            seq_lens.data_ptr(), page_size, float(scale), out.data_ptr(), ctypes.byref(shape),
+                            ctypes.byref(plan.plan), plan.items.data_ptr() if plan.items is not None else None,
+                            plan.indptr.data_ptr() if plan.indptr is not None else None, plan.n_items,
+                            plan.workspace.data_ptr(), plan.workspace.numel(), _stream_ptr(stream))
+    _check(rc, "pkv_paged_decode")
+    return out
+
+
+def workspace_status(plan: DecodePlan, stream=None) -> int:
+    """Synchronize and return the raw device error mask of a plan's workspace (0 = clean)."""
+    L = lib()
+    err = c_i32(0)
+    L.pkv_workspace_status(plan.workspace.data_ptr(), _stream_ptr(stream), ctypes.byref(err))
+    return int(err.value)
+
+
+class HostDecoder:
+    """Caller-owned buffers for pkv_decode_host, grown on demand: one device
+    buffer (torch) and one page-locked host staging buffer."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.dev = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self.host = torch.empty(0, dtype=torch.uint8).pin_memory()
+
+    def ensure(self, seq_lens_host, shape: Shape, rules=None):
+        L = lib()
+        lens, _ = _lens_array(seq_lens_host)
+        arr, n = rules_array(rules)
+        db, hb = c_sz(0), c_sz(0)
+        _check(L.pkv_decode_host_bytes(lens, ctypes.byref(shape), arr, n, ctypes.byref(db), ctypes.byref(hb)),
+               "pkv_decode_host_bytes")
+        if self.dev.numel() < db.value:
+            self.dev = torch.zeros(db.value, dtype=torch.uint8, device=self.device)
+        if self.host.numel() < hb.value:
+            self.host = torch.zeros(hb.value, dtype=torch.uint8).pin_memory()
+
+    def __call__(self, q_host: torch.Tensor, block_table_host: torch.Tensor, seq_lens_host: torch.Tensor,
+                 out_host: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, scale: float, shape: Shape,
+                 rules=None, stream=None) -> Plan:
+        L = lib()
+        arr, n = rules_array(rules)
+        plan = Plan()
+        rc = L.pkv_decode_host(q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(),
+                               out_host.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), float(scale),
+                               ctypes.byref(shape), arr, n, self.dev.data_ptr(), self.dev.numel(),
+                               self.host.data_ptr(), self.host.numel(), _stream_ptr(stream), ctypes.byref(plan))
+        _check(rc, "pkv_decode_host")
+        return plan
+
+
+def decode_host(*args, **kwargs):
+    """One-shot pkv_decode_host with freshly allocated buffers (see HostDecoder)."""
+    q_host, bt_host, lens_host, out_host, k_pool, v_pool, scale, shape = args[:8]
+    dec = HostDecoder(k_pool.device)
+    dec.ensure(lens_host, shape, kwargs.get("rules"))
+    return dec(*args, **kwargs)

@@ -1,0 +1,1058 @@
+// Paged GQA decode attention for B200 (sm_100a): the split kernel, the merge
+// and the decode entry points of the C ABI (include/pkv.h).
+//
+// Method: "PersistentKV: Page-Aware Decode Scheduling for Long-Context LLM
+// Serving on Commodity GPUs" (gist.science explainer), Technical summary >
+// Methodology > 1 "Native block-table decode engine":
+//   - GQA: the G = H_q / H_kv query heads of one KV head are handled by one
+//     block, so every K/V byte is read from HBM once;
+//   - layout: K/V pages are read through the block table in place, never
+//     repacked into a contiguous tensor;
+//   - sequence splitting: a row's token range is cut into disjoint chunks;
+//     each chunk yields a partial online-softmax state (running max m,
+//     denominator l, fp32 accumulator) and a merge combines them exactly;
+//   - row-local bounds: chunk ranges come from each row's real length; an
+//     empty chunk writes the neutral state (m = -inf, l = 0, acc = 0) and
+//     reads nothing;
+//   - compact work queue: a 1D grid over the non-empty (row, KV head, chunk)
+//     items only.
+//
+// B200 design (the pages' kernels were written for an RTX 3060):
+//   - one producer warp streams whole 16-token pages of K and V for one KV
+//     head (4 KiB each at D = 128) with TMA tensor copies into an NST-stage
+//     shared-memory ring, completion tracked by mbarriers; the copies use the
+//     128-byte swizzle so the tensor-core fragment loads below are free of
+//     bank conflicts;
+//   - NW consumer warps take pages round robin; per page a warp computes
+//     S^T = K Q^T (16 tokens x 8 heads, mma.sync m16n8k16, bf16 in, fp32
+//     accumulate), the online-softmax update with warp shuffles, transposes
+//     P in registers (movmatrix) and accumulates O^T += V^T P^T on the tensor
+//     cores.  Decode does G flops per K/V byte, far below any tensor-core
+//     ridge: the kernel is HBM-bound and the warp-level MMAs keep the math
+//     off the critical path for every G <= 16 at the same cost per page;
+//   - the warps' states are combined in shared memory; a chunk that covers
+//     the whole (row, KV head) writes the bf16 output directly, otherwise it
+//     writes its partial state and the last block to finish that (row, KV
+//     head) (an atomic ticket) merges all states in ascending chunk order,
+//     so the result is deterministic and no second launch is needed.
+//   - every device-side wait is bounded (2 s); on a timeout the kernel
+//     records an error bit in the workspace and gives up instead of hanging.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "pkv_internal.h"
+
+namespace pkv {
+
+constexpr int kBoxD = 64;                   // head-dim elements per TMA box row (128 bytes)
+constexpr int kBoxBytes = kBoxD * kPage * 2; // one [16 tokens][64 d] bf16 box = 2 KiB
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kWaitLimitIters = 1u << 30;
+
+struct __align__(64) Params {
+    CUtensorMap tm_k;  // pool views [pages][H_kv][P][D] -> boxes of [1][1][16][64]
+    CUtensorMap tm_v;
+    const __nv_bfloat16 *q;
+    __nv_bfloat16 *out;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    const int4 *items;
+    const int32_t *indptr;
+    float *ws_m;
+    float *ws_l;
+    float *ws_acc;
+    uint32_t *ws_counters;
+    uint32_t *ws_error;
+    float scale_log2;  // scale * log2(e): logits are kept in the log2 domain
+    int32_t B, H_q, H_kv, G, max_pages, num_pool_pages;
+    int32_t mode, num_splits, chunk_pages, separate_merge;
+    int32_t n_items;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs (or
+// kWaitLimitIters polls) with the timeout bit set in the error word.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1; i < kWaitLimitIters; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs)
+            break;
+    }
+    atomicOr(err, kErrTimeout);
+    return false;
+}
+
+__device__ __forceinline__ uint64_t evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// TMA tiled copy of one [1][1][16][64] box of a pool view into shared memory.
+__device__ __forceinline__ void tma_load_box(uint32_t dst, const CUtensorMap *tm, uint32_t bar, int d0, int head,
+                                             int page, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(d0), "r"(0), "r"(head), "r"(page), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *tm)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                              uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D = A * B + D, m16n8k16, bf16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 b16 matrix held one row pair per lane.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// 2^x on the SFU (ex2.approx: relative error ~2^-22); 2^-inf = +0.
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16 *dst, float4 v)
+{
+    uint2 u;
+    u.x = pack_bf16(v.x, v.y);
+    u.y = pack_bf16(v.z, v.w);
+    *reinterpret_cast<uint2 *>(dst) = u;
+}
+
+__device__ __forceinline__ float4 fma4(float4 a, float s, float4 b)  // a * s + b
+{
+    return make_float4(fmaf(a.x, s, b.x), fmaf(a.y, s, b.y), fmaf(a.z, s, b.z), fmaf(a.w, s, b.w));
+}
+
+__device__ __forceinline__ float4 scale4(float4 a, float s)
+{
+    return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel configuration
+
+template <int D, int NT, int NW, int NST>
+struct Cfg {
+    static_assert(D == 64 || D == 128, "head_dim");
+    static constexpr int kHalves = D / kBoxD;
+    static constexpr int kStageBytes = D * kPage * 2;  // one K (or V) page of one KV head
+    static constexpr int kThreads = (NW + 1) * 32;     // NW consumer warps + 1 producer warp
+    static constexpr int kGP = 8 * NT;                 // query heads per block, padded to the MMA's n = 8
+    static constexpr int kOStride = D + 4;             // floats per (warp, head) row in the combine buffer
+    static constexpr int kCombineBytes = NW * kGP * (kOStride + 2) * 4;
+    static constexpr int kRingBytes = 2 * NST * kStageBytes;
+    static constexpr int kBarOff = ((kRingBytes > kCombineBytes ? kRingBytes : kCombineBytes) + 63) / 64 * 64;
+    static constexpr int kMiscOff = kBarOff + 2 * NST * 8;
+    static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + slack to align the base to 1024
+};
+
+// Merge the nslots partial states of one (row, KV head) in ascending slot
+// order and write the bf16 output of its G query heads.
+template <int D>
+__device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslots, int tid, int nthreads)
+{
+    const int G = p.G;
+    constexpr int D4 = D / 4;
+    for (int e = tid; e < G * D4; e += nthreads) {
+        const int g = e / D4;
+        const int d4 = (e % D4) * 4;
+        float M = -INFINITY, L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < nslots; s0 += 8) {
+            float ms[8], ls[8];
+            float4 as[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                ms[u] = -INFINITY;
+                ls[u] = 0.f;
+                as[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s0 + u < nslots) {
+                    const int64_t idx = (int64_t)(slot0 + s0 + u) * G + g;
+                    ms[u] = __ldcg(p.ws_m + idx);
+                    ls[u] = __ldcg(p.ws_l + idx);
+                    as[u] = __ldcg(reinterpret_cast<const float4 *>(p.ws_acc + idx * D + d4));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (ms[u] == -INFINITY)
+                    continue;  // neutral state: weight 0
+                const float Mn = fmaxf(M, ms[u]);
+                const float a = exp2_approx(M - Mn);
+                const float b = exp2_approx(ms[u] - Mn);
+                L = fmaf(L, a, ls[u] * b);
+                O = fma4(O, a, scale4(as[u], b));
+                M = Mn;
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+    }
+}
+
+// One block = one work item (row, KV head, token range) for all G query heads.
+template <int D, int NT, int NW, int NST>
+__global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_constant__ Params p)
+{
+    using C = Cfg<D, NT, NW, NST>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t k_ring = sbase;
+    const uint32_t v_ring = sbase + NST * C::kStageBytes;
+    const uint32_t bar_full = sbase + C::kBarOff;
+    const uint32_t bar_empty = bar_full + NST * 8;
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + C::kMiscOff);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t row_cap = (int64_t)p.max_pages * kPage;
+
+    // ---- which (row, KV head, token range) this block owns ----
+    int row, h, tb, te, slot0 = 0, nslots = 1, my_slot = 0;
+    if (p.mode == PKV_WORK_QUEUE) {
+        const int4 it = __ldg(p.items + blockIdx.x);
+        row = it.x;
+        h = it.y;
+        tb = it.z;
+        te = it.w;
+        bool ok = row >= 0 && row < p.B && h >= 0 && h < p.H_kv && tb >= 0 && tb <= te && te <= row_cap &&
+                  (tb % kPage) == 0;
+        if (ok) {
+            const int pair = row * p.H_kv + h;
+            slot0 = __ldg(p.indptr + pair);
+            nslots = __ldg(p.indptr + pair + 1) - slot0;
+            my_slot = blockIdx.x;
+            ok = nslots >= 1 && slot0 >= 0 && my_slot >= slot0 && my_slot < slot0 + nslots &&
+                 slot0 + nslots <= p.n_items;
+        }
+        if (!ok) {
+            if (tid == 0)
+                atomicOr(p.ws_error, kErrItem);
+            return;
+        }
+    } else {
+        const int S = p.mode == PKV_SPLIT_S ? p.num_splits : 1;
+        const int pair = blockIdx.x / S;
+        const int c = blockIdx.x % S;
+        row = pair / p.H_kv;
+        h = pair % p.H_kv;
+        int N = __ldg(p.seq_lens + row);
+        if (N < 0 || N > row_cap) {
+            if (tid == 0)
+                atomicOr(p.ws_error, kErrSeqLen);
+            N = N < 0 ? 0 : (int)row_cap;
+        }
+        if (p.mode == PKV_SPLIT_S) {
+            const int64_t span = (int64_t)p.chunk_pages * kPage;
+            if (c == 0 && tid == 0 && (int64_t)S * span < N)
+                atomicOr(p.ws_error, kErrItem);  // the plan's S * C pages do not cover this row
+            const int64_t b = (int64_t)c * span;
+            tb = (int)(b < N ? b : N);
+            te = (int)(b < N ? (b + span < N ? b + span : N) : N);  // empty chunk: tb == te
+            nslots = S;
+            slot0 = pair * S;
+            my_slot = slot0 + c;
+        } else {
+            tb = 0;
+            te = N;
+        }
+    }
+    const int pair = row * p.H_kv + h;
+    const int pg0 = tb / kPage;
+    const int npages = te > tb ? (te + kPage - 1) / kPage - pg0 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+    }
+    __syncthreads();
+
+    // Per-warp softmax state for the heads g = 8*nt + 2*(lane%4) + j.
+    float m_run[NT][2], l_run[NT][2];
+    float o[D / 16][NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        m_run[nt][0] = m_run[nt][1] = -INFINITY;
+        l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+            o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    }
+    const int r = lane >> 2;  // fragment row group
+    const int c4 = lane & 3;  // fragment column pair
+
+    if (warp == NW) {
+        // ================= producer: block table -> TMA page copies =================
+        const int32_t *bt = p.block_table + (int64_t)row * p.max_pages + pg0;
+        const uint64_t policy = evict_first_policy();
+        int e_next = lane < npages ? __ldg(bt + lane) : 0;
+        bool ok = true;
+        for (int base = 0; base < npages && ok; base += 32) {
+            int e = e_next;
+            e_next = base + 32 + lane < npages ? __ldg(bt + base + 32 + lane) : 0;
+            const bool bad = base + lane < npages && (e < 0 || e >= p.num_pool_pages);
+            if (__any_sync(0xffffffffu, bad) && lane == 0)
+                atomicOr(p.ws_error, kErrPageId);
+            if (bad)
+                e = 0;  // read a real page instead; the error bit reports the bad entry
+            const int cnt = npages - base < 32 ? npages - base : 32;
+            for (int j = 0; j < cnt; ++j) {
+                const int phys = __shfl_sync(0xffffffffu, e, j);
+                const int pidx = base + j;
+                const int s = pidx % NST;
+                const int k = pidx / NST;
+                if (lane == 0) {
+                    if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, p.ws_error))
+                        ok = false;
+                    if (ok) {
+                        const uint32_t fb = bar_full + 8 * s;
+                        mbar_expect_tx(fb, 2 * C::kStageBytes);
+#pragma unroll
+                        for (int hf = 0; hf < C::kHalves; ++hf) {
+                            tma_load_box(k_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_k, fb, hf * kBoxD, h,
+                                         phys, policy);
+                            tma_load_box(v_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_v, fb, hf * kBoxD, h,
+                                         phys, policy);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok)
+                    break;
+            }
+        }
+    } else {
+        // ================= consumers: tensor-core attention over pages =================
+        // Q as the MMA's B operand (k = head_dim, n = query head), loaded once.
+        uint32_t qf[D / 16][NT][2];
+        const __nv_bfloat16 *qb = p.q + ((int64_t)row * p.H_q + (int64_t)h * p.G) * D;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int g = nt * 8 + r;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t lo = 0, hi = 0;
+                if (g < p.G) {
+                    const uint32_t *src = reinterpret_cast<const uint32_t *>(qb + (int64_t)g * D + ks * 16 + 2 * c4);
+                    lo = __ldg(src);
+                    hi = __ldg(src + 4);
+                }
+                qf[ks][nt][0] = lo;
+                qf[ks][nt][1] = hi;
+            }
+        }
+        // ldmatrix lane roles: matrix mi = lane / 8, row ri = lane % 8 (= token % 8).
+        const int mi = lane >> 3;
+        const int ri = lane & 7;
+        const uint32_t k_off = (uint32_t)((8 * (mi & 1) + ri) * 128);   // K as A (rows = tokens)
+        const int k_hi = mi >> 1;
+        const uint32_t v_off = (uint32_t)((8 * (mi >> 1) + ri) * 128);  // V^T as A via .trans
+        const int v_hi = mi & 1;
+        const float sl2 = p.scale_log2;
+
+        for (int pidx = warp; pidx < npages; pidx += NW) {
+            const int s = pidx % NST;
+            const bool ready = mbar_wait(bar_full + 8 * s, (pidx / NST) & 1, p.ws_error);
+            if (!__all_sync(0xffffffffu, ready))
+                break;
+            const uint32_t ks_base = k_ring + s * C::kStageBytes;
+            const uint32_t vs_base = v_ring + s * C::kStageBytes;
+            const int tok0 = (pg0 + pidx) * kPage;
+            const int nvalid = te - tok0 < kPage ? te - tok0 : kPage;
+            if (nvalid < kPage) {
+                // Tail page: zero V rows past the row's end, so that stale or
+                // NaN slots cannot leak through P = 0 in the PV product.
+                uint8_t *vs = smem + (vs_base - sbase);
+                const int dead = kPage - nvalid;
+                for (int i = lane; i < dead * C::kHalves * 8; i += 32) {
+                    const int rr = i >> 3;
+                    const int hf = rr / dead;
+                    const int t = nvalid + rr % dead;
+                    *reinterpret_cast<uint4 *>(vs + hf * kBoxBytes + t * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+            // S^T[t][g] = K[t] . q[g]
+            float sacc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int chunk = (((ks & 3) << 1) + k_hi) ^ ri;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(ks_base + (ks >> 2) * kBoxBytes + k_off + (chunk << 4), a0, a1, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_bf16(sacc[nt], a0, a1, a2, a3, qf[ks][nt][0], qf[ks][nt][1]);
+            }
+            // Online softmax over this page (log2 domain), tokens past the end masked.
+            const bool lo_ok = r < nvalid;
+            const bool hi_ok = r + 8 < nvalid;
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float x0 = lo_ok ? sacc[nt][0] * sl2 : -INFINITY;
+                const float x1 = lo_ok ? sacc[nt][1] * sl2 : -INFINITY;
+                const float x2 = hi_ok ? sacc[nt][2] * sl2 : -INFINITY;
+                const float x3 = hi_ok ? sacc[nt][3] * sl2 : -INFINITY;
+                float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+                for (int sh = 4; sh < 32; sh <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
+                }
+                const float mn0 = fmaxf(m_run[nt][0], mx0);
+                const float mn1 = fmaxf(m_run[nt][1], mx1);
+                const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+                const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+                const float al0 = exp2_approx(m_run[nt][0] - mu0);
+                const float al1 = exp2_approx(m_run[nt][1] - mu1);
+                const float p0 = exp2_approx(x0 - mu0);
+                const float p1 = exp2_approx(x1 - mu1);
+                const float p2 = exp2_approx(x2 - mu0);
+                const float p3 = exp2_approx(x3 - mu1);
+                l_run[nt][0] = fmaf(l_run[nt][0], al0, p0 + p2);
+                l_run[nt][1] = fmaf(l_run[nt][1], al1, p1 + p3);
+                m_run[nt][0] = mn0;
+                m_run[nt][1] = mn1;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    o[mt][nt][0] *= al0;
+                    o[mt][nt][1] *= al1;
+                    o[mt][nt][2] *= al0;
+                    o[mt][nt][3] *= al1;
+                }
+                // P^T as the B operand (k = token, n = head): transpose the two 8x8 halves.
+                pb[nt][0] = movmatrix_trans(pack_bf16(p0, p1));
+                pb[nt][1] = movmatrix_trans(pack_bf16(p2, p3));
+            }
+            // O^T[d][g] += V^T[d][t] P^T[t][g]
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                const int chunk = (((mt & 3) << 1) + v_hi) ^ ri;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_trans(vs_base + (mt >> 2) * kBoxBytes + v_off + (chunk << 4), a0, a1, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            }
+            __syncwarp();
+            if (nvalid < kPage)
+                fence_proxy_async_smem();  // our zero stores precede the next TMA write of this stage
+            if (lane == 0)
+                mbar_arrive(bar_empty + 8 * s);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int sh = 4; sh < 32; sh <<= 1)
+                    l_run[nt][j] += __shfl_xor_sync(0xffffffffu, l_run[nt][j], sh);
+    }
+
+    // ---- combine the warps' states (the ring is idle now; reuse it) ----
+    __syncthreads();
+    float *cb_o = reinterpret_cast<float *>(smem);
+    float *cb_m = cb_o + NW * C::kGP * C::kOStride;
+    float *cb_l = cb_m + NW * C::kGP;
+    if (warp < NW) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int g = nt * 8 + 2 * c4 + j;
+                float *dst = cb_o + (warp * C::kGP + g) * C::kOStride;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    dst[mt * 16 + r] = o[mt][nt][j];
+                    dst[mt * 16 + r + 8] = o[mt][nt][2 + j];
+                }
+                if (r == 0) {
+                    cb_m[warp * C::kGP + g] = m_run[nt][j];
+                    cb_l[warp * C::kGP + g] = l_run[nt][j];
+                }
+            }
+    }
+    __syncthreads();
+
+    constexpr int D4 = D / 4;
+    const int G = p.G;
+    for (int e = tid; e < G * D4; e += C::kThreads) {
+        const int g = e / D4;
+        const int d4 = (e % D4) * 4;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            M = fmaxf(M, cb_m[w * C::kGP + g]);
+        float L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float mw = cb_m[w * C::kGP + g];
+            if (mw == -INFINITY)
+                continue;
+            const float sc = exp2_approx(mw - M);
+            L = fmaf(cb_l[w * C::kGP + g], sc, L);
+            O = fma4(*reinterpret_cast<const float4 *>(cb_o + (w * C::kGP + g) * C::kOStride + d4), sc, O);
+        }
+        if (nslots == 1) {
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+        } else {
+            const int64_t idx = (int64_t)my_slot * G + g;
+            *reinterpret_cast<float4 *>(p.ws_acc + idx * D + d4) = O;
+            if (d4 == 0) {
+                p.ws_m[idx] = M;
+                p.ws_l[idx] = L;
+            }
+        }
+    }
+
+    // ---- the last block of a split (row, KV head) merges its states ----
+    if (nslots > 1 && !p.separate_merge) {
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const uint32_t prev = atomicAdd(p.ws_counters + pair, 1u);
+            misc[0] = prev == (uint32_t)(nslots - 1);
+        }
+        __syncthreads();
+        if (misc[0]) {
+            __threadfence();
+            merge_pair<D>(p, row, h, slot0, nslots, tid, C::kThreads);
+            if (tid == 0)
+                p.ws_counters[pair] = 0u;  // ready for the next call
+        }
+    }
+}
+
+// Separate merge: one block per (row, KV head); pairs with one slot were
+// finalized by the split kernel.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Params p)
+{
+    const int pair = blockIdx.x;
+    const int row = pair / p.H_kv;
+    const int h = pair % p.H_kv;
+    int slot0, nslots;
+    if (p.mode == PKV_SPLIT_S) {
+        slot0 = pair * p.num_splits;
+        nslots = p.num_splits;
+    } else {
+        slot0 = __ldg(p.indptr + pair);
+        nslots = __ldg(p.indptr + pair + 1) - slot0;
+        if (slot0 < 0 || nslots < 0 || slot0 + nslots > p.n_items) {
+            if (threadIdx.x == 0)
+                atomicOr(p.ws_error, kErrItem);
+            return;
+        }
+    }
+    if (nslots <= 1)
+        return;
+    merge_pair<D>(p, row, h, slot0, nslots, threadIdx.x, blockDim.x);
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+
+namespace {
+
+constexpr int kNW = 4;   // consumer warps per block
+constexpr int kNST = 8;  // pipeline stages (pages in the shared-memory ring)
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+struct MapKey {
+    const void *base;
+    int64_t dims[4];
+    int64_t strides[3];
+    bool operator==(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+// Tensor maps are pure host encodings; a small cache saves re-encoding the
+// same pool every step.
+int pool_tensor_map(CUtensorMap *out, const void *base, const pkv_shape &s)
+{
+    static std::mutex mu;
+    static MapKey keys[8];
+    static CUtensorMap maps[8];
+    static int used = 0, next = 0;
+    MapKey key;
+    std::memset(&key, 0, sizeof key);
+    key.base = base;
+    key.dims[0] = s.head_dim;
+    key.dims[1] = s.page_size;
+    key.dims[2] = s.H_kv;
+    key.dims[3] = s.num_pool_pages;
+    key.strides[0] = s.kv_stride_token * 2;
+    key.strides[1] = s.kv_stride_head * 2;
+    key.strides[2] = s.kv_stride_page * 2;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (keys[i] == key) {
+                *out = maps[i];
+                return PKV_OK;
+            }
+    }
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return PKV_ERR_CUDA;
+    cuuint64_t dims[4], strides[3];
+    for (int i = 0; i < 4; ++i)
+        dims[i] = (cuuint64_t)key.dims[i];
+    for (int i = 0; i < 3; ++i)
+        strides[i] = (cuuint64_t)key.strides[i];
+    cuuint32_t box[4] = {(cuuint32_t)kBoxD, (cuuint32_t)s.page_size, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap tm;
+    CUresult rc = enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (rc != CUDA_SUCCESS)
+        return PKV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    keys[next] = key;
+    maps[next] = tm;
+    next = (next + 1) % 8;
+    if (used < 8)
+        ++used;
+    *out = tm;
+    return PKV_OK;
+}
+
+// cudaFuncSetAttribute is per kernel and per device; `done_mask` (one per
+// kernel instantiation) remembers the devices already configured.
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes, std::atomic<uint64_t> &done_mask)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+    if (bit && (done_mask.load() & bit))
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit)
+        done_mask.fetch_or(bit);
+    return e;
+}
+
+template <int D, int NT>
+cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st)
+{
+    using C = Cfg<D, NT, kNW, kNST>;
+    static std::atomic<uint64_t> configured{0};
+    auto kernel = split_kernel<D, NT, kNW, kNST>;
+    cudaError_t e = set_smem(kernel, C::kSmemBytes, configured);
+    if (e != cudaSuccess)
+        return e;
+    kernel<<<(unsigned)grid, C::kThreads, C::kSmemBytes, st>>>(prm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split_any(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st)
+{
+    if (D == 128)
+        return NT == 1 ? launch_split<128, 1>(prm, grid, st) : launch_split<128, 2>(prm, grid, st);
+    return NT == 1 ? launch_split<64, 1>(prm, grid, st) : launch_split<64, 2>(prm, grid, st);
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_fast_path(const pkv_shape &s)
+{
+    const int G = s.H_q / s.H_kv;
+    if (s.page_size != kPage || (s.head_dim != 64 && s.head_dim != 128) || G < 1 || G > 16)
+        return PKV_ERR_UNSUPPORTED;
+    if (s.kv_stride_token % 8 || s.kv_stride_head % 8 || s.kv_stride_page % 8 || s.kv_stride_token <= 0 ||
+        s.kv_stride_head <= 0 || s.kv_stride_page <= 0)
+        return PKV_ERR_UNSUPPORTED;
+    return PKV_OK;
+}
+
+}  // namespace
+
+// Internal entry shared by pkv_paged_decode and pkv_decode_host.
+int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, const int32_t *block_table,
+                      const int32_t *seq_lens, int32_t page_size, float scale, void *out, const pkv_shape *shape,
+                      const pkv_plan *plan, const pkv_work_item *items, const int32_t *indptr, int32_t n_items,
+                      void *workspace, size_t workspace_bytes, cudaStream_t st)
+{
+    if (check_shape(shape) != PKV_OK || !plan || page_size != shape->page_size)
+        return PKV_ERR_INVALID;
+    const pkv_shape &s = *shape;
+    const pkv_plan &pl = *plan;
+    if (pl.mode != PKV_NO_SPLIT && pl.mode != PKV_SPLIT_S && pl.mode != PKV_WORK_QUEUE)
+        return PKV_ERR_INVALID;
+    if (pl.mode == PKV_SPLIT_S && (pl.num_splits < 1 || pl.chunk_pages < 1))
+        return PKV_ERR_INVALID;
+    if (pl.mode == PKV_WORK_QUEUE && (!items || !indptr || n_items < (int64_t)s.B * s.H_kv))
+        return PKV_ERR_INVALID;
+    int rc = check_fast_path(s);
+    if (rc != PKV_OK)
+        return rc;
+    if (s.B == 0)
+        return PKV_OK;
+    if (!q || !k_pool || !v_pool || !seq_lens || !out || !workspace || (!block_table && s.max_pages_per_seq > 0))
+        return PKV_ERR_INVALID;
+    if (s.num_pool_pages < 1 || s.max_pages_per_seq < 1)
+        return PKV_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+        !aligned(workspace, 256) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+        (items && !aligned(items, 16)) || (indptr && !aligned(indptr, 4)))
+        return PKV_ERR_UNSUPPORTED;
+    const WsLayout ws = ws_layout(s, pl, n_items);
+    if (workspace_bytes < ws.total)
+        return PKV_ERR_CAPACITY;
+
+    Params prm;
+    std::memset(&prm, 0, sizeof prm);
+    if ((rc = pool_tensor_map(&prm.tm_k, k_pool, s)) != PKV_OK)
+        return rc;
+    if ((rc = pool_tensor_map(&prm.tm_v, v_pool, s)) != PKV_OK)
+        return rc;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.block_table = block_table;
+    prm.seq_lens = seq_lens;
+    prm.items = reinterpret_cast<const int4 *>(items);
+    prm.indptr = indptr;
+    prm.ws_error = reinterpret_cast<uint32_t *>(wsb + ws.error_off);
+    prm.ws_counters = reinterpret_cast<uint32_t *>(wsb + ws.counters_off);
+    prm.ws_m = reinterpret_cast<float *>(wsb + ws.m_off);
+    prm.ws_l = reinterpret_cast<float *>(wsb + ws.l_off);
+    prm.ws_acc = reinterpret_cast<float *>(wsb + ws.acc_off);
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.B = s.B;
+    prm.H_q = s.H_q;
+    prm.H_kv = s.H_kv;
+    prm.G = s.H_q / s.H_kv;
+    prm.max_pages = s.max_pages_per_seq;
+    prm.num_pool_pages = s.num_pool_pages;
+    prm.mode = pl.mode;
+    prm.num_splits = pl.mode == PKV_SPLIT_S ? pl.num_splits : 1;
+    prm.chunk_pages = pl.chunk_pages;
+    prm.separate_merge = (pl.flags & PKV_FLAG_SEPARATE_MERGE) ? 1 : 0;
+    prm.n_items = n_items;
+
+    const int64_t pairs = (int64_t)s.B * s.H_kv;
+    const int64_t grid = pl.mode == PKV_NO_SPLIT ? pairs : pl.mode == PKV_SPLIT_S ? pairs * pl.num_splits : n_items;
+    if (grid > INT32_MAX || pairs > INT32_MAX)
+        return PKV_ERR_UNSUPPORTED;
+    const int NT = prm.G <= 8 ? 1 : 2;
+    if (launch_split_any(s.head_dim, NT, prm, grid, st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const bool need_merge = pl.mode != PKV_NO_SPLIT && prm.separate_merge;
+    if (need_merge) {
+        if (s.head_dim == 128)
+            merge_kernel<128><<<(unsigned)pairs, 128, 0, st>>>(prm);
+        else
+            merge_kernel<64><<<(unsigned)pairs, 128, 0, st>>>(prm);
+        if (cudaGetLastError() != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
+
+int status_from_error_word(uint32_t w)
+{
+    if (w & kErrTimeout)
+        return PKV_ERR_TIMEOUT;
+    if (w)
+        return PKV_ERR_DEVICE_INPUT;
+    return PKV_OK;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+int pkv_paged_decode(const void *q, const void *k_pool, const void *v_pool, const int32_t *block_table,
+                     const int32_t *seq_lens, int32_t page_size, float scale, void *out, const pkv_shape *shape,
+                     const pkv_plan *plan, const pkv_work_item *items, const int32_t *indptr, int32_t n_items,
+                     void *workspace, size_t workspace_bytes, void *stream)
+{
+    return paged_decode_impl(q, k_pool, v_pool, block_table, seq_lens, page_size, scale, out, shape, plan, items,
+                             indptr, n_items, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int pkv_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!workspace || workspace_bytes < kWsAlign)
+        return PKV_ERR_INVALID;
+    if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+int pkv_workspace_status(const void *workspace, void *stream, int32_t *device_error)
+{
+    if (!workspace)
+        return PKV_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t w = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    if (cudaMemcpy(&w, workspace, sizeof w, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    if (device_error)
+        *device_error = (int32_t)w;
+    return status_from_error_word(w);
+}
+
+namespace {
+
+struct HostLayout {
+    pkv_plan plan;
+    int32_t n_items = 0;
+    WsLayout ws;
+    size_t q_off, bt_off, lens_off, out_off, items_off, indptr_off, dev_total;
+    size_t h_items_off, h_indptr_off, h_err_off, host_total;
+};
+
+int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_rule *rules, int32_t n_rules,
+                HostLayout *L)
+{
+    int rc = pkv_select_policy(lens, shape, rules, n_rules, &L->plan);
+    if (rc != PKV_OK)
+        return rc;
+    L->n_items = 0;
+    if (L->plan.mode == PKV_WORK_QUEUE) {
+        rc = pkv_work_queue_size(lens, shape, L->plan.chunk_pages, &L->n_items);
+        if (rc != PKV_OK)
+            return rc;
+    }
+    const pkv_shape &s = *shape;
+    L->ws = ws_layout(s, L->plan, L->n_items);
+    const size_t pairs = (size_t)s.B * s.H_kv;
+    size_t off = L->ws.total;
+    L->q_off = off;
+    off += round_up((size_t)s.B * s.H_q * s.head_dim * 2, kWsAlign);
+    L->bt_off = off;
+    off += round_up((size_t)s.B * s.max_pages_per_seq * 4, kWsAlign);
+    L->lens_off = off;
+    off += round_up((size_t)s.B * 4, kWsAlign);
+    L->out_off = off;
+    off += round_up((size_t)s.B * s.H_q * s.head_dim * 2, kWsAlign);
+    L->items_off = off;
+    off += round_up((size_t)L->n_items * sizeof(pkv_work_item), kWsAlign);
+    L->indptr_off = off;
+    off += round_up((pairs + 1) * 4, kWsAlign);
+    L->dev_total = off;
+    L->h_items_off = 0;
+    L->h_indptr_off = round_up((size_t)L->n_items * sizeof(pkv_work_item), 64);
+    L->h_err_off = L->h_indptr_off + round_up((pairs + 1) * 4, 64);
+    L->host_total = L->h_err_off + 64;
+    return PKV_OK;
+}
+
+}  // namespace
+
+int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape *shape, const pkv_policy_rule *rules,
+                          int32_t n_rules, size_t *device_bytes, size_t *host_bytes)
+{
+    if (!device_bytes || !host_bytes)
+        return PKV_ERR_INVALID;
+    HostLayout L;
+    int rc = host_layout(seq_lens_host, shape, rules, n_rules, &L);
+    if (rc != PKV_OK)
+        return rc;
+    *device_bytes = L.dev_total;
+    *host_bytes = L.host_total;
+    return PKV_OK;
+}
+
+int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const int32_t *seq_lens_host,
+                    void *out_host, const void *k_pool, const void *v_pool, float scale, const pkv_shape *shape,
+                    const pkv_policy_rule *rules, int32_t n_rules, void *device_buffer, size_t device_buffer_bytes,
+                    void *host_staging, size_t host_staging_bytes, void *stream, pkv_plan *plan_out)
+{
+    HostLayout L;
+    int rc = host_layout(seq_lens_host, shape, rules, n_rules, &L);
+    if (rc != PKV_OK)
+        return rc;
+    if (plan_out)
+        *plan_out = L.plan;
+    const pkv_shape &s = *shape;
+    if (s.B == 0)
+        return PKV_OK;
+    if (!q_host || !block_table_host || !out_host || !device_buffer || !host_staging)
+        return PKV_ERR_INVALID;
+    if (device_buffer_bytes < L.dev_total || host_staging_bytes < L.host_total)
+        return PKV_ERR_CAPACITY;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *dev = static_cast<uint8_t *>(device_buffer);
+    uint8_t *hst = static_cast<uint8_t *>(host_staging);
+    pkv_work_item *h_items = reinterpret_cast<pkv_work_item *>(hst + L.h_items_off);
+    int32_t *h_indptr = reinterpret_cast<int32_t *>(hst + L.h_indptr_off);
+    uint32_t *h_err = reinterpret_cast<uint32_t *>(hst + L.h_err_off);
+    if (L.plan.mode == PKV_WORK_QUEUE) {
+        int32_t n = 0;
+        rc = pkv_build_work_queue(seq_lens_host, shape, L.plan.chunk_pages, h_items, L.n_items, h_indptr, &n);
+        if (rc != PKV_OK)
+            return rc;
+    }
+    const size_t q_bytes = (size_t)s.B * s.H_q * s.head_dim * 2;
+    const size_t bt_bytes = (size_t)s.B * s.max_pages_per_seq * 4;
+    const size_t pairs = (size_t)s.B * s.H_kv;
+    bool ok = cudaMemcpyAsync(dev + L.q_off, q_host, q_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+              cudaMemcpyAsync(dev + L.bt_off, block_table_host, bt_bytes, cudaMemcpyHostToDevice, st) ==
+                  cudaSuccess &&
+              cudaMemcpyAsync(dev + L.lens_off, seq_lens_host, (size_t)s.B * 4, cudaMemcpyHostToDevice, st) ==
+                  cudaSuccess &&
+              cudaMemsetAsync(dev, 0, L.ws.m_off, st) == cudaSuccess;  // error word + completion counters
+    if (ok && L.plan.mode == PKV_WORK_QUEUE)
+        ok = cudaMemcpyAsync(dev + L.items_off, h_items, (size_t)L.n_items * sizeof(pkv_work_item),
+                             cudaMemcpyHostToDevice, st) == cudaSuccess &&
+             cudaMemcpyAsync(dev + L.indptr_off, h_indptr, (pairs + 1) * 4, cudaMemcpyHostToDevice, st) ==
+                 cudaSuccess;
+    if (!ok)
+        return PKV_ERR_CUDA;
+    rc = paged_decode_impl(dev + L.q_off, k_pool, v_pool, reinterpret_cast<const int32_t *>(dev + L.bt_off),
+                           reinterpret_cast<const int32_t *>(dev + L.lens_off), s.page_size, scale, dev + L.out_off,
+                           shape, &L.plan, reinterpret_cast<const pkv_work_item *>(dev + L.items_off),
+                           reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, dev, L.ws.total, st);
+    if (rc != PKV_OK)
+        return rc;
+    if (cudaMemcpyAsync(out_host, dev + L.out_off, q_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(h_err, dev, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return status_from_error_word(*h_err);
+}
+
+}  // extern "C"

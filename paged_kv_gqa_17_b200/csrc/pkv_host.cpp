@@ -1,0 +1,273 @@
+// Host planner of libpkv.so: policy lookup, compact work-queue builder,
+// workload counters and workspace sizing.  Pure C++, no CUDA.
+//
+// Sources: "PersistentKV: Page-Aware Decode Scheduling for Long-Context LLM
+// Serving on Commodity GPUs" (gist.science explainer), Technical summary >
+// Methodology > 1 ("Row-local bounds", "Compact work queue") and 2
+// ("Calibrated adaptive policy"); Key contributions ("page-aware scheduling",
+// "scheduler-induced workload counters"); Results (launch fan-out, merge-state
+// traffic).
+#include <algorithm>
+#include <climits>
+#include <cstring>
+#include <unordered_set>
+
+#include "pkv_internal.h"
+
+namespace pkv {
+
+int check_shape(const pkv_shape *s)
+{
+    if (!s)
+        return PKV_ERR_INVALID;
+    if (s->B < 0 || s->H_q <= 0 || s->H_kv <= 0 || s->head_dim <= 0 || s->page_size <= 0)
+        return PKV_ERR_INVALID;
+    if (s->H_q % s->H_kv != 0 || s->max_pages_per_seq < 0 || s->num_pool_pages < 0)
+        return PKV_ERR_INVALID;
+    return PKV_OK;
+}
+
+namespace {
+
+// Built-in policy table, measured on B200 (seed 20260622, checked on 20260623).
+// It is the same table as paged_kv_gqa_17_b200/policy_b200.json.
+const pkv_policy_rule kDefaultRules[] = {
+    // b_lo, b_hi, nmax_lo, nmax_hi, mode, num_splits, chunk_pages, flags
+    {1, 2, 0, 1024, PKV_NO_SPLIT, 1, 0, 0},
+    {1, 2, 1024, INT32_MAX, PKV_SPLIT_S, 37, 0, 0},
+    {2, INT32_MAX, 0, 1024, PKV_NO_SPLIT, 1, 0, 0},
+    {2, INT32_MAX, 1024, INT32_MAX, PKV_WORK_QUEUE, 1, 32, 0},
+};
+constexpr int32_t kNumDefaultRules = (int32_t)(sizeof(kDefaultRules) / sizeof(kDefaultRules[0]));
+
+int check_lens(const int32_t *lens, int32_t B)
+{
+    if (B > 0 && !lens)
+        return PKV_ERR_INVALID;
+    for (int32_t i = 0; i < B; ++i)
+        if (lens[i] < 0)
+            return PKV_ERR_INVALID;
+    return PKV_OK;
+}
+
+int check_rules(const pkv_policy_rule *rules, int32_t n)
+{
+    if (n < 0 || (n > 0 && !rules))
+        return PKV_ERR_INVALID;
+    for (int32_t k = 0; k < n; ++k) {
+        const pkv_policy_rule &r = rules[k];
+        if (r.mode != PKV_NO_SPLIT && r.mode != PKV_SPLIT_S && r.mode != PKV_WORK_QUEUE)
+            return PKV_ERR_INVALID;
+        if (r.mode == PKV_SPLIT_S && r.num_splits < 1)
+            return PKV_ERR_INVALID;
+        if (r.mode == PKV_WORK_QUEUE && r.chunk_pages < 1)
+            return PKV_ERR_INVALID;
+    }
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char *pkv_version(void) { return "pkv-b200 0.1.0 (sm_100a)"; }
+
+const char *pkv_status_string(int status)
+{
+    switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported shape or layout";
+    case PKV_ERR_CAPACITY: return "buffer too small";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_TIMEOUT: return "device wait timed out";
+    case PKV_ERR_DEVICE_INPUT: return "out-of-range device input";
+    default: return "unknown status";
+    }
+}
+
+int pkv_default_policy(pkv_policy_rule *rules, int32_t capacity, int32_t *n_rules)
+{
+    if (!n_rules)
+        return PKV_ERR_INVALID;
+    *n_rules = kNumDefaultRules;
+    if (capacity < kNumDefaultRules)
+        return PKV_ERR_CAPACITY;
+    if (!rules)
+        return PKV_ERR_INVALID;
+    std::memcpy(rules, kDefaultRules, sizeof kDefaultRules);
+    return PKV_OK;
+}
+
+int pkv_select_policy(const int32_t *seq_lens_host, const pkv_shape *shape,
+                      const pkv_policy_rule *rules, int32_t n_rules, pkv_plan *plan)
+{
+    if (!plan || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    if (!rules) {
+        rules = kDefaultRules;
+        n_rules = kNumDefaultRules;
+    }
+    int rc = check_lens(seq_lens_host, shape->B);
+    if (rc == PKV_OK)
+        rc = check_rules(rules, n_rules);
+    if (rc != PKV_OK)
+        return rc;
+    const int32_t B = shape->B;
+    int32_t n_max = 0;
+    for (int32_t i = 0; i < B; ++i)
+        n_max = std::max(n_max, seq_lens_host[i]);
+    const int64_t pages_max = ceil_div(n_max, shape->page_size);
+    const pkv_policy_rule *chosen = nullptr;
+    for (int32_t k = 0; k < n_rules && !chosen; ++k) {
+        const pkv_policy_rule &r = rules[k];
+        if (r.b_lo <= B && B < r.b_hi && r.nmax_lo <= n_max && n_max < r.nmax_hi)
+            chosen = &r;
+    }
+    if (!chosen || B == 0 || pages_max == 0) {
+        *plan = {PKV_NO_SPLIT, 1, 0, 0};
+        return PKV_OK;
+    }
+    if (chosen->mode == PKV_NO_SPLIT) {
+        *plan = {PKV_NO_SPLIT, 1, 0, chosen->flags};
+        return PKV_OK;
+    }
+    const int64_t C = chosen->mode == PKV_SPLIT_S ? ceil_div(pages_max, chosen->num_splits)
+                                                  : (int64_t)chosen->chunk_pages;
+    *plan = {chosen->mode, (int32_t)ceil_div(pages_max, C), (int32_t)C, chosen->flags};
+    return PKV_OK;
+}
+
+int pkv_work_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape, int32_t chunk_pages,
+                        int32_t *n_items)
+{
+    if (!n_items || chunk_pages < 1 || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    int rc = check_lens(seq_lens_host, shape->B);
+    if (rc != PKV_OK)
+        return rc;
+    int64_t n = 0;
+    for (int32_t i = 0; i < shape->B; ++i)
+        n += std::max<int64_t>(1, ceil_div(ceil_div(seq_lens_host[i], shape->page_size), chunk_pages));
+    n *= shape->H_kv;
+    if (n > INT32_MAX)
+        return PKV_ERR_CAPACITY;
+    *n_items = (int32_t)n;
+    return PKV_OK;
+}
+
+int pkv_build_work_queue(const int32_t *seq_lens_host, const pkv_shape *shape, int32_t chunk_pages,
+                         pkv_work_item *items, int32_t capacity, int32_t *indptr, int32_t *n_items)
+{
+    int32_t need = 0;
+    int rc = pkv_work_queue_size(seq_lens_host, shape, chunk_pages, &need);
+    if (rc != PKV_OK)
+        return rc;
+    *n_items = need;
+    if (capacity < need)
+        return PKV_ERR_CAPACITY;
+    if ((need > 0 && !items) || !indptr)
+        return PKV_ERR_INVALID;
+    const int64_t span = (int64_t)chunk_pages * shape->page_size;
+    int32_t k = 0;
+    for (int32_t i = 0; i < shape->B; ++i) {
+        const int32_t n = seq_lens_host[i];
+        for (int32_t h = 0; h < shape->H_kv; ++h) {
+            indptr[(int64_t)i * shape->H_kv + h] = k;
+            if (n == 0) {
+                items[k++] = {i, h, 0, 0};
+                continue;
+            }
+            for (int64_t b = 0; b < n; b += span)
+                items[k++] = {i, h, (int32_t)b, (int32_t)std::min<int64_t>(b + span, n)};
+        }
+    }
+    indptr[(int64_t)shape->B * shape->H_kv] = k;
+    return PKV_OK;
+}
+
+int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, const pkv_plan *plan,
+                      pkv_counters *c)
+{
+    if (!plan || !c || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    int rc = check_lens(seq_lens_host, shape->B);
+    if (rc != PKV_OK)
+        return rc;
+    const int64_t B = shape->B, H_kv = shape->H_kv, D = shape->head_dim, P = shape->page_size;
+    const int64_t G = shape->H_q / shape->H_kv;
+    const int64_t state = G * (D + 2) * 4;
+    const int64_t S = plan->num_splits, C = plan->chunk_pages;
+    const bool separate = (plan->flags & PKV_FLAG_SEPARATE_MERGE) != 0;
+    pkv_counters out{};
+    int64_t zero_rows = 0, tokens = 0, pages = 0;
+    std::unordered_set<int32_t> distinct;
+    for (int64_t i = 0; i < B; ++i) {
+        const int32_t n = seq_lens_host[i];
+        zero_rows += n == 0;
+        tokens += n;
+        pages += ceil_div(n, P);
+        if (n > 0)
+            distinct.insert(n);
+    }
+    switch (plan->mode) {
+    case PKV_NO_SPLIT:
+        out.launches = 1;
+        out.work_items = B * H_kv;
+        out.empty_items = H_kv * zero_rows;
+        break;
+    case PKV_SPLIT_S: {
+        if (S < 1 || C < 1)
+            return PKV_ERR_INVALID;
+        out.launches = 1 + (separate && S > 1);
+        out.work_items = B * H_kv * S;
+        int64_t empty = 0;
+        for (int64_t i = 0; i < B; ++i)
+            empty += S - std::min<int64_t>(S, ceil_div(ceil_div(seq_lens_host[i], P), C));
+        out.empty_items = H_kv * empty;
+        out.merge_state_bytes = S > 1 ? 2 * B * H_kv * S * state : 0;
+        break;
+    }
+    case PKV_WORK_QUEUE: {
+        if (C < 1)
+            return PKV_ERR_INVALID;
+        out.launches = 1 + (separate && S > 1);
+        int64_t items = 0, multi = 0;
+        for (int64_t i = 0; i < B; ++i) {
+            const int64_t k = std::max<int64_t>(1, ceil_div(ceil_div(seq_lens_host[i], P), C));
+            items += k;
+            if (k > 1)
+                multi += k;
+        }
+        out.work_items = H_kv * items;
+        out.empty_items = H_kv * zero_rows;
+        out.merge_state_bytes = 2 * H_kv * multi * state;
+        out.queue_bytes = 16 * out.work_items + 4 * (B * H_kv + 1);
+        break;
+    }
+    default:
+        return PKV_ERR_INVALID;
+    }
+    out.kv_bytes = tokens * H_kv * 2 * D * 2;
+    out.kv_bytes_streamed = pages * P * H_kv * 2 * D * 2;
+    out.q_bytes = B * shape->H_q * D * 2;
+    out.out_bytes = out.q_bytes;
+    out.bucket_launches = 2 * (int64_t)distinct.size();
+    *c = out;
+    return PKV_OK;
+}
+
+int pkv_workspace_bytes(const pkv_shape *shape, const pkv_plan *plan, int32_t n_items, size_t *bytes)
+{
+    if (!plan || !bytes || check_shape(shape) != PKV_OK || n_items < 0)
+        return PKV_ERR_INVALID;
+    if (plan->mode == PKV_SPLIT_S && plan->num_splits < 1)
+        return PKV_ERR_INVALID;
+    *bytes = ws_layout(*shape, *plan, n_items).total;
+    return PKV_OK;
+}
+
+}  // extern "C"
