@@ -67,6 +67,12 @@ typedef enum {
 /* pkv_plan.flags / pkv_policy_rule.flags */
 #define PKV_FLAG_SEPARATE_MERGE 1 /* merge partial states in a second kernel instead of in the
                                      last block that finishes a (row, KV head) */
+#define PKV_FLAG_NO_PDL 2         /* launch without programmatic dependent launch (by default the
+                                     kernels may be scheduled while the previous kernel on the
+                                     stream finishes; they wait for it before any memory access) */
+#define PKV_FLAG_DEEP_RING 4      /* split kernel with a 12-page shared-memory ring (two blocks per
+                                     SM) instead of 8 pages (three blocks per SM): more bytes in
+                                     flight per block, for grids of about two blocks per SM */
 
 /* Problem shape and pool layout.  Pool element (page, kv_head, slot, d) of
  * k_pool / v_pool lives at  page*kv_stride_page + kv_head*kv_stride_head +

@@ -121,6 +121,22 @@ __device__ __forceinline__ uint64_t global_timer_ns()
     return t;
 }
 
+// Optional timeline tracing (build with -DPKV_TRACE): thread 0 of each block
+// records global-timer stamps at fixed points of the kernel.
+#ifdef PKV_TRACE
+constexpr int kTraceBlocks = 65536;
+__device__ unsigned long long g_pkv_trace[kTraceBlocks][16];
+#define PKV_TRACE_POINT(slot)                                                  \
+    do {                                                                       \
+        if (threadIdx.x == 0 && blockIdx.x < kTraceBlocks)                     \
+            g_pkv_trace[blockIdx.x][slot] = global_timer_ns();                 \
+    } while (0)
+#else
+#define PKV_TRACE_POINT(slot) \
+    do {                      \
+    } while (0)
+#endif
+
 // Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs (or
 // kWaitLimitIters polls) with the timeout bit set in the error word.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err)
@@ -154,6 +170,43 @@ __device__ __forceinline__ void tma_load_box(uint32_t dst, const CUtensorMap *tm
         " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(d0), "r"(0), "r"(head), "r"(page), "r"(bar), "l"(policy)
         : "memory");
+}
+
+// Bulk (non-tensor) async copy global -> shared, completion on an mbarrier.
+// Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Ticket: atomic add with release (orders this block's earlier writes, made
+// visible to thread 0 by the preceding __syncthreads) and acquire (the last
+// arriver sees every other block's released writes).
+__device__ __forceinline__ uint32_t ticket_acq_rel(uint32_t *ctr)
+{
+    uint32_t prev;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr) : "memory");
+    return prev;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Programmatic dependent launch: wait for the grids this one depends on
+// (complete, memory visible); allow dependents to be scheduled.  Both are
+// no-ops when the kernel was launched without the PDL attribute.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *tm)
@@ -238,6 +291,11 @@ __device__ __forceinline__ float4 scale4(float4 a, float s)
 template <int D, int NT, int NW, int NST>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head_dim");
+    // Pages go to warps round robin and to stages round robin; when NST is a
+    // multiple of NW every use of a stage belongs to the same warp, so a
+    // stage's mbarrier can never be more than one phase ahead of its waiter
+    // (otherwise phase parities could alias).
+    static_assert(NST % NW == 0, "stages must be a multiple of consumer warps");
     static constexpr int kHalves = D / kBoxD;
     static constexpr int kStageBytes = D * kPage * 2;  // one K (or V) page of one KV head
     static constexpr int kThreads = (NW + 1) * 32;     // NW consumer warps + 1 producer warp
@@ -246,8 +304,9 @@ struct Cfg {
     static constexpr int kCombineBytes = NW * kGP * (kOStride + 2) * 4;
     static constexpr int kRingBytes = 2 * NST * kStageBytes;
     static constexpr int kBarOff = ((kRingBytes > kCombineBytes ? kRingBytes : kCombineBytes) + 63) / 64 * 64;
-    static constexpr int kMiscOff = kBarOff + 2 * NST * 8;
+    static constexpr int kMiscOff = kBarOff + 2 * NST * 8;  // int flag, then two merge mbarriers at +8, +16
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + slack to align the base to 1024
+    static constexpr int kMaxMergeTasks = (kGP * (D / 4) + kThreads - 1) / kThreads;
 };
 
 // Merge the nslots partial states of one (row, KV head) in ascending slot
@@ -294,6 +353,122 @@ __device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslot
     }
 }
 
+// Merge of one (row, KV head)'s n partial states by the block that finished
+// it last, staged through the idle shared-memory ring.  The weights
+// w_s = 2^(m_s - M) (M = max_s m_s, 0 for a neutral state) and the
+// denominator L = sum_s w_s l_s are computed once per head; the fp32
+// accumulators arrive in chunks by bulk async copies (double buffered), and
+// out = sum_s w_s acc_s / L is accumulated in ascending slot order.
+// Returns false when the ring cannot hold the weights plus two slots.
+template <int D, int NT, int NW, int NST>
+__device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0, int row, int h, int slot0, int n,
+                                  int tid)
+{
+    using C = Cfg<D, NT, NW, NST>;
+    const int G = p.G;
+    constexpr int D4 = D / 4;
+    const int slot_bytes = G * D * 4;
+    const int wbytes = ((2 * n * G + 32) * 4 + 1023) / 1024 * 1024;
+    const int half = (C::kRingBytes - wbytes) / 2 / 1024 * 1024;
+    const int hs = half > 0 ? half / slot_bytes : 0;  // slots per buffer
+    if (hs < 1)
+        return false;
+    float *w_s = reinterpret_cast<float *>(smem);  // [n][G]: m, then the weights
+    float *l_s = w_s + n * G;                      // [n][G]
+    float *ML = l_s + n * G;                       // M[16], L[16]
+    const uint32_t stage0 = smem_addr(smem) + wbytes;
+    const int nch = (n + hs - 1) / hs;
+    if (tid == 0) {
+        fence_proxy_async_global();  // the states were written by other blocks' generic stores
+        for (int ch = 0; ch < 2 && ch < nch; ++ch) {
+            const int cnt = min(hs, n - ch * hs);
+            mbar_expect_tx(mbar0 + 8 * ch, cnt * slot_bytes);
+            bulk_g2s(stage0 + ch * half, p.ws_acc + (int64_t)(slot0 + ch * hs) * G * D, cnt * slot_bytes,
+                     mbar0 + 8 * ch);
+        }
+    }
+    for (int i = tid; i < n * G; i += C::kThreads) {
+        w_s[i] = __ldcg(p.ws_m + (int64_t)slot0 * G + i);
+        l_s[i] = __ldcg(p.ws_l + (int64_t)slot0 * G + i);
+    }
+    __syncthreads();
+    // One warp per head: M = max_s m_s, the weights, and L = sum_s w_s l_s,
+    // each reduced over the lanes by a fixed xor-shuffle tree.
+    const int lane = tid & 31;
+    for (int g = tid >> 5; g < G; g += C::kThreads / 32) {
+        float M = -INFINITY;
+        for (int s = lane; s < n; s += 32)
+            M = fmaxf(M, w_s[s * G + g]);
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1)
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+        float L = 0.f;
+        for (int s = lane; s < n; s += 32) {
+            const float m = w_s[s * G + g];
+            const float wgt = m == -INFINITY ? 0.f : exp2_approx(m - M);
+            w_s[s * G + g] = wgt;
+            L = fmaf(wgt, l_s[s * G + g], L);
+        }
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1)
+            L += __shfl_xor_sync(0xffffffffu, L, sh);
+        if (lane == 0)
+            ML[16 + g] = L;
+    }
+    __syncthreads();
+    float4 O[C::kMaxMergeTasks];
+#pragma unroll
+    for (int k = 0; k < C::kMaxMergeTasks; ++k)
+        O[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int ch = 0; ch < nch; ++ch) {
+        mbar_wait(mbar0 + 8 * (ch & 1), (ch >> 1) & 1, p.ws_error);
+        const float *st = reinterpret_cast<const float *>(smem + wbytes + (ch & 1) * half);
+        const int first = ch * hs;
+        const int cnt = min(hs, n - first);
+#pragma unroll
+        for (int k = 0; k < C::kMaxMergeTasks; ++k) {
+            const int e = tid + k * C::kThreads;
+            if (e < G * D4) {
+                const int g = e / D4;
+                const int d4 = (e % D4) * 4;
+                float4 O2 = make_float4(0.f, 0.f, 0.f, 0.f);  // second chain for ILP
+                int s = 0;
+                for (; s + 1 < cnt; s += 2) {
+                    O[k] = fma4(*reinterpret_cast<const float4 *>(st + (s * G + g) * D + d4),
+                                w_s[(first + s) * G + g], O[k]);
+                    O2 = fma4(*reinterpret_cast<const float4 *>(st + ((s + 1) * G + g) * D + d4),
+                              w_s[(first + s + 1) * G + g], O2);
+                }
+                if (s < cnt)
+                    O[k] = fma4(*reinterpret_cast<const float4 *>(st + (s * G + g) * D + d4), w_s[(first + s) * G + g],
+                                O[k]);
+                O[k] = make_float4(O[k].x + O2.x, O[k].y + O2.y, O[k].z + O2.z, O[k].w + O2.w);
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && ch + 2 < nch) {
+            fence_proxy_async_smem();  // our reads of this buffer precede its refill
+            const int c2 = ch + 2;
+            const int cnt2 = min(hs, n - c2 * hs);
+            mbar_expect_tx(mbar0 + 8 * (c2 & 1), cnt2 * slot_bytes);
+            bulk_g2s(stage0 + (c2 & 1) * half, p.ws_acc + (int64_t)(slot0 + c2 * hs) * G * D, cnt2 * slot_bytes,
+                     mbar0 + 8 * (c2 & 1));
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < C::kMaxMergeTasks; ++k) {
+        const int e = tid + k * C::kThreads;
+        if (e < G * D4) {
+            const int g = e / D4;
+            const int d4 = (e % D4) * 4;
+            const float L = ML[16 + g];
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O[k], inv));
+        }
+    }
+    return true;
+}
+
 // One block = one work item (row, KV head, token range) for all G query heads.
 template <int D, int NT, int NW, int NST>
 __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_constant__ Params p)
@@ -312,9 +487,18 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int64_t row_cap = (int64_t)p.max_pages * kPage;
+    PKV_TRACE_POINT(0);
+    // Under programmatic dependent launch this block may start while the
+    // previous kernel on the stream is still running: wait before touching
+    // any global memory it may have written.
+    grid_dependency_wait();
 
     // ---- which (row, KV head, token range) this block owns ----
+    // The producer warp fetches the first 32 block-table entries of the
+    // range as soon as the range's first page is known, which for the
+    // no-split and split-S grids is before the row length arrives.
     int row, h, tb, te, slot0 = 0, nslots = 1, my_slot = 0;
+    int e_first = 0;
     if (p.mode == PKV_WORK_QUEUE) {
         const int4 it = __ldg(p.items + blockIdx.x);
         row = it.x;
@@ -336,12 +520,22 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
                 atomicOr(p.ws_error, kErrItem);
             return;
         }
+        if (warp == NW) {
+            const int idx = tb / kPage + lane;
+            if (idx < p.max_pages)
+                e_first = __ldg(p.block_table + (int64_t)row * p.max_pages + idx);
+        }
     } else {
         const int S = p.mode == PKV_SPLIT_S ? p.num_splits : 1;
         const int pair = blockIdx.x / S;
         const int c = blockIdx.x % S;
         row = pair / p.H_kv;
         h = pair % p.H_kv;
+        if (warp == NW) {
+            const int64_t idx = (p.mode == PKV_SPLIT_S ? (int64_t)c * p.chunk_pages : 0) + lane;
+            if (idx < p.max_pages)
+                e_first = __ldg(p.block_table + (int64_t)row * p.max_pages + idx);
+        }
         int N = __ldg(p.seq_lens + row);
         if (N < 0 || N > row_cap) {
             if (tid == 0)
@@ -372,6 +566,8 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
+        mbar_init(sbase + C::kMiscOff + 8, 1);
+        mbar_init(sbase + C::kMiscOff + 16, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
@@ -380,6 +576,15 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         prefetch_tensormap(&p.tm_v);
     }
     __syncthreads();
+    PKV_TRACE_POINT(1);
+#ifdef PKV_TRACE
+    if (tid == 0 && blockIdx.x < kTraceBlocks) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        g_pkv_trace[blockIdx.x][6] = smid;
+        g_pkv_trace[blockIdx.x][7] = npages;
+    }
+#endif
 
     // Per-warp softmax state for the heads g = 8*nt + 2*(lane%4) + j.
     float m_run[NT][2], l_run[NT][2];
@@ -399,7 +604,11 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         // ================= producer: block table -> TMA page copies =================
         const int32_t *bt = p.block_table + (int64_t)row * p.max_pages + pg0;
         const uint64_t policy = evict_first_policy();
-        int e_next = lane < npages ? __ldg(bt + lane) : 0;
+#ifdef PKV_TRACE
+        long long prod_wait = 0;
+        const long long prod_t0 = clock64();
+#endif
+        int e_next = lane < npages ? e_first : 0;
         bool ok = true;
         for (int base = 0; base < npages && ok; base += 32) {
             int e = e_next;
@@ -416,8 +625,14 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
                 const int s = pidx % NST;
                 const int k = pidx / NST;
                 if (lane == 0) {
+#ifdef PKV_TRACE
+                    const long long tw0 = clock64();
+#endif
                     if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, p.ws_error))
                         ok = false;
+#ifdef PKV_TRACE
+                    prod_wait += clock64() - tw0;
+#endif
                     if (ok) {
                         const uint32_t fb = bar_full + 8 * s;
                         mbar_expect_tx(fb, 2 * C::kStageBytes);
@@ -435,6 +650,12 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
                     break;
             }
         }
+#ifdef PKV_TRACE
+        if (lane == 0 && blockIdx.x < kTraceBlocks) {
+            g_pkv_trace[blockIdx.x][10] = prod_wait;
+            g_pkv_trace[blockIdx.x][11] = clock64() - prod_t0;
+        }
+#endif
     } else {
         // ================= consumers: tensor-core attention over pages =================
         // Q as the MMA's B operand (k = head_dim, n = query head), loaded once.
@@ -463,10 +684,20 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         const uint32_t v_off = (uint32_t)((8 * (mi >> 1) + ri) * 128);  // V^T as A via .trans
         const int v_hi = mi & 1;
         const float sl2 = p.scale_log2;
+#ifdef PKV_TRACE
+        long long cons_wait = 0;
+        const long long cons_t0 = clock64();
+#endif
 
         for (int pidx = warp; pidx < npages; pidx += NW) {
             const int s = pidx % NST;
+#ifdef PKV_TRACE
+            const long long tw0 = clock64();
+#endif
             const bool ready = mbar_wait(bar_full + 8 * s, (pidx / NST) & 1, p.ws_error);
+#ifdef PKV_TRACE
+            cons_wait += clock64() - tw0;
+#endif
             if (!__all_sync(0xffffffffu, ready))
                 break;
             const uint32_t ks_base = k_ring + s * C::kStageBytes;
@@ -500,6 +731,22 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
                 for (int nt = 0; nt < NT; ++nt)
                     mma_bf16(sacc[nt], a0, a1, a2, a3, qf[ks][nt][0], qf[ks][nt][1]);
             }
+            // V^T fragments to registers, then hand the stage back to the
+            // producer before the softmax and PV math.
+            uint32_t vf[D / 16][4];
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                const int chunk = (((mt & 3) << 1) + v_hi) ^ ri;
+                ldsm_x4_trans(vs_base + (mt >> 2) * kBoxBytes + v_off + (chunk << 4), vf[mt][0], vf[mt][1],
+                              vf[mt][2], vf[mt][3]);
+            }
+            __syncwarp();
+            if (nvalid < kPage)
+                fence_proxy_async_smem();  // our zero stores precede the next TMA write of this stage
+            if (lane == 0)
+                mbar_arrive(bar_empty + 8 * s);  // release: orders the fragment loads before the refill
+            if (pidx == 0)
+                PKV_TRACE_POINT(2);
             // Online softmax over this page (log2 domain), tokens past the end masked.
             const bool lo_ok = r < nvalid;
             const bool hi_ok = r + 8 < nvalid;
@@ -543,20 +790,17 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             }
             // O^T[d][g] += V^T[d][t] P^T[t][g]
 #pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                const int chunk = (((mt & 3) << 1) + v_hi) ^ ri;
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_trans(vs_base + (mt >> 2) * kBoxBytes + v_off + (chunk << 4), a0, a1, a2, a3);
+            for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
-                    mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-            }
-            __syncwarp();
-            if (nvalid < kPage)
-                fence_proxy_async_smem();  // our zero stores precede the next TMA write of this stage
-            if (lane == 0)
-                mbar_arrive(bar_empty + 8 * s);
+                    mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
         }
+#ifdef PKV_TRACE
+        if (tid == 0 && blockIdx.x < kTraceBlocks) {
+            g_pkv_trace[blockIdx.x][8] = cons_wait;
+            g_pkv_trace[blockIdx.x][9] = clock64() - cons_t0;
+        }
+#endif
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -567,7 +811,9 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     }
 
     // ---- combine the warps' states (the ring is idle now; reuse it) ----
+    grid_launch_dependents();  // the next kernel may start its prologue
     __syncthreads();
+    PKV_TRACE_POINT(3);
     float *cb_o = reinterpret_cast<float *>(smem);
     float *cb_m = cb_o + NW * C::kGP * C::kOStride;
     float *cb_l = cb_m + NW * C::kGP;
@@ -624,20 +870,21 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         }
     }
 
+    PKV_TRACE_POINT(4);
     // ---- the last block of a split (row, KV head) merges its states ----
     if (nslots > 1 && !p.separate_merge) {
-        __threadfence();
         __syncthreads();
         if (tid == 0) {
-            const uint32_t prev = atomicAdd(p.ws_counters + pair, 1u);
+            const uint32_t prev = ticket_acq_rel(p.ws_counters + pair);
             misc[0] = prev == (uint32_t)(nslots - 1);
         }
         __syncthreads();
         if (misc[0]) {
-            __threadfence();
-            merge_pair<D>(p, row, h, slot0, nslots, tid, C::kThreads);
+            if (!merge_pair_staged<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid))
+                merge_pair<D>(p, row, h, slot0, nslots, tid, C::kThreads);
             if (tid == 0)
                 p.ws_counters[pair] = 0u;  // ready for the next call
+            PKV_TRACE_POINT(5);
         }
     }
 }
@@ -647,6 +894,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Params p)
 {
+    grid_dependency_wait();  // the split kernel's partial states are complete and visible
     const int pair = blockIdx.x;
     const int row = pair / p.H_kv;
     const int h = pair % p.H_kv;
@@ -673,8 +921,21 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Para
 
 namespace {
 
-constexpr int kNW = 4;   // consumer warps per block
-constexpr int kNST = 8;  // pipeline stages (pages in the shared-memory ring)
+// Block shapes: kNW consumer warps and a ring of kNST pages (three blocks fit
+// per SM), or the deep ring of kNSTDeep pages (two blocks per SM, more bytes in
+// flight per block; chosen per plan with PKV_FLAG_DEEP_RING).
+#ifndef PKV_NW
+#define PKV_NW 4
+#endif
+#ifndef PKV_NST
+#define PKV_NST 8
+#endif
+#ifndef PKV_NST_DEEP
+#define PKV_NST_DEEP 12
+#endif
+constexpr int kNW = PKV_NW;
+constexpr int kNST = PKV_NST;
+constexpr int kNSTDeep = PKV_NST_DEEP;
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
@@ -768,24 +1029,48 @@ cudaError_t set_smem(K kernel, int bytes, std::atomic<uint64_t> &done_mask)
     return e;
 }
 
-template <int D, int NT>
-cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st)
+template <typename... Args>
+cudaError_t launch_ex(void (*kernel)(Args...), unsigned grid, unsigned block, size_t smem, cudaStream_t st, bool pdl,
+                      const Params &prm)
 {
-    using C = Cfg<D, NT, kNW, kNST>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, prm);
+}
+
+template <int D, int NT, int NST>
+cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+{
+    using C = Cfg<D, NT, kNW, NST>;
     static std::atomic<uint64_t> configured{0};
-    auto kernel = split_kernel<D, NT, kNW, kNST>;
+    auto kernel = split_kernel<D, NT, kNW, NST>;
     cudaError_t e = set_smem(kernel, C::kSmemBytes, configured);
     if (e != cudaSuccess)
         return e;
-    kernel<<<(unsigned)grid, C::kThreads, C::kSmemBytes, st>>>(prm);
-    return cudaGetLastError();
+    e = launch_ex(kernel, (unsigned)grid, C::kThreads, C::kSmemBytes, st, pdl, prm);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_split_any(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st)
+template <int NST>
+cudaError_t launch_split_nst(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
 {
     if (D == 128)
-        return NT == 1 ? launch_split<128, 1>(prm, grid, st) : launch_split<128, 2>(prm, grid, st);
-    return NT == 1 ? launch_split<64, 1>(prm, grid, st) : launch_split<64, 2>(prm, grid, st);
+        return NT == 1 ? launch_split<128, 1, NST>(prm, grid, st, pdl) : launch_split<128, 2, NST>(prm, grid, st, pdl);
+    return NT == 1 ? launch_split<64, 1, NST>(prm, grid, st, pdl) : launch_split<64, 2, NST>(prm, grid, st, pdl);
+}
+
+cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+{
+    return deep ? launch_split_nst<kNSTDeep>(D, NT, prm, grid, st, pdl)
+                : launch_split_nst<kNST>(D, NT, prm, grid, st, pdl);
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -872,15 +1157,15 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     if (grid > INT32_MAX || pairs > INT32_MAX)
         return PKV_ERR_UNSUPPORTED;
     const int NT = prm.G <= 8 ? 1 : 2;
-    if (launch_split_any(s.head_dim, NT, prm, grid, st) != cudaSuccess)
+    const bool pdl = (pl.flags & PKV_FLAG_NO_PDL) == 0;
+    const bool deep = (pl.flags & PKV_FLAG_DEEP_RING) != 0;
+    if (launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl) != cudaSuccess)
         return PKV_ERR_CUDA;
     const bool need_merge = pl.mode != PKV_NO_SPLIT && prm.separate_merge;
     if (need_merge) {
-        if (s.head_dim == 128)
-            merge_kernel<128><<<(unsigned)pairs, 128, 0, st>>>(prm);
-        else
-            merge_kernel<64><<<(unsigned)pairs, 128, 0, st>>>(prm);
-        if (cudaGetLastError() != cudaSuccess)
+        cudaError_t e = s.head_dim == 128 ? launch_ex(merge_kernel<128>, (unsigned)pairs, 128, 0, st, pdl, prm)
+                                          : launch_ex(merge_kernel<64>, (unsigned)pairs, 128, 0, st, pdl, prm);
+        if (e != cudaSuccess || cudaGetLastError() != cudaSuccess)
             return PKV_ERR_CUDA;
     }
     return PKV_OK;
@@ -909,6 +1194,14 @@ int pkv_paged_decode(const void *q, const void *k_pool, const void *v_pool, cons
     return paged_decode_impl(q, k_pool, v_pool, block_table, seq_lens, page_size, scale, out, shape, plan, items,
                              indptr, n_items, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
+
+#ifdef PKV_TRACE
+// Copy the timeline of the first blocks (16 uint64 per block) to the host.
+__attribute__((visibility("default"))) int pkv_trace_read(void *host, size_t bytes)
+{
+    return cudaMemcpyFromSymbol(host, g_pkv_trace, bytes) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+#endif
 
 int pkv_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
 {

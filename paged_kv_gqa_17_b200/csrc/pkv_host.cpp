@@ -34,9 +34,9 @@ namespace {
 const pkv_policy_rule kDefaultRules[] = {
     // b_lo, b_hi, nmax_lo, nmax_hi, mode, num_splits, chunk_pages, flags
     {1, 2, 0, 1024, PKV_NO_SPLIT, 1, 0, 0},
-    {1, 2, 1024, INT32_MAX, PKV_SPLIT_S, 37, 0, 0},
+    {1, 2, 1024, INT32_MAX, PKV_SPLIT_S, 37, 0, PKV_FLAG_DEEP_RING},
     {2, INT32_MAX, 0, 1024, PKV_NO_SPLIT, 1, 0, 0},
-    {2, INT32_MAX, 1024, INT32_MAX, PKV_WORK_QUEUE, 1, 32, 0},
+    {2, INT32_MAX, 1024, INT32_MAX, PKV_WORK_QUEUE, 1, 16, 0},
 };
 constexpr int32_t kNumDefaultRules = (int32_t)(sizeof(kDefaultRules) / sizeof(kDefaultRules[0]));
 

@@ -30,6 +30,10 @@ MODES = {
     "wq3": rule(2, 1, 3),
     "wq16": rule(2, 1, 16),
     "wq3_sep": rule(2, 1, 3, 1),
+    "split32_deep": rule(1, 32, 0, 4),
+    "wq3_deep_sep": rule(2, 1, 3, 5),
+    "split7_nopdl": rule(1, 7, 0, 2),
+    "wq16_deep_nopdl": rule(2, 1, 16, 6),
 }
 
 
@@ -64,7 +68,8 @@ CASES = {
 
 
 @pytest.mark.parametrize("case", sorted(CASES))
-@pytest.mark.parametrize("mode", ["nosplit", "split7", "split32", "split32_sep", "wq3", "wq3_sep"])
+@pytest.mark.parametrize("mode", ["nosplit", "split7", "split32", "split32_sep", "wq3", "wq3_sep", "split32_deep",
+                                  "wq3_deep_sep", "split7_nopdl"])
 def test_ragged_shapes(case, mode):
     lens, H_q, H_kv, D = CASES[case]
     w = to_device(W.make_custom(lens, H_q, H_kv, D, seed=101, poison=True, q_scale=3.0))
