@@ -231,6 +231,40 @@ PKV_API int pkv_paged_decode(const void *q, const void *k_pool, const void *v_po
                              const pkv_work_item *items, const int32_t *indptr, int32_t n_items,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* Scratch bytes held inside the library for pkv_paged_decode_noalloc. */
+#define PKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* pkv_paged_decode for callers that cannot allocate device memory.  The
+ * paper has no counterpart; this is a convenience of this library.
+ * Some callers cannot call cudaMalloc at the point where they decode: a
+ * plugin inside a host framework that owns every device allocation and
+ * hands out no scratch, a deployment that must run in a fixed, pre-sized
+ * memory budget, or a latency-critical loop that cannot afford the device
+ * synchronization an allocation may cause.  They pass the same inputs and
+ * output as pkv_paged_decode but no workspace: the error word, completion
+ * counters and partial softmax states live in a 16 MiB array compiled into
+ * the library (PKV_NOALLOC_SCRATCH_BYTES; every GPU that loads the library
+ * holds it until the process exits).  The call allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ *  - A plan whose workspace (pkv_workspace_bytes) exceeds the array returns
+ *    PKV_ERR_CAPACITY before anything is queued.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Each call queues a memset that zeroes the error word and the counters,
+ *    then the kernels; the array keeps the last call's contents otherwise.
+ *  - All calls share the one array: calls that may overlap on the GPU (two
+ *    streams, two threads) race and corrupt each other's results.  Order
+ *    them on one stream.
+ *  - Errors the kernels detect on device data cannot be read back through
+ *    this entry point; use pkv_paged_decode with a workspace to diagnose.
+ * Other arguments, layouts and return codes as pkv_paged_decode. */
+PKV_API int pkv_paged_decode_noalloc(const void *q, const void *k_pool, const void *v_pool,
+                                     const int32_t *block_table, const int32_t *seq_lens,
+                                     int32_t page_size, float scale, void *out, const pkv_shape *shape,
+                                     const pkv_plan *plan, const pkv_work_item *items,
+                                     const int32_t *indptr, int32_t n_items, void *stream);
+
 /* Sizes of the caller buffers pkv_decode_host needs for this batch and
  * policy table (rules NULL = built-in): *device_bytes of device memory and
  * *host_bytes of host staging memory (page-locked memory makes the copies

@@ -86,6 +86,8 @@ SIGNATURES = [
     ("pkv_workspace_status", ctypes.c_int, [c_p, c_p, c_p]),
     ("pkv_paged_decode", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_i32, ctypes.c_float, c_p, c_p, c_p, c_p, c_p, c_i32, c_p, c_sz, c_p]),
+    ("pkv_paged_decode_noalloc", ctypes.c_int,
+     [c_p, c_p, c_p, c_p, c_p, c_i32, ctypes.c_float, c_p, c_p, c_p, c_p, c_p, c_i32, c_p]),
     ("pkv_decode_host_bytes", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_p, c_p]),
     ("pkv_decode_host", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p]),
@@ -281,6 +283,25 @@ def paged_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, bl
                             plan.indptr.data_ptr() if plan.indptr is not None else None, plan.n_items,
                             plan.workspace.data_ptr(), plan.workspace.numel(), _stream_ptr(stream))
     _check(rc, "pkv_paged_decode")
+    return out
+
+
+def paged_decode_noalloc(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, block_table: torch.Tensor,
+                         seq_lens: torch.Tensor, page_size: int, scale: float, plan: DecodePlan,
+                         out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pkv_paged_decode_noalloc: like paged_decode, but the library's own fixed
+    scratch array replaces the plan's workspace (for callers that cannot
+    allocate device memory; see include/pkv.h)."""
+    L = lib()
+    if out is None:
+        out = torch.empty_like(q)
+    rc = L.pkv_paged_decode_noalloc(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
+                                    seq_lens.data_ptr(), page_size, float(scale), out.data_ptr(),
+                                    ctypes.byref(plan.shape), ctypes.byref(plan.plan),
+                                    plan.items.data_ptr() if plan.items is not None else None,
+                                    plan.indptr.data_ptr() if plan.indptr is not None else None, plan.n_items,
+                                    _stream_ptr(stream))
+    _check(rc, "pkv_paged_decode_noalloc")
     return out
 
 

@@ -1229,6 +1229,33 @@ int pkv_workspace_status(const void *workspace, void *stream, int32_t *device_er
 
 namespace {
 
+// ---------------------------------------------------------------------------
+// Scratch for pkv_paged_decode_noalloc: a fixed array in the library's device
+// image, so that callers without an allocator can still run split plans.
+// Every GPU that loads the library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the symbol is only a host-side handle; the address has to be looked up once
+// per device (with that device current) and is cached here.
+void *noalloc_scratch_address()
+{
+    static std::mutex mu;
+    static void *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess)
+            return nullptr;
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
 struct HostLayout {
     pkv_plan plan;
     int32_t n_items = 0;
@@ -1274,6 +1301,30 @@ int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_ru
 }
 
 }  // namespace
+
+int pkv_paged_decode_noalloc(const void *q, const void *k_pool, const void *v_pool, const int32_t *block_table,
+                             const int32_t *seq_lens, int32_t page_size, float scale, void *out,
+                             const pkv_shape *shape, const pkv_plan *plan, const pkv_work_item *items,
+                             const int32_t *indptr, int32_t n_items, void *stream)
+{
+    if (check_shape(shape) != PKV_OK || !plan || n_items < 0)
+        return PKV_ERR_INVALID;
+    const WsLayout ws = ws_layout(*shape, *plan, n_items);
+    if (ws.total > kNoAllocScratchBytes)
+        return PKV_ERR_CAPACITY;  // the plan needs more scratch than the library holds
+    if (shape->B == 0)
+        return PKV_OK;
+    void *scratch = noalloc_scratch_address();
+    if (!scratch)
+        return PKV_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // The array keeps whatever the previous call left in it: the error word
+    // and the completion counters must start at zero, the partial states not.
+    if (cudaMemsetAsync(scratch, 0, ws.m_off, st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return paged_decode_impl(q, k_pool, v_pool, block_table, seq_lens, page_size, scale, out, shape, plan, items,
+                             indptr, n_items, scratch, kNoAllocScratchBytes, st);
+}
 
 int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape *shape, const pkv_policy_rule *rules,
                           int32_t n_rules, size_t *device_bytes, size_t *host_bytes)

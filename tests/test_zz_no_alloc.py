@@ -1,0 +1,90 @@
+"""pkv_paged_decode_noalloc against pkv_paged_decode, through the C ABI.
+
+The no-alloc entry point serves callers that cannot allocate device memory
+where they decode (a plugin in a framework that owns all allocations, a
+fixed memory budget, a loop that cannot take an allocation's device
+synchronization): it takes no workspace and uses a fixed scratch array inside
+the library instead.  Its results must match the workspace entry point's
+within the tests' tolerance, call after call, even when consecutive calls use
+different plans and so leave different contents in the shared scratch.
+
+This file is named to be collected last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_gqa_17_b200 import binding as bd
+from paged_kv_gqa_17_b200 import workloads as W
+
+from .gpu_util import ATOL, RTOL, to_device
+
+pytestmark = pytest.mark.gpu
+
+ANY = (0, 2**31 - 1, 0, 2**31 - 1)
+RULES = [
+    bd.Rule(*ANY, 1, 37, 0, 4),   # split-S, fused merge, deep ring
+    bd.Rule(*ANY, 2, 1, 3, 0),    # work queue, fused merge
+    bd.Rule(*ANY, 2, 1, 5, 1),    # work queue, separate merge kernel
+    bd.Rule(*ANY, 0, 1, 0, 0),    # no split
+    bd.Rule(*ANY, 1, 9, 0, 0),    # split-S again, other slot layout
+]
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_gqa_17_b200 import build
+
+    build.build()
+    return bd.lib()
+
+
+def _noalloc(L, w, dp, lens_dev):
+    out = torch.full_like(w.q, float("nan"))
+    rc = L.pkv_paged_decode_noalloc(
+        w.q.data_ptr(), w.k_pool.data_ptr(), w.v_pool.data_ptr(), w.block_table.data_ptr(), lens_dev.data_ptr(),
+        w.P, ctypes.c_float(w.scale), out.data_ptr(), ctypes.byref(dp.shape), ctypes.byref(dp.plan),
+        dp.items.data_ptr() if dp.items is not None else None,
+        dp.indptr.data_ptr() if dp.indptr is not None else None, dp.n_items,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, rc
+    return out
+
+
+def _close(a: torch.Tensor, b: torch.Tensor, what: str):
+    x = a.float().cpu().double().numpy()
+    y = b.float().cpu().double().numpy()
+    assert np.isfinite(x).all(), what
+    assert (np.abs(x - y) <= ATOL + RTOL * np.abs(y)).all(), f"{what}: max diff {np.abs(x - y).max():.3e}"
+
+
+@pytest.mark.parametrize("lens,H_q,H_kv,D", [([3000, 17, 1024, 0, 513], 32, 8, 128), ([700, 64], 8, 2, 64)])
+def test_noalloc_matches_workspace_entry_point(L, lens, H_q, H_kv, D):
+    w = to_device(W.make_custom(lens, H_q, H_kv, D, seed=301, poison=True))
+    lens_dev = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    for rule in RULES:
+        dp = bd.plan_decode(w.seq_lens, shape, "cuda", rules=[rule])
+        ref = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens_dev, w.P, w.scale, plan=dp)
+        torch.cuda.synchronize()
+        assert bd.workspace_status(dp) == 0
+        first = _noalloc(L, w, dp, lens_dev)
+        second = _noalloc(L, w, dp, lens_dev)  # the scratch now holds the first call's states
+        torch.cuda.synchronize()
+        _close(first, ref, f"first call, plan {dp.plan}")
+        _close(second, ref, f"second call, plan {dp.plan}")
+
+
+def test_noalloc_rejects_plans_larger_than_its_scratch(L):
+    # B=64 rows, G=8, D=128 and 5000 work items need 5000*8*(128+2)*4 bytes of
+    # partial states, more than the 16 MiB array: rejected before any launch.
+    shape = bd.make_shape(64, 64, 8, 128, 16, 8192, 100000)
+    plan = bd.Plan(2, 600, 8, 0)
+    assert bd.workspace_bytes(shape, plan, 5000) > (16 << 20)
+    rc = L.pkv_paged_decode_noalloc(None, None, None, None, None, 16, ctypes.c_float(1.0), None,
+                                    ctypes.byref(shape), ctypes.byref(plan), None, None, 5000, None)
+    assert rc == -3
