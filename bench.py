@@ -81,25 +81,29 @@ def measured_peak():
 
 
 def kernel_source_hash():
+    """Hash of the CUDA sources (the .cu files and the headers they include)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_gqa_17_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        if name.endswith((".cu", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the split kernel from the committed ncu summary,
-    if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of the split kernel from the committed ncu summary
+    (profiles/traffic.txt: `workload kernel_source_hash bytes` per line), if it
+    was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
-            doc = json.load(f)
-        rec = doc.get(workload)
-        if rec and rec.get("kernel_source_hash") == kernel_source_hash():
-            return int(rec["dram_bytes_per_launch"])
-    except (OSError, ValueError, KeyError):
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and not line.startswith("#") and parts[0] == workload:
+                    if parts[1] == kernel_source_hash():
+                        return int(parts[2])
+    except (OSError, ValueError):
         pass
     return None
 
