@@ -61,7 +61,9 @@ typedef enum {
 typedef enum {
     PKV_NO_SPLIT = 0,   /* one block per (row, KV head) covers the whole row; no merge */
     PKV_SPLIT_S = 1,    /* rectangular grid (row, KV head, split); empty splits write the neutral state */
-    PKV_WORK_QUEUE = 2  /* 1D grid over the compact queue of non-empty (row, KV head, chunk) items */
+    PKV_WORK_QUEUE = 2, /* 1D grid over the compact queue of non-empty (row, KV head, chunk) items */
+    PKV_BALANCED = 3    /* the compact queue cut into equal page shares for a fixed grid of T blocks
+                           (one wave on the GPU): each block streams its items back to back */
 } pkv_mode;
 
 /* pkv_plan.flags / pkv_policy_rule.flags */
@@ -97,6 +99,7 @@ typedef struct {
  *   NO_SPLIT:    {0, 1, 0, flags}
  *   SPLIT_S:     {1, S', C, flags}  C = ceil(pages_max / S), S' = ceil(pages_max / C)
  *   WORK_QUEUE:  {2, S', C, flags}  C from the rule,        S' = ceil(pages_max / C)
+ *   BALANCED:    {3, T, 0, flags}   T blocks from the rule's num_splits
  * where pages_max = ceil(N_max / P).  S' is the most chunks any row needs. */
 typedef struct {
     int32_t mode;
@@ -122,7 +125,7 @@ typedef struct {
     int32_t b_lo, b_hi;
     int32_t nmax_lo, nmax_hi;
     int32_t mode;         /* pkv_mode */
-    int32_t num_splits;   /* SPLIT_S: requested S >= 1 */
+    int32_t num_splits;   /* SPLIT_S: requested S >= 1; BALANCED: blocks T >= 1 */
     int32_t chunk_pages;  /* WORK_QUEUE: chunk size C >= 1 in pages */
     int32_t flags;        /* PKV_FLAG_* */
 } pkv_policy_rule;
@@ -182,12 +185,32 @@ PKV_API int pkv_build_work_queue(const int32_t *seq_lens_host, const pkv_shape *
                                  int32_t chunk_pages, pkv_work_item *items, int32_t capacity,
                                  int32_t *indptr, int32_t *n_items);
 
+/* Number of items pkv_build_balanced_queue emits for n_blocks blocks. */
+PKV_API int pkv_balanced_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape,
+                                    int32_t n_blocks, int32_t *n_items);
+
+/* Build the balanced work queue [PKV, Methodology 1 "Compact work queue",
+ * "Row-local bounds"; cut for a fixed grid].  The (row, KV head) pairs are
+ * laid end to end in lexicographic order, ceil(N_i / P) pages each; of the U
+ * pages in total, block b (T = n_blocks) owns pages
+ * [floor(b*U/T), floor((b+1)*U/T)).  Each maximal run of one pair's pages
+ * inside one block's share is an item {row, kv_head, tok_begin, tok_end}
+ * (page-aligned begin, end clipped to N_i); a row with N_i = 0 gets one empty
+ * item per head.  Items are in lexicographic order.  indptr (host int32,
+ * B*H_kv + 1 + n_blocks + 1 entries) receives the pair offsets as in
+ * pkv_build_work_queue, followed by the block offsets: block b owns items
+ * indptr[B*H_kv + 1 + b] .. indptr[B*H_kv + 2 + b].  Capacity errors as in
+ * pkv_build_work_queue. */
+PKV_API int pkv_build_balanced_queue(const int32_t *seq_lens_host, const pkv_shape *shape,
+                                     int32_t n_blocks, pkv_work_item *items, int32_t capacity,
+                                     int32_t *indptr, int32_t *n_items);
+
 /* Closed-form workload counters of `plan` on this batch (host, pure). */
 PKV_API int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape,
                               const pkv_plan *plan, pkv_counters *counters);
 
 /* Device workspace that pkv_paged_decode needs for this shape and plan
- * (n_items: WORK_QUEUE queue length, ignored otherwise).  The workspace holds
+ * (n_items: WORK_QUEUE / BALANCED queue length, ignored otherwise).  The workspace holds
  * a device error word, one completion counter per (row, KV head) pair and the
  * fp32 partial states (m, l, acc) of every split. */
 PKV_API int pkv_workspace_bytes(const pkv_shape *shape, const pkv_plan *plan, int32_t n_items,
@@ -212,7 +235,8 @@ PKV_API int pkv_workspace_status(const void *workspace, void *stream, int32_t *d
  *   block_table  int32 [B][max_pages_per_seq]; entries past a row's last page are never read
  *   seq_lens     int32 [B]; N_i in [0, max_pages_per_seq * P]
  *   out          bf16 [B][H_q][D], contiguous; fully overwritten (rows with N_i = 0 get zeros)
- *   items,indptr WORK_QUEUE only: the queue from pkv_build_work_queue, copied to the device
+ *   items,indptr WORK_QUEUE / BALANCED: the queue from pkv_build_work_queue or
+ *                pkv_build_balanced_queue (indptr with its block offsets), copied to the device
  *   workspace    >= pkv_workspace_bytes(), zeroed once (pkv_workspace_init)
  * page_size must equal shape->page_size; scale multiplies the logits.
  * The split kernel streams whole K/V pages through the block table into

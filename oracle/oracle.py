@@ -27,6 +27,7 @@ from . import build_oracle
 NO_SPLIT = 0
 SPLIT_S = 1
 WORK_QUEUE = 2
+BALANCED = 3  # the compact work queue, cut into equal shares for a fixed number of blocks
 FLAG_SEPARATE_MERGE = 1
 INT32_MAX = 2**31 - 1
 
@@ -225,6 +226,64 @@ def build_work_queue(seq_lens: Sequence[int], H_kv: int, P: int, chunk_pages: in
     return items, indptr
 
 
+def build_balanced_queue(seq_lens: Sequence[int], H_kv: int, P: int, n_blocks: int):
+    """Compact work queue cut into equal shares for `n_blocks` blocks.
+
+    The (row, KV head) pairs are laid end to end in lexicographic order, each
+    contributing ceil(N_i / P) pages; of the U pages in total, block b owns
+    pages [floor(b*U/T), floor((b+1)*U/T)) (T = n_blocks).  Every maximal run
+    of one pair's pages inside one block's share is an item
+    (row, kv_head, tok_begin, tok_end), so items stay row-local and
+    page-aligned [PKV, Methodology 1 "Compact work queue", "Row-local
+    bounds"].  A row with N_i = 0 gets one empty item per head, owned by the
+    last block whose share starts at or before the pair's position.
+
+    Returns (items in lexicographic order, indptr over pairs as in
+    build_work_queue, block_ptr of length T + 1: block b owns items
+    block_ptr[b] .. block_ptr[b+1]).
+    """
+    if n_blocks < 1 or H_kv < 1 or P < 1:
+        raise ValueError("n_blocks, H_kv and P must be positive")
+    lens = [int(n) for n in seq_lens]
+    if any(n < 0 for n in lens):
+        raise ValueError("negative sequence length")
+    T = n_blocks
+    pages = [_ceil_div(n, P) for n in lens]
+    U = H_kv * sum(pages)
+    starts = [(b * U) // T for b in range(T + 1)]
+
+    def owner(u):
+        b = T - 1
+        while starts[b] > u:
+            b -= 1
+        return b
+
+    items, owners, indptr = [], [], [0]
+    u = 0
+    for i, n in enumerate(lens):
+        for h in range(H_kv):
+            if n == 0:
+                items.append((i, h, 0, 0))
+                owners.append(owner(u))
+            else:
+                x = u
+                while x < u + pages[i]:
+                    b = owner(x)
+                    y = min(u + pages[i], starts[b + 1])
+                    items.append((i, h, (x - u) * P, min((y - u) * P, n)))
+                    owners.append(b)
+                    x = y
+            indptr.append(len(items))
+            u += pages[i]
+    block_ptr = [0] * (T + 1)
+    k = 0
+    for b in range(T + 1):
+        while k < len(owners) and owners[k] < b:
+            k += 1
+        block_ptr[b] = k
+    return items, indptr, block_ptr
+
+
 @dataclass(frozen=True)
 class Rule:
     """One row of a policy table: half-open ranges on B and N_max -> a plan."""
@@ -248,6 +307,7 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tup
       NO_SPLIT    -> (0, 1, 0, flags)
       SPLIT_S     -> C = ceil(pages_max / S), S' = ceil(pages_max / C): (1, S', C, flags)
       WORK_QUEUE  -> C from the rule,      S' = ceil(pages_max / C): (2, S', C, flags)
+      BALANCED    -> T blocks from the rule's num_splits:              (3, T, 0, flags)
     where pages_max = ceil(N_max / P).
     """
     if P < 1:
@@ -260,10 +320,10 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tup
     pages_max = _ceil_div(n_max, P)
     chosen = None
     for r in rules:
-        if r.mode not in (NO_SPLIT, SPLIT_S, WORK_QUEUE):
+        if r.mode not in (NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED):
             raise ValueError("unknown mode in policy table")
-        if r.mode == SPLIT_S and r.num_splits < 1:
-            raise ValueError("SPLIT_S rule needs num_splits >= 1")
+        if r.mode in (SPLIT_S, BALANCED) and r.num_splits < 1:
+            raise ValueError("SPLIT_S and BALANCED rules need num_splits >= 1")
         if r.mode == WORK_QUEUE and r.chunk_pages < 1:
             raise ValueError("WORK_QUEUE rule needs chunk_pages >= 1")
         if chosen is None and r.b_lo <= B < r.b_hi and r.nmax_lo <= n_max < r.nmax_hi:
@@ -272,6 +332,8 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tup
         return (NO_SPLIT, 1, 0, 0)
     if chosen.mode == NO_SPLIT:
         return (NO_SPLIT, 1, 0, chosen.flags)
+    if chosen.mode == BALANCED:
+        return (BALANCED, chosen.num_splits, 0, chosen.flags)
     if chosen.mode == SPLIT_S:
         C = _ceil_div(pages_max, chosen.num_splits)
     else:
@@ -285,7 +347,7 @@ def load_rules(path: str) -> List[Rule]:
 
     with open(path) as f:
         doc = json.load(f)
-    names = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE}
+    names = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE, "BALANCED": BALANCED}
     out = []
     for r in doc["rules"]:
         mode = names[r["mode"]] if isinstance(r["mode"], str) else int(r["mode"])
@@ -316,14 +378,15 @@ class Counters:
 def counters(seq_lens: Sequence[int], H_q: int, H_kv: int, D: int, P: int, plan) -> Counters:
     """Closed-form counters for a plan.
 
-    launches: kernels per step (the attention kernel, plus a separate merge
-      kernel when the plan asks for one and some pair has more than one chunk);
+    launches: kernels per step (the attention kernel, plus the merge kernel
+      when a split plan asks for a separate merge);
     work_items: blocks of the attention kernel; empty_items: those that only
       write the neutral state (or a zero output);
     merge_state_bytes: partial states written and read back by the merge,
       2 * slots * G * (D + 2) * 4 over every (row, head) pair with more than one slot;
     kv_bytes: K and V of the valid tokens; kv_bytes_streamed: whole pages;
-    queue_bytes: items (16 B each) plus indptr (4 B per pair, +4) sent to the device;
+    queue_bytes: items (16 B each) plus indptr (4 B per pair, +4; for BALANCED
+      also 4 B per block, +4) sent to the device;
     bucket_launches: exact-length bucketing, one split and one merge launch per
       distinct non-zero length [PKV, Results: "16.00 -> 2.00 launches per step"].
     """
@@ -344,14 +407,22 @@ def counters(seq_lens: Sequence[int], H_q: int, H_kv: int, D: int, P: int, plan)
         empty = H_kv * sum(S - min(S, _ceil_div(p, C)) for p in pages)
         merge = 2 * B * H_kv * S * state if S > 1 else 0
         qbytes = 0
-        launches = 1 + (1 if (flags & FLAG_SEPARATE_MERGE) and S > 1 else 0)
+        launches = 1 + (1 if flags & FLAG_SEPARATE_MERGE else 0)
     elif mode == WORK_QUEUE:
         per_pair = [max(1, _ceil_div(p, C)) for p in pages]
         work = H_kv * sum(per_pair)
         empty = H_kv * sum(1 for n in lens if n == 0)
         merge = 2 * H_kv * sum(k for k in per_pair if k > 1) * state
         qbytes = 16 * work + 4 * (B * H_kv + 1)
-        launches = 1 + (1 if (flags & FLAG_SEPARATE_MERGE) and S > 1 else 0)
+        launches = 1 + (1 if flags & FLAG_SEPARATE_MERGE else 0)
+    elif mode == BALANCED:
+        items, indptr, _ = build_balanced_queue(lens, H_kv, P, S)
+        per_pair = [indptr[k + 1] - indptr[k] for k in range(B * H_kv)]
+        work = S
+        empty = H_kv * sum(1 for n in lens if n == 0)
+        merge = 2 * sum(k for k in per_pair if k > 1) * state
+        qbytes = 16 * len(items) + 4 * (B * H_kv + 1) + 4 * (S + 1)
+        launches = 1 + (1 if flags & FLAG_SEPARATE_MERGE else 0)
     else:
         raise ValueError("unknown mode")
     kv = sum(lens) * H_kv * 2 * D * 2

@@ -16,7 +16,8 @@ _LAZY = {
     "lib", "paged_decode", "plan_decode", "DecodePlan", "Shape", "Plan", "Rule",
     "select_policy", "build_work_queue", "workspace_bytes", "plan_counters",
     "load_rules", "default_rules", "decode_host", "PkvError",
-    "NO_SPLIT", "SPLIT_S", "WORK_QUEUE", "FLAG_SEPARATE_MERGE",
+    "NO_SPLIT", "SPLIT_S", "WORK_QUEUE", "BALANCED", "FLAG_SEPARATE_MERGE", "FLAG_NO_PDL", "FLAG_DEEP_RING",
+    "build_balanced_queue", "paged_decode_noalloc",
 }
 
 

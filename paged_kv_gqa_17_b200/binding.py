@@ -18,10 +18,10 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libpkv.so")
 
-NO_SPLIT, SPLIT_S, WORK_QUEUE = 0, 1, 2
-FLAG_SEPARATE_MERGE = 1
+NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED = 0, 1, 2, 3
+FLAG_SEPARATE_MERGE, FLAG_NO_PDL, FLAG_DEEP_RING = 1, 2, 4
 INT32_MAX = 2**31 - 1
-_MODE_NAMES = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE}
+_MODE_NAMES = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE, "BALANCED": BALANCED}
 
 c_i32, c_i64, c_p, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
 
@@ -80,6 +80,8 @@ SIGNATURES = [
     ("pkv_select_policy", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_p]),
     ("pkv_work_queue_size", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_build_work_queue", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p]),
+    ("pkv_balanced_queue_size", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
+    ("pkv_build_balanced_queue", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p]),
     ("pkv_plan_counters", ctypes.c_int, [c_p, c_p, c_p, c_p]),
     ("pkv_workspace_bytes", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_workspace_init", ctypes.c_int, [c_p, c_sz, c_p]),
@@ -207,6 +209,20 @@ def build_work_queue(seq_lens_host, shape: Shape, chunk_pages: int):
     return items[:n.value], indptr
 
 
+def build_balanced_queue(seq_lens_host, shape: Shape, n_blocks: int):
+    """-> (items int32 [n][4], indptr int32 [B*H_kv + 1 + n_blocks + 1]: pair offsets, then block offsets)."""
+    L = lib()
+    lens, _ = _lens_array(seq_lens_host)
+    n = c_i32(0)
+    _check(L.pkv_balanced_queue_size(lens, ctypes.byref(shape), n_blocks, ctypes.byref(n)),
+           "pkv_balanced_queue_size")
+    items = torch.zeros((max(1, n.value), 4), dtype=torch.int32)
+    indptr = torch.zeros(shape.B * shape.H_kv + 1 + n_blocks + 1, dtype=torch.int32)
+    _check(L.pkv_build_balanced_queue(lens, ctypes.byref(shape), n_blocks, items.data_ptr(), n.value,
+                                      indptr.data_ptr(), ctypes.byref(n)), "pkv_build_balanced_queue")
+    return items[:n.value], indptr
+
+
 def plan_counters(seq_lens_host, shape: Shape, plan: Plan) -> dict:
     L = lib()
     lens, _ = _lens_array(seq_lens_host)
@@ -249,8 +265,11 @@ def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[
         plan = select_policy(seq_lens_host, shape, rules)
     items = indptr = None
     n_items = 0
-    if plan.mode == WORK_QUEUE:
-        items_h, indptr_h = build_work_queue(seq_lens_host, shape, plan.chunk_pages)
+    if plan.mode in (WORK_QUEUE, BALANCED):
+        if plan.mode == WORK_QUEUE:
+            items_h, indptr_h = build_work_queue(seq_lens_host, shape, plan.chunk_pages)
+        else:
+            items_h, indptr_h = build_balanced_queue(seq_lens_host, shape, plan.num_splits)
         n_items = int(items_h.shape[0])
         items = items_h.to(device)
         indptr = indptr_h.to(device)

@@ -11,6 +11,7 @@
 #include <climits>
 #include <cstring>
 #include <unordered_set>
+#include <vector>
 
 #include "pkv_internal.h"
 
@@ -56,9 +57,9 @@ int check_rules(const pkv_policy_rule *rules, int32_t n)
         return PKV_ERR_INVALID;
     for (int32_t k = 0; k < n; ++k) {
         const pkv_policy_rule &r = rules[k];
-        if (r.mode != PKV_NO_SPLIT && r.mode != PKV_SPLIT_S && r.mode != PKV_WORK_QUEUE)
+        if (r.mode != PKV_NO_SPLIT && r.mode != PKV_SPLIT_S && r.mode != PKV_WORK_QUEUE && r.mode != PKV_BALANCED)
             return PKV_ERR_INVALID;
-        if (r.mode == PKV_SPLIT_S && r.num_splits < 1)
+        if ((r.mode == PKV_SPLIT_S || r.mode == PKV_BALANCED) && r.num_splits < 1)
             return PKV_ERR_INVALID;
         if (r.mode == PKV_WORK_QUEUE && r.chunk_pages < 1)
             return PKV_ERR_INVALID;
@@ -135,6 +136,10 @@ int pkv_select_policy(const int32_t *seq_lens_host, const pkv_shape *shape,
         *plan = {PKV_NO_SPLIT, 1, 0, chosen->flags};
         return PKV_OK;
     }
+    if (chosen->mode == PKV_BALANCED) {
+        *plan = {PKV_BALANCED, chosen->num_splits, 0, chosen->flags};
+        return PKV_OK;
+    }
     const int64_t C = chosen->mode == PKV_SPLIT_S ? ceil_div(pages_max, chosen->num_splits)
                                                   : (int64_t)chosen->chunk_pages;
     *plan = {chosen->mode, (int32_t)ceil_div(pages_max, C), (int32_t)C, chosen->flags};
@@ -189,6 +194,103 @@ int pkv_build_work_queue(const int32_t *seq_lens_host, const pkv_shape *shape, i
     return PKV_OK;
 }
 
+}  // extern "C"
+
+namespace pkv {
+namespace {
+
+// Walks the balanced queue of a batch; calls emit(row, kv_head, tok_begin,
+// tok_end, block) for every item in order.  Returns the item count.
+template <typename Emit>
+int64_t walk_balanced(const int32_t *lens, const pkv_shape &s, int32_t T, Emit emit)
+{
+    const int64_t P = s.page_size;
+    int64_t U = 0;
+    for (int32_t i = 0; i < s.B; ++i)
+        U += ceil_div(lens[i], P);
+    U *= s.H_kv;
+    // last block whose share starts at or before page u
+    auto owner = [&](int64_t u, int64_t hint) {
+        int64_t b = hint;
+        while (b + 1 < T && balanced_start(U, T, b + 1) <= u)
+            ++b;
+        return b;
+    };
+    int64_t n = 0, u = 0, b = 0;
+    for (int32_t i = 0; i < s.B; ++i) {
+        const int64_t N = lens[i];
+        const int64_t pg = ceil_div(N, P);
+        for (int32_t h = 0; h < s.H_kv; ++h) {
+            if (N == 0) {
+                b = owner(u, b);
+                emit(i, h, 0, 0, b);
+                ++n;
+            }
+            for (int64_t x = u; x < u + pg;) {
+                b = owner(x, b);
+                const int64_t y = std::min(u + pg, balanced_start(U, T, b + 1));
+                emit(i, h, (x - u) * P, std::min((y - u) * P, N), b);
+                ++n;
+                x = y;
+            }
+            u += pg;
+        }
+    }
+    return n;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+int pkv_balanced_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape, int32_t n_blocks,
+                            int32_t *n_items)
+{
+    if (!n_items || n_blocks < 1 || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    int rc = check_lens(seq_lens_host, shape->B);
+    if (rc != PKV_OK)
+        return rc;
+    const int64_t n = walk_balanced(seq_lens_host, *shape, n_blocks, [](int32_t, int32_t, int64_t, int64_t, int64_t) {});
+    if (n > INT32_MAX)
+        return PKV_ERR_CAPACITY;
+    *n_items = (int32_t)n;
+    return PKV_OK;
+}
+
+int pkv_build_balanced_queue(const int32_t *seq_lens_host, const pkv_shape *shape, int32_t n_blocks,
+                             pkv_work_item *items, int32_t capacity, int32_t *indptr, int32_t *n_items)
+{
+    int32_t need = 0;
+    int rc = pkv_balanced_queue_size(seq_lens_host, shape, n_blocks, &need);
+    if (rc != PKV_OK)
+        return rc;
+    *n_items = need;
+    if (capacity < need)
+        return PKV_ERR_CAPACITY;
+    if ((need > 0 && !items) || !indptr)
+        return PKV_ERR_INVALID;
+    const int64_t pairs = (int64_t)shape->B * shape->H_kv;
+    int32_t *pair_ptr = indptr;
+    int32_t *block_ptr = indptr + pairs + 1;
+    int32_t k = 0;
+    int64_t last_pair = -1, next_block = 0;
+    walk_balanced(seq_lens_host, *shape, n_blocks, [&](int32_t i, int32_t h, int64_t tb, int64_t te, int64_t b) {
+        const int64_t pair = (int64_t)i * shape->H_kv + h;
+        while (last_pair < pair)
+            pair_ptr[++last_pair] = k;
+        while (next_block <= b)
+            block_ptr[next_block++] = k;
+        items[k++] = {i, h, (int32_t)tb, (int32_t)te};
+    });
+    while (last_pair < pairs)
+        pair_ptr[++last_pair] = k;
+    while (next_block <= n_blocks)
+        block_ptr[next_block++] = k;
+    return PKV_OK;
+}
+
 int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, const pkv_plan *plan,
                       pkv_counters *c)
 {
@@ -222,7 +324,7 @@ int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, cons
     case PKV_SPLIT_S: {
         if (S < 1 || C < 1)
             return PKV_ERR_INVALID;
-        out.launches = 1 + (separate && S > 1);
+        out.launches = 1 + separate;
         out.work_items = B * H_kv * S;
         int64_t empty = 0;
         for (int64_t i = 0; i < B; ++i)
@@ -234,7 +336,7 @@ int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, cons
     case PKV_WORK_QUEUE: {
         if (C < 1)
             return PKV_ERR_INVALID;
-        out.launches = 1 + (separate && S > 1);
+        out.launches = 1 + separate;
         int64_t items = 0, multi = 0;
         for (int64_t i = 0; i < B; ++i) {
             const int64_t k = std::max<int64_t>(1, ceil_div(ceil_div(seq_lens_host[i], P), C));
@@ -246,6 +348,25 @@ int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, cons
         out.empty_items = H_kv * zero_rows;
         out.merge_state_bytes = 2 * H_kv * multi * state;
         out.queue_bytes = 16 * out.work_items + 4 * (B * H_kv + 1);
+        break;
+    }
+    case PKV_BALANCED: {
+        if (S < 1)
+            return PKV_ERR_INVALID;
+        out.launches = 1 + separate;
+        out.work_items = S;
+        out.empty_items = H_kv * zero_rows;
+        std::vector<int32_t> per_pair((size_t)(B * H_kv), 0);
+        const int64_t n = walk_balanced(seq_lens_host, *shape, (int32_t)S,
+                                        [&](int32_t i, int32_t h, int64_t, int64_t, int64_t) {
+                                            ++per_pair[(size_t)((int64_t)i * H_kv + h)];
+                                        });
+        int64_t multi = 0;
+        for (int32_t k : per_pair)
+            if (k > 1)
+                multi += k;
+        out.merge_state_bytes = 2 * multi * state;
+        out.queue_bytes = 16 * n + 4 * (B * H_kv + 1) + 4 * (S + 1);
         break;
     }
     default:

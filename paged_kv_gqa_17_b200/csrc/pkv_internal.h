@@ -39,7 +39,7 @@ inline WsLayout ws_layout(const pkv_shape &s, const pkv_plan &p, int32_t n_items
     const int64_t G = s.H_kv > 0 ? s.H_q / s.H_kv : 0;
     if (p.mode == PKV_SPLIT_S)
         w.n_slots = pairs * p.num_splits;
-    else if (p.mode == PKV_WORK_QUEUE)
+    else if (p.mode == PKV_WORK_QUEUE || p.mode == PKV_BALANCED)
         w.n_slots = n_items;
     size_t off = kWsAlign;  // error word section
     w.counters_off = off;
@@ -57,5 +57,9 @@ inline WsLayout ws_layout(const pkv_shape &s, const pkv_plan &p, int32_t n_items
 // Shape checks shared by the host entry points; PKV_OK when the shape is
 // well formed (fast-path support is checked separately by the decode call).
 int check_shape(const pkv_shape *s);
+
+// Balanced queue: block b owns pages [floor(b*U/T), floor((b+1)*U/T)) of
+// the U pages of all (row, KV head) pairs laid end to end.
+inline int64_t balanced_start(int64_t U, int64_t T, int64_t b) { return (b * U) / T; }
 
 }  // namespace pkv

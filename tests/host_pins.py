@@ -129,12 +129,14 @@ def policy_semantics(O):
     # B = 8 misses [2, 8) and falls to the catch-all
     assert O.select_policy([100] * 8, P, rules) == (O.WORK_QUEUE, 1, 8, 0)
     assert O.select_policy([1000, 5] * 2, P, rules) == (O.WORK_QUEUE, 3, 24, 1)
+    # a balanced rule takes its block count as given
+    assert O.select_policy([5000, 7], P, [R(0, 9, 0, O.INT32_MAX, 3, num_splits=296, flags=4)]) == (3, 296, 0, 4)
     # no rule matches -> single kernel; empty batch and all-empty rows -> single kernel
     assert O.select_policy([10], P, rules[:1]) == (O.NO_SPLIT, 1, 0, 0)
     assert O.select_policy([], P, rules) == (O.NO_SPLIT, 1, 0, 0)
     assert O.select_policy([0, 0], P, rules) == (O.NO_SPLIT, 1, 0, 0)
     for bad in ([R(0, 9, 0, 9, 7)], [R(0, 9, 0, 9, O.SPLIT_S, num_splits=0)],
-                [R(0, 9, 0, 9, O.WORK_QUEUE, chunk_pages=0)]):
+                [R(0, 9, 0, 9, O.WORK_QUEUE, chunk_pages=0)], [R(0, 9, 0, 9, 3, num_splits=0)]):
         try:
             O.select_policy([5], P, bad)
         except ValueError:
@@ -181,8 +183,89 @@ def merge_state_closed(O):
         assert wq.kv_bytes == rect.kv_bytes == sum(lens) * H_kv * 4 * D
 
 
+def _balanced_cases(seed=11, n=25):
+    rng = random.Random(seed)
+    fixed = [([32768], 8, 16, 296), ([32768], 8, 16, 37), ([0, 0], 2, 16, 5), ([5], 1, 16, 8), ([], 4, 16, 3),
+             ([100, 0, 3000, 17], 8, 16, 296), ([1, 1, 1], 3, 16, 1)]
+    yield from fixed
+    for _ in range(n):
+        B = rng.randint(1, 9)
+        lens = [rng.choice([0, rng.randint(1, 40), rng.randint(1, 5000)]) for _ in range(B)]
+        yield lens, rng.randint(1, 8), rng.choice([8, 16]), rng.randint(1, 300)
+
+
+def balanced_shares(O):
+    """Closed form: block b streams exactly floor((b+1)U/T) - floor(bU/T) pages,
+    which is floor(U/T) or ceil(U/T)."""
+    for lens, H_kv, P, T in _balanced_cases():
+        items, indptr, bptr = O.build_balanced_queue(lens, H_kv, P, T)
+        U = H_kv * sum(_cdiv(n, P) for n in lens)
+        assert len(bptr) == T + 1 and bptr[0] == 0 and bptr[-1] == len(items), ("balanced_shares", lens, T)
+        for b in range(T):
+            got = sum(_cdiv(e, P) - bg // P for (_, _, bg, e) in items[bptr[b]:bptr[b + 1]] if e > bg)
+            want = ((b + 1) * U) // T - (b * U) // T
+            assert got == want and U // T <= got <= _cdiv(U, T), ("balanced_shares", lens, T, b, got, want)
+
+
+def balanced_cover(O):
+    for lens, H_kv, P, T in _balanced_cases(12):
+        items, indptr, bptr = O.build_balanced_queue(lens, H_kv, P, T)
+        assert len(indptr) == len(lens) * H_kv + 1
+        for i, n in enumerate(lens):
+            for h in range(H_kv):
+                pair = items[indptr[i * H_kv + h]:indptr[i * H_kv + h + 1]]
+                assert all(it[0] == i and it[1] == h for it in pair), "balanced_cover: wrong pair"
+                if n == 0:
+                    assert pair == [(i, h, 0, 0)], "balanced_cover: empty row"
+                    continue
+                pos = 0
+                for (_, _, b, e) in pair:
+                    assert b == pos and e > b and b % P == 0, ("balanced_cover", lens, T, pair)
+                    pos = e
+                assert pos == n, ("balanced_cover: gap", lens, T)
+
+
+def _small_balanced_cases(seed=13, n=25):
+    rng = random.Random(seed)
+    yield from [([0, 0], 2, 16, 5), ([5], 1, 16, 8), ([], 4, 16, 3), ([100, 0, 300, 17], 4, 16, 40), ([1, 1, 1], 3, 16, 1)]
+    for _ in range(n):
+        B = rng.randint(1, 5)
+        lens = [rng.choice([0, rng.randint(1, 40), rng.randint(1, 600)]) for _ in range(B)]
+        yield lens, rng.randint(1, 4), rng.choice([8, 16]), rng.randint(1, 64)
+
+
+def balanced_bruteforce(O):
+    """Assign every page on its own to the block whose share holds it (found by
+    scanning all blocks), then group runs of one pair inside one block."""
+    for lens, H_kv, P, T in _small_balanced_cases():
+        items, indptr, bptr = O.build_balanced_queue(lens, H_kv, P, T)
+        U = H_kv * sum(_cdiv(n, P) for n in lens)
+        owner_of_page = []
+        for u in range(U):
+            owner_of_page.append([b for b in range(T) if (b * U) // T <= u < ((b + 1) * U) // T][0])
+        want, want_owner, u = [], [], 0
+        for i, n in enumerate(lens):
+            for h in range(H_kv):
+                pg = _cdiv(n, P)
+                if n == 0:
+                    want.append((i, h, 0, 0))
+                    want_owner.append(max(b for b in range(T) if (b * U) // T <= u))
+                for j in range(pg):
+                    b = owner_of_page[u + j]
+                    if j > 0 and want_owner[-1] == b and want[-1][:2] == (i, h):
+                        r = want[-1]
+                        want[-1] = (i, h, r[2], min((j + 1) * P, n))
+                    else:
+                        want.append((i, h, j * P, min((j + 1) * P, n)))
+                        want_owner.append(b)
+                u += pg
+        assert items == want, ("balanced_bruteforce", lens, H_kv, P, T)
+        got_owner = [b for b in range(T) for _ in range(bptr[b + 1] - bptr[b])]
+        assert got_owner == want_owner, ("balanced_bruteforce owners", lens, T)
+
+
 HOST_PINS = (queue_closed_form, queue_cover, queue_bruteforce, policy_paper, policy_semantics,
-             launch_fanout, merge_state_closed)
+             launch_fanout, merge_state_closed, balanced_shares, balanced_cover, balanced_bruteforce)
 
 
 def run_all(O):

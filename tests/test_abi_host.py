@@ -100,10 +100,21 @@ def test_work_queue_matches_oracle_bit_exactly(L):
             assert indptr.tolist() == w_indptr
 
 
+def test_balanced_queue_matches_oracle_bit_exactly(L):
+    for lens, H_kv, G, D in _cases(4):
+        shape = _shape(lens, H_kv, G, D)
+        for T in (1, 3, 37, 296):
+            items, indptr = bd.build_balanced_queue(lens, shape, T)
+            w_items, w_indptr, w_bptr = O.build_balanced_queue(lens, H_kv, 16, T)
+            assert [tuple(x) for x in items.tolist()] == w_items, (lens, T)
+            assert indptr.tolist() == w_indptr + w_bptr, (lens, T)
+
+
 def test_counters_match_oracle(L):
     for lens, H_kv, G, D in _cases(3):
         shape = _shape(lens, H_kv, G, D)
-        for rules in ([bd.Rule(0, 2**31 - 1, 0, 2**31 - 1, m, 5, 7, f) for m, f in ((0, 0), (1, 0), (1, 1), (2, 0), (2, 1))]):
+        for rules in ([bd.Rule(0, 2**31 - 1, 0, 2**31 - 1, m, 5, 7, f)
+                       for m, f in ((0, 0), (1, 0), (1, 1), (2, 0), (2, 1), (3, 0), (3, 1))]):
             plan = bd.select_policy(lens, shape, [rules])
             got = bd.plan_counters(lens, shape, plan)
             want = O.counters(lens, H_kv * G, H_kv, D, 16, plan.tuple()).__dict__
@@ -172,6 +183,16 @@ def test_host_pins_hold_for_the_c_planner(L):
             shape = bd.make_shape(len(lens), H_kv, H_kv, 64, P, 1, 1)
             items, indptr = bd.build_work_queue(lens, shape, C)
             return [tuple(x) for x in items.tolist()], indptr.tolist()
+
+        @staticmethod
+        def build_balanced_queue(lens, H_kv, P, T):
+            if T < 1:
+                raise ValueError
+            shape = bd.make_shape(len(lens), H_kv, H_kv, 64, P, 1, 1)
+            items, indptr = bd.build_balanced_queue(lens, shape, T)
+            ptr = indptr.tolist()
+            pairs = len(lens) * H_kv
+            return [tuple(x) for x in items.tolist()], ptr[:pairs + 1], ptr[pairs + 1:]
 
         @staticmethod
         def select_policy(lens, P, rules):

@@ -8,7 +8,6 @@ the GPU or the CUDA library.
 import os
 import subprocess
 import sys
-import types
 
 import pytest
 
@@ -45,6 +44,10 @@ PY_MUTANTS = {
                                   "return (chosen.mode, chosen.num_splits if chosen.mode == SPLIT_S else _ceil_div(pages_max, C), C, chosen.flags)"),
     "bucket launches count rows": ("2 * distinct)", "2 * B)"),
     "merge traffic counts single-chunk pairs": ("sum(k for k in per_pair if k > 1)", "sum(per_pair)"),
+    "balanced owner off by one": ("        while starts[b] > u:", "        while starts[b] >= u and b > 0:"),
+    "balanced share rounded up": ("starts = [(b * U) // T for b in range(T + 1)]",
+                                  "starts = [min(U, -(-(b * U) // T)) for b in range(T + 1)]"),
+    "balanced item not clipped to row": ("min((y - u) * P, n)", "(y - u) * P"),
 }
 
 
@@ -77,17 +80,33 @@ def test_c_oracle_mutant_is_caught(tmp_path, name):
     assert r.returncode != 0, f"planted mistake {name!r} passed every pin:\n{r.stdout}"
 
 
+_PY_RUNNER = """
+import sys, types
+sys.path.insert(0, {root!r})
+from tests import host_pins
+mod = types.ModuleType("oracle._mutant")
+mod.__dict__["__package__"] = "oracle"
+sys.modules[mod.__name__] = mod  # dataclasses look their module up here
+exec(compile(open({path!r}).read(), "oracle_mutant.py", "exec"), mod.__dict__)
+failed = host_pins.run_all(mod)
+print("FAILED_PINS", len(failed))
+sys.exit(3 if failed else 0)
+"""
+
+
 @pytest.mark.parametrize("name", sorted(PY_MUTANTS))
-def test_py_oracle_mutant_is_caught(name):
+def test_py_oracle_mutant_is_caught(tmp_path, name):
+    """Each mutant runs in its own process with a time limit: a mutant that
+    never finishes (a loop that stops advancing) counts as caught."""
     old, new = PY_MUTANTS[name]
     src = open(os.path.join(ORACLE_DIR, "oracle.py")).read()
     assert old in src, f"mutation site for {name!r} not found"
-    mod = types.ModuleType("oracle._mutant")
-    mod.__dict__["__package__"] = "oracle"
-    sys.modules[mod.__name__] = mod  # dataclasses look their module up here
+    path = tmp_path / "oracle_mutant.py"
+    path.write_text(src.replace(old, new))
+    root = os.path.dirname(HERE)
     try:
-        exec(compile(src.replace(old, new), "oracle_mutant.py", "exec"), mod.__dict__)
-        failed = host_pins.run_all(mod)
-    finally:
-        del sys.modules[mod.__name__]
-    assert failed, f"planted mistake {name!r} passed every pin"
+        r = subprocess.run([sys.executable, "-c", _PY_RUNNER.format(root=root, path=str(path))],
+                           capture_output=True, text=True, timeout=30)
+    except subprocess.TimeoutExpired:
+        return
+    assert r.returncode != 0, f"planted mistake {name!r} passed every pin:\n{r.stdout}"
