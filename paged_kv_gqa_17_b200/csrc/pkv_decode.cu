@@ -209,6 +209,12 @@ __device__ __forceinline__ void grid_launch_dependents()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Barrier among the first `threads` threads of the block (named barrier `id`).
+__device__ __forceinline__ void named_barrier(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *tm)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
@@ -353,6 +359,109 @@ __device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslot
     }
 }
 
+// Attention over one 16-token page in ring stage (ks_base, vs_base) for the
+// G heads of one KV head: S^T = K Q^T on the tensor cores, the stage handed
+// back to the producer as soon as the K/V fragments are in registers, the
+// online-softmax update of (m, l, o) in the log2 domain with tokens >= nvalid
+// masked, and O^T += V^T P^T.
+template <int D, int NT>
+__device__ __forceinline__ void attend_page(uint8_t *smem, uint32_t sbase, uint32_t ks_base, uint32_t vs_base,
+                                            uint32_t bar_empty_s, int nvalid, int lane, int r, int ri,
+                                            uint32_t k_off, int k_hi, uint32_t v_off, int v_hi, float sl2,
+                                            const uint32_t (&qf)[D / 16][NT][2], float (&m_run)[NT][2],
+                                            float (&l_run)[NT][2], float (&o)[D / 16][NT][4])
+{
+    constexpr int kHalves = D / kBoxD;
+    if (nvalid < kPage) {
+        // Tail page: zero V rows past the row's end, so that stale or
+        // NaN slots cannot leak through P = 0 in the PV product.
+        uint8_t *vs = smem + (vs_base - sbase);
+        const int dead = kPage - nvalid;
+        for (int i = lane; i < dead * kHalves * 8; i += 32) {
+            const int rr = i >> 3;
+            const int hf = rr / dead;
+            const int t = nvalid + rr % dead;
+            *reinterpret_cast<uint4 *>(vs + hf * kBoxBytes + t * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+    }
+    // S^T[t][g] = K[t] . q[g]
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+        sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        const int chunk = (((ks & 3) << 1) + k_hi) ^ ri;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(ks_base + (ks >> 2) * kBoxBytes + k_off + (chunk << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            mma_bf16(sacc[nt], a0, a1, a2, a3, qf[ks][nt][0], qf[ks][nt][1]);
+    }
+    // V^T fragments to registers, then hand the stage back to the
+    // producer before the softmax and PV math.
+    uint32_t vf[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        const int chunk = (((mt & 3) << 1) + v_hi) ^ ri;
+        ldsm_x4_trans(vs_base + (mt >> 2) * kBoxBytes + v_off + (chunk << 4), vf[mt][0], vf[mt][1],
+                      vf[mt][2], vf[mt][3]);
+    }
+    __syncwarp();
+    if (nvalid < kPage)
+        fence_proxy_async_smem();  // our zero stores precede the next TMA write of this stage
+    if (lane == 0)
+        mbar_arrive(bar_empty_s);  // release: orders the fragment loads before the refill
+    // Online softmax over this page (log2 domain), tokens past the end masked.
+    const bool lo_ok = r < nvalid;
+    const bool hi_ok = r + 8 < nvalid;
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const float x0 = lo_ok ? sacc[nt][0] * sl2 : -INFINITY;
+        const float x1 = lo_ok ? sacc[nt][1] * sl2 : -INFINITY;
+        const float x2 = hi_ok ? sacc[nt][2] * sl2 : -INFINITY;
+        const float x3 = hi_ok ? sacc[nt][3] * sl2 : -INFINITY;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int sh = 4; sh < 32; sh <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
+        }
+        const float mn0 = fmaxf(m_run[nt][0], mx0);
+        const float mn1 = fmaxf(m_run[nt][1], mx1);
+        const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = exp2_approx(m_run[nt][0] - mu0);
+        const float al1 = exp2_approx(m_run[nt][1] - mu1);
+        const float p0 = exp2_approx(x0 - mu0);
+        const float p1 = exp2_approx(x1 - mu1);
+        const float p2 = exp2_approx(x2 - mu0);
+        const float p3 = exp2_approx(x3 - mu1);
+        l_run[nt][0] = fmaf(l_run[nt][0], al0, p0 + p2);
+        l_run[nt][1] = fmaf(l_run[nt][1], al1, p1 + p3);
+        m_run[nt][0] = mn0;
+        m_run[nt][1] = mn1;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            o[mt][nt][0] *= al0;
+            o[mt][nt][1] *= al1;
+            o[mt][nt][2] *= al0;
+            o[mt][nt][3] *= al1;
+        }
+        // P^T as the B operand (k = token, n = head): transpose the two 8x8 halves.
+        pb[nt][0] = movmatrix_trans(pack_bf16(p0, p1));
+        pb[nt][1] = movmatrix_trans(pack_bf16(p2, p3));
+    }
+    // O^T[d][g] += V^T[d][t] P^T[t][g]
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+}
+
 // Merge of one (row, KV head)'s n partial states by the block that finished
 // it last, staged through the idle shared-memory ring.  The weights
 // w_s = 2^(m_s - M) (M = max_s m_s, 0 for a neutral state) and the
@@ -362,7 +471,7 @@ __device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslot
 // Returns false when the ring cannot hold the weights plus two slots.
 template <int D, int NT, int NW, int NST>
 __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0, int row, int h, int slot0, int n,
-                                  int tid)
+                                  int tid, uint32_t (&uses)[2])
 {
     using C = Cfg<D, NT, NW, NST>;
     const int G = p.G;
@@ -421,7 +530,7 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
     for (int k = 0; k < C::kMaxMergeTasks; ++k)
         O[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int ch = 0; ch < nch; ++ch) {
-        mbar_wait(mbar0 + 8 * (ch & 1), (ch >> 1) & 1, p.ws_error);
+        mbar_wait(mbar0 + 8 * (ch & 1), (uses[ch & 1] + (ch >> 1)) & 1, p.ws_error);
         const float *st = reinterpret_cast<const float *>(smem + wbytes + (ch & 1) * half);
         const int first = ch * hs;
         const int cnt = min(hs, n - first);
@@ -466,6 +575,8 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
             store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O[k], inv));
         }
     }
+    uses[0] += (nch + 1) / 2;  // barrier 0 carried the even chunks, barrier 1 the odd ones
+    uses[1] += nch / 2;
     return true;
 }
 
@@ -704,96 +815,10 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             const uint32_t vs_base = v_ring + s * C::kStageBytes;
             const int tok0 = (pg0 + pidx) * kPage;
             const int nvalid = te - tok0 < kPage ? te - tok0 : kPage;
-            if (nvalid < kPage) {
-                // Tail page: zero V rows past the row's end, so that stale or
-                // NaN slots cannot leak through P = 0 in the PV product.
-                uint8_t *vs = smem + (vs_base - sbase);
-                const int dead = kPage - nvalid;
-                for (int i = lane; i < dead * C::kHalves * 8; i += 32) {
-                    const int rr = i >> 3;
-                    const int hf = rr / dead;
-                    const int t = nvalid + rr % dead;
-                    *reinterpret_cast<uint4 *>(vs + hf * kBoxBytes + t * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-                }
-                __syncwarp();
-            }
-            // S^T[t][g] = K[t] . q[g]
-            float sacc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const int chunk = (((ks & 3) << 1) + k_hi) ^ ri;
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(ks_base + (ks >> 2) * kBoxBytes + k_off + (chunk << 4), a0, a1, a2, a3);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_bf16(sacc[nt], a0, a1, a2, a3, qf[ks][nt][0], qf[ks][nt][1]);
-            }
-            // V^T fragments to registers, then hand the stage back to the
-            // producer before the softmax and PV math.
-            uint32_t vf[D / 16][4];
-#pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                const int chunk = (((mt & 3) << 1) + v_hi) ^ ri;
-                ldsm_x4_trans(vs_base + (mt >> 2) * kBoxBytes + v_off + (chunk << 4), vf[mt][0], vf[mt][1],
-                              vf[mt][2], vf[mt][3]);
-            }
-            __syncwarp();
-            if (nvalid < kPage)
-                fence_proxy_async_smem();  // our zero stores precede the next TMA write of this stage
-            if (lane == 0)
-                mbar_arrive(bar_empty + 8 * s);  // release: orders the fragment loads before the refill
+            attend_page<D, NT>(smem, sbase, ks_base, vs_base, bar_empty + 8 * s, nvalid, lane, r, ri, k_off, k_hi,
+                               v_off, v_hi, sl2, qf, m_run, l_run, o);
             if (pidx == 0)
                 PKV_TRACE_POINT(2);
-            // Online softmax over this page (log2 domain), tokens past the end masked.
-            const bool lo_ok = r < nvalid;
-            const bool hi_ok = r + 8 < nvalid;
-            uint32_t pb[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float x0 = lo_ok ? sacc[nt][0] * sl2 : -INFINITY;
-                const float x1 = lo_ok ? sacc[nt][1] * sl2 : -INFINITY;
-                const float x2 = hi_ok ? sacc[nt][2] * sl2 : -INFINITY;
-                const float x3 = hi_ok ? sacc[nt][3] * sl2 : -INFINITY;
-                float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-                for (int sh = 4; sh < 32; sh <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
-                }
-                const float mn0 = fmaxf(m_run[nt][0], mx0);
-                const float mn1 = fmaxf(m_run[nt][1], mx1);
-                const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-                const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-                const float al0 = exp2_approx(m_run[nt][0] - mu0);
-                const float al1 = exp2_approx(m_run[nt][1] - mu1);
-                const float p0 = exp2_approx(x0 - mu0);
-                const float p1 = exp2_approx(x1 - mu1);
-                const float p2 = exp2_approx(x2 - mu0);
-                const float p3 = exp2_approx(x3 - mu1);
-                l_run[nt][0] = fmaf(l_run[nt][0], al0, p0 + p2);
-                l_run[nt][1] = fmaf(l_run[nt][1], al1, p1 + p3);
-                m_run[nt][0] = mn0;
-                m_run[nt][1] = mn1;
-#pragma unroll
-                for (int mt = 0; mt < D / 16; ++mt) {
-                    o[mt][nt][0] *= al0;
-                    o[mt][nt][1] *= al1;
-                    o[mt][nt][2] *= al0;
-                    o[mt][nt][3] *= al1;
-                }
-                // P^T as the B operand (k = token, n = head): transpose the two 8x8 halves.
-                pb[nt][0] = movmatrix_trans(pack_bf16(p0, p1));
-                pb[nt][1] = movmatrix_trans(pack_bf16(p2, p3));
-            }
-            // O^T[d][g] += V^T[d][t] P^T[t][g]
-#pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
         }
 #ifdef PKV_TRACE
         if (tid == 0 && blockIdx.x < kTraceBlocks) {
@@ -880,12 +905,311 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         }
         __syncthreads();
         if (misc[0]) {
-            if (!merge_pair_staged<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid))
+            uint32_t uses[2] = {0, 0};
+            if (!merge_pair_staged<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid,
+                                                   uses))
                 merge_pair<D>(p, row, h, slot0, nslots, tid, C::kThreads);
             if (tid == 0)
                 p.ws_counters[pair] = 0u;  // ready for the next call
             PKV_TRACE_POINT(5);
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Balanced persistent grid: block b streams the items of its equal page share
+// (the balanced queue) back to back through one ring.  The producer never
+// stops at item boundaries; the consumer warps close each item with a combine
+// in a dedicated buffer, and the merges this block owns (it was the last to
+// finish a pair) run at the end, when the ring is idle.
+
+template <int D, int NT, int NW, int NST>
+struct BCfg {
+    using Base = Cfg<D, NT, NW, NST>;
+    static constexpr int kThreads = Base::kThreads;
+    static constexpr int kStageBytes = Base::kStageBytes;
+    static constexpr int kRingBytes = Base::kRingBytes;
+    static constexpr int kGP = Base::kGP;
+    static constexpr int kOStride = Base::kOStride;
+    static constexpr int kCombOff = kRingBytes;
+    static constexpr int kCombBytes = NW * kGP * (kOStride + 2) * 4;
+    static constexpr int kBarOff = (kCombOff + kCombBytes + 63) / 64 * 64;
+    static constexpr int kMiscOff = kBarOff + 2 * NST * 8;  // flags, two merge mbarriers, deferred merges
+    static constexpr int kMaxDeferred = 32;
+    static constexpr int kListOff = kMiscOff + 64;
+    static constexpr int kSmemBytes = kListOff + 16 * kMaxDeferred + 1024;
+};
+
+// Page range of one balanced-queue item; false (and no pages) for an item
+// that does not describe a valid range of a valid (row, KV head).
+__device__ __forceinline__ bool item_pages(const Params &p, const int4 &it, int &pg0, int &np)
+{
+    const int64_t row_cap = (int64_t)p.max_pages * kPage;
+    const bool ok = it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w &&
+                    it.w <= row_cap && (it.z % kPage) == 0;
+    pg0 = ok ? it.z / kPage : 0;
+    np = ok && it.w > it.z ? (it.w + kPage - 1) / kPage - pg0 : 0;
+    return ok;
+}
+
+template <int D, int NT, int NW, int NST>
+__global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_constant__ Params p)
+{
+    using C = BCfg<D, NT, NW, NST>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t k_ring = sbase;
+    const uint32_t v_ring = sbase + NST * C::kStageBytes;
+    const uint32_t bar_full = sbase + C::kBarOff;
+    const uint32_t bar_empty = bar_full + NST * 8;
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + C::kMiscOff);  // [0] deferred count, [1] merge now
+    int4 *deferred = reinterpret_cast<int4 *>(smem + C::kListOff);
+    float *cb_o = reinterpret_cast<float *>(smem + C::kCombOff);
+    float *cb_m = cb_o + NW * C::kGP * C::kOStride;
+    float *cb_l = cb_m + NW * C::kGP;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    constexpr int kConsumers = NW * 32;
+    grid_dependency_wait();
+
+    const int pairs = p.B * p.H_kv;
+    const int32_t *block_ptr = p.indptr + pairs + 1;
+    const int it0 = __ldg(block_ptr + blockIdx.x);
+    const int it1 = __ldg(block_ptr + blockIdx.x + 1);
+    if (it0 < 0 || it1 < it0 || it1 > p.n_items) {
+        if (tid == 0)
+            atomicOr(p.ws_error, kErrItem);
+        return;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(sbase + C::kMiscOff + 8, 1);
+        mbar_init(sbase + C::kMiscOff + 16, 1);
+        misc[0] = 0;
+        misc[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+    }
+    __syncthreads();
+
+    const int r = lane >> 2;
+    const int c4 = lane & 3;
+    if (warp == NW) {
+        // ================= producer =================
+        const uint64_t policy = evict_first_policy();
+        int gp = 0;
+        bool ok = true;
+        for (int it = it0; it < it1 && ok; ++it) {
+            const int4 item = __ldg(p.items + it);
+            int pg0, np;
+            if (!item_pages(p, item, pg0, np) && lane == 0)
+                atomicOr(p.ws_error, kErrItem);
+            const int32_t *bt = p.block_table + (int64_t)item.x * p.max_pages + pg0;
+            for (int base = 0; base < np && ok; base += 32) {
+                int e = base + lane < np ? __ldg(bt + base + lane) : 0;
+                const bool bad = base + lane < np && (e < 0 || e >= p.num_pool_pages);
+                if (__any_sync(0xffffffffu, bad) && lane == 0)
+                    atomicOr(p.ws_error, kErrPageId);
+                if (bad)
+                    e = 0;
+                const int cnt = np - base < 32 ? np - base : 32;
+                for (int j = 0; j < cnt; ++j, ++gp) {
+                    const int phys = __shfl_sync(0xffffffffu, e, j);
+                    const int s = gp % NST;
+                    const int k = gp / NST;
+                    if (lane == 0) {
+                        if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, p.ws_error))
+                            ok = false;
+                        if (ok) {
+                            const uint32_t fb = bar_full + 8 * s;
+                            mbar_expect_tx(fb, 2 * C::kStageBytes);
+#pragma unroll
+                            for (int hf = 0; hf < D / kBoxD; ++hf) {
+                                tma_load_box(k_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_k, fb, hf * kBoxD,
+                                             item.y, phys, policy);
+                                tma_load_box(v_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_v, fb, hf * kBoxD,
+                                             item.y, phys, policy);
+                            }
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok)
+                        break;
+                }
+            }
+        }
+    } else {
+        // ================= consumers =================
+        const int mi = lane >> 3;
+        const int ri = lane & 7;
+        const uint32_t k_off = (uint32_t)((8 * (mi & 1) + ri) * 128);
+        const int k_hi = mi >> 1;
+        const uint32_t v_off = (uint32_t)((8 * (mi >> 1) + ri) * 128);
+        const int v_hi = mi & 1;
+        const float sl2 = p.scale_log2;
+        const int G = p.G;
+        constexpr int D4 = D / 4;
+        int gp_base = 0;
+        bool alive = true;
+        for (int it = it0; it < it1; ++it) {
+            const int4 item = __ldg(p.items + it);
+            int pg0, np;
+            const bool item_ok = item_pages(p, item, pg0, np);
+            const int row = item.x, h = item.y, te = item.w;
+            uint32_t qf[D / 16][NT][2];
+            float m_run[NT][2], l_run[NT][2];
+            float o[D / 16][NT][4];
+            const __nv_bfloat16 *qb = p.q + ((int64_t)(item_ok ? row : 0) * p.H_q + (int64_t)(item_ok ? h : 0) * G) * D;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int g = nt * 8 + r;
+                m_run[nt][0] = m_run[nt][1] = -INFINITY;
+                l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt)
+                    o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    uint32_t lo = 0, hi = 0;
+                    if (g < G) {
+                        const uint32_t *src =
+                            reinterpret_cast<const uint32_t *>(qb + (int64_t)g * D + ks * 16 + 2 * c4);
+                        lo = __ldg(src);
+                        hi = __ldg(src + 4);
+                    }
+                    qf[ks][nt][0] = lo;
+                    qf[ks][nt][1] = hi;
+                }
+            }
+            // this warp's pages of the item: global page index gp with gp % NW == warp
+            for (int gp = gp_base + ((warp - gp_base % NW) + NW) % NW; alive && gp < gp_base + np; gp += NW) {
+                const int s = gp % NST;
+                const bool ready = mbar_wait(bar_full + 8 * s, (gp / NST) & 1, p.ws_error);
+                if (!__all_sync(0xffffffffu, ready)) {
+                    alive = false;
+                    break;
+                }
+                const int pidx = gp - gp_base;
+                const int tok0 = (pg0 + pidx) * kPage;
+                const int nvalid = te - tok0 < kPage ? te - tok0 : kPage;
+                attend_page<D, NT>(smem, sbase, k_ring + s * C::kStageBytes, v_ring + s * C::kStageBytes,
+                                   bar_empty + 8 * s, nvalid, lane, r, ri, k_off, k_hi, v_off, v_hi, sl2, qf, m_run,
+                                   l_run, o);
+            }
+            gp_base += np;
+            // ---- close the item: combine the consumer warps' states ----
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int sh = 4; sh < 32; sh <<= 1)
+                        l_run[nt][j] += __shfl_xor_sync(0xffffffffu, l_run[nt][j], sh);
+                    const int g = nt * 8 + 2 * c4 + j;
+                    float *dst = cb_o + (warp * C::kGP + g) * C::kOStride;
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        dst[mt * 16 + r] = o[mt][nt][j];
+                        dst[mt * 16 + r + 8] = o[mt][nt][2 + j];
+                    }
+                    if (r == 0) {
+                        cb_m[warp * C::kGP + g] = m_run[nt][j];
+                        cb_l[warp * C::kGP + g] = l_run[nt][j];
+                    }
+                }
+            named_barrier(1, kConsumers);
+            const int pair = item_ok ? row * p.H_kv + h : 0;
+            int slot0 = 0, nslots = 0;
+            if (item_ok) {
+                slot0 = __ldg(p.indptr + pair);
+                nslots = __ldg(p.indptr + pair + 1) - slot0;
+            }
+            const bool slot_ok = item_ok && nslots >= 1 && slot0 >= 0 && it >= slot0 && it < slot0 + nslots &&
+                                 slot0 + nslots <= p.n_items;
+            if (!slot_ok && item_ok && tid == 0)
+                atomicOr(p.ws_error, kErrItem);
+            if (slot_ok) {
+                for (int e = tid; e < G * D4; e += kConsumers) {
+                    const int g = e / D4;
+                    const int d4 = (e % D4) * 4;
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < NW; ++w)
+                        M = fmaxf(M, cb_m[w * C::kGP + g]);
+                    float L = 0.f;
+                    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int w = 0; w < NW; ++w) {
+                        const float mw = cb_m[w * C::kGP + g];
+                        if (mw == -INFINITY)
+                            continue;
+                        const float sc = exp2_approx(mw - M);
+                        L = fmaf(cb_l[w * C::kGP + g], sc, L);
+                        O = fma4(*reinterpret_cast<const float4 *>(cb_o + (w * C::kGP + g) * C::kOStride + d4), sc, O);
+                    }
+                    if (nslots == 1) {
+                        const float inv = L > 0.f ? 1.f / L : 0.f;
+                        store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+                    } else {
+                        const int64_t idx = (int64_t)it * G + g;
+                        *reinterpret_cast<float4 *>(p.ws_acc + idx * D + d4) = O;
+                        if (d4 == 0) {
+                            p.ws_m[idx] = M;
+                            p.ws_l[idx] = L;
+                        }
+                    }
+                }
+            }
+            named_barrier(1, kConsumers);  // partial stored by all consumers; combine buffer free
+            if (slot_ok && nslots > 1 && !p.separate_merge) {
+                if (tid == 0) {
+                    const uint32_t prev = ticket_acq_rel(p.ws_counters + pair);
+                    if (prev == (uint32_t)(nslots - 1)) {
+                        const int k = misc[0];
+                        if (k < C::kMaxDeferred) {
+                            deferred[k] = make_int4(row, h, slot0, nslots);
+                            misc[0] = k + 1;
+                        } else {
+                            misc[1] = 1;  // list full: merge right away
+                        }
+                    }
+                }
+                named_barrier(1, kConsumers);
+                if (misc[1]) {
+                    merge_pair<D>(p, row, h, slot0, nslots, tid, kConsumers);
+                    named_barrier(1, kConsumers);
+                    if (tid == 0) {
+                        p.ws_counters[pair] = 0u;
+                        misc[1] = 0;
+                    }
+                    named_barrier(1, kConsumers);
+                }
+            }
+        }
+    }
+
+    // ---- merges this block owns, through the now idle ring ----
+    grid_launch_dependents();
+    __syncthreads();
+    const int nd = misc[0];
+    uint32_t uses[2] = {0, 0};
+    for (int k = 0; k < nd; ++k) {
+        const int4 d = deferred[k];
+        if (!merge_pair_staged<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, d.x, d.y, d.z, d.w, tid, uses))
+            merge_pair<D>(p, d.x, d.y, d.z, d.w, tid, C::kThreads);
+        __syncthreads();
+        if (tid == 0)
+            p.ws_counters[d.x * p.H_kv + d.y] = 0u;  // ready for the next call
     }
 }
 
@@ -1067,6 +1391,35 @@ cudaError_t launch_split_nst(int D, int NT, const Params &prm, int64_t grid, cud
     return NT == 1 ? launch_split<64, 1, NST>(prm, grid, st, pdl) : launch_split<64, 2, NST>(prm, grid, st, pdl);
 }
 
+#ifndef PKV_NST_BAL
+#define PKV_NST_BAL 8
+#endif
+#ifndef PKV_NST_BAL_DEEP
+#define PKV_NST_BAL_DEEP 20
+#endif
+
+template <int D, int NT, int NST>
+cudaError_t launch_balanced(const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+{
+    using C = BCfg<D, NT, kNW, NST>;
+    static std::atomic<uint64_t> configured{0};
+    auto kernel = balanced_kernel<D, NT, kNW, NST>;
+    cudaError_t e = set_smem(kernel, C::kSmemBytes, configured);
+    if (e != cudaSuccess)
+        return e;
+    e = launch_ex(kernel, (unsigned)grid, C::kThreads, C::kSmemBytes, st, pdl, prm);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int NST>
+cudaError_t launch_balanced_nst(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+{
+    if (D == 128)
+        return NT == 1 ? launch_balanced<128, 1, NST>(prm, grid, st, pdl)
+                       : launch_balanced<128, 2, NST>(prm, grid, st, pdl);
+    return NT == 1 ? launch_balanced<64, 1, NST>(prm, grid, st, pdl) : launch_balanced<64, 2, NST>(prm, grid, st, pdl);
+}
+
 cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
 {
     return deep ? launch_split_nst<kNSTDeep>(D, NT, prm, grid, st, pdl)
@@ -1098,11 +1451,14 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         return PKV_ERR_INVALID;
     const pkv_shape &s = *shape;
     const pkv_plan &pl = *plan;
-    if (pl.mode != PKV_NO_SPLIT && pl.mode != PKV_SPLIT_S && pl.mode != PKV_WORK_QUEUE)
+    if (pl.mode != PKV_NO_SPLIT && pl.mode != PKV_SPLIT_S && pl.mode != PKV_WORK_QUEUE && pl.mode != PKV_BALANCED)
         return PKV_ERR_INVALID;
     if (pl.mode == PKV_SPLIT_S && (pl.num_splits < 1 || pl.chunk_pages < 1))
         return PKV_ERR_INVALID;
-    if (pl.mode == PKV_WORK_QUEUE && (!items || !indptr || n_items < (int64_t)s.B * s.H_kv))
+    if ((pl.mode == PKV_WORK_QUEUE || pl.mode == PKV_BALANCED) &&
+        (!items || !indptr || n_items < (int64_t)s.B * s.H_kv))
+        return PKV_ERR_INVALID;
+    if (pl.mode == PKV_BALANCED && pl.num_splits < 1)
         return PKV_ERR_INVALID;
     int rc = check_fast_path(s);
     if (rc != PKV_OK)
@@ -1153,13 +1509,22 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.n_items = n_items;
 
     const int64_t pairs = (int64_t)s.B * s.H_kv;
-    const int64_t grid = pl.mode == PKV_NO_SPLIT ? pairs : pl.mode == PKV_SPLIT_S ? pairs * pl.num_splits : n_items;
+    const int64_t grid = pl.mode == PKV_NO_SPLIT ? pairs
+                         : pl.mode == PKV_SPLIT_S ? pairs * pl.num_splits
+                         : pl.mode == PKV_BALANCED ? (int64_t)pl.num_splits
+                                                   : n_items;
     if (grid > INT32_MAX || pairs > INT32_MAX)
         return PKV_ERR_UNSUPPORTED;
     const int NT = prm.G <= 8 ? 1 : 2;
     const bool pdl = (pl.flags & PKV_FLAG_NO_PDL) == 0;
     const bool deep = (pl.flags & PKV_FLAG_DEEP_RING) != 0;
-    if (launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl) != cudaSuccess)
+    cudaError_t le;
+    if (pl.mode == PKV_BALANCED)
+        le = deep ? launch_balanced_nst<PKV_NST_BAL_DEEP>(s.head_dim, NT, prm, grid, st, pdl)
+                  : launch_balanced_nst<PKV_NST_BAL>(s.head_dim, NT, prm, grid, st, pdl);
+    else
+        le = launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl);
+    if (le != cudaSuccess)
         return PKV_ERR_CUDA;
     const bool need_merge = pl.mode != PKV_NO_SPLIT && prm.separate_merge;
     if (need_merge) {

@@ -34,6 +34,12 @@ MODES = {
     "wq3_deep_sep": rule(2, 1, 3, 5),
     "split7_nopdl": rule(1, 7, 0, 2),
     "wq16_deep_nopdl": rule(2, 1, 16, 6),
+    "bal1": rule(3, 1),
+    "bal7": rule(3, 7),
+    "bal37": rule(3, 37),
+    "bal296": rule(3, 296),
+    "bal148_deep": rule(3, 148, 0, 4),
+    "bal64_sep": rule(3, 64, 0, 1),
 }
 
 
@@ -69,7 +75,8 @@ CASES = {
 
 @pytest.mark.parametrize("case", sorted(CASES))
 @pytest.mark.parametrize("mode", ["nosplit", "split7", "split32", "split32_sep", "wq3", "wq3_sep", "split32_deep",
-                                  "wq3_deep_sep", "split7_nopdl"])
+                                  "wq3_deep_sep", "split7_nopdl", "bal1", "bal7", "bal296", "bal148_deep",
+                                  "bal64_sep"])
 def test_ragged_shapes(case, mode):
     lens, H_q, H_kv, D = CASES[case]
     w = to_device(W.make_custom(lens, H_q, H_kv, D, seed=101, poison=True, q_scale=3.0))
@@ -87,7 +94,7 @@ def test_nhd_layout(mode):
     assert_close(got, ref, f"nhd/{mode}")
 
 
-@pytest.mark.parametrize("mode", ["nosplit", "split32", "wq3"])
+@pytest.mark.parametrize("mode", ["nosplit", "split32", "wq3", "bal37"])
 def test_peaked_logits(mode):
     """q scaled x8: logits ~ N(0, 64), a few tokens dominate; tests the
     running-max rescaling across pages and across splits."""
@@ -100,7 +107,7 @@ def test_peaked_logits(mode):
 
 def test_all_rows_empty_and_zero_batch():
     w = to_device(W.make_custom([0, 0, 0], 8, 2, 64, seed=104, poison=True))
-    for mode in ("nosplit", "split7", "wq3"):
+    for mode in ("nosplit", "split7", "wq3", "bal7"):
         got, _ = run(w, mode_rule=MODES[mode])
         assert (got == 0).all(), mode
     w = to_device(W.make_custom([], 8, 2, 64, seed=105))
@@ -112,7 +119,7 @@ def test_all_rows_empty_and_zero_batch():
 def test_single_token_rows_are_exact():
     """N = 1: the output is that token's V exactly (rounded to bf16, a no-op)."""
     w = to_device(W.make_custom([1, 1, 1], 16, 4, 128, seed=106, poison=True))
-    for mode in ("nosplit", "split7", "wq3"):
+    for mode in ("nosplit", "split7", "wq3", "bal7", "bal1"):
         got, _ = run(w, mode_rule=MODES[mode])
         for i in range(w.B):
             page = int(w.block_table[i, 0])
@@ -137,14 +144,14 @@ def test_deterministic_and_page_permutation_bit_identical():
 def test_split_counts_do_not_change_the_answer_beyond_rounding():
     w = to_device(W.make_custom([5000, 1234], 32, 8, 128, seed=108, poison=True))
     ref = oracle_full(w)
-    for mode in ("nosplit", "split2", "split7", "split32", "wq1", "wq16"):
+    for mode in ("nosplit", "split2", "split7", "split32", "wq1", "wq16", "bal1", "bal7", "bal37", "bal296"):
         got, _ = run(w, mode_rule=MODES[mode])
         assert_close(got, ref, mode)
 
 
 def test_workspace_counters_are_zero_after_a_call():
     w = to_device(W.make_custom([3000, 100], 32, 8, 128, seed=109))
-    for mode in ("split32", "wq3"):
+    for mode in ("split32", "wq3", "bal37", "bal1"):
         _, dp = run(w, mode_rule=MODES[mode])
         pairs = w.B * w.H_kv
         counters = dp.workspace[256:256 + 4 * pairs]
@@ -201,3 +208,24 @@ def test_prefix_sharing_config_sampled():
     pairs = [(r, int(rng.integers(w.H_q))) for r in rows] + [(int(np.argmax(w.seq_lens)), 63)]
     ref = oracle_sampled(w, pairs)
     assert_close(np.stack([got[r, h] for r, h in pairs]), ref, f"prefix plan {dp.plan}")
+
+
+@pytest.mark.parametrize("name", ["long", "crossover", "mixed"])
+@pytest.mark.parametrize("mode", ["bal296", "bal148_deep"])
+def test_full_size_configs_balanced_sampled(name, mode):
+    w = to_device(W.make(name, poison=True))
+    got, dp = run(w, mode_rule=MODES[mode])
+    rng = np.random.default_rng(9)
+    pairs = [(int(rng.integers(w.B)), int(rng.integers(w.H_q))) for _ in range(10)] + [(w.B - 1, w.H_q - 1)]
+    assert_close(np.stack([got[r, h] for r, h in pairs]), oracle_sampled(w, pairs), f"{name} plan {dp.plan}")
+
+
+def test_balanced_deterministic_across_runs_and_deferred_merges():
+    """Many short rows per block (B=40, 24 blocks) exercise several items and
+    several owned merges per block; results are bit-identical run to run."""
+    lens = [int(x) for x in np.random.default_rng(3).integers(1, 3000, 40)]
+    w = to_device(W.make_custom(lens, 16, 4, 128, seed=111, poison=True))
+    a, dp = run(w, mode_rule=rule(3, 24))
+    b, _ = run(w, mode_rule=rule(3, 24))
+    assert np.array_equal(a, b)
+    assert_close(a, oracle_full(w), "balanced B=40 T=24")
