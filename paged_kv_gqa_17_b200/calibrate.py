@@ -1,0 +1,162 @@
+"""Calibrate the built-in policy table on the GPU from measured timings.
+
+    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--steps 30]
+
+The policy maps (batch size B, longest row N_max) to an execution plan
+[PersistentKV explainer, Technical summary > Methodology > 2 "Calibrated
+adaptive policy": thresholds calibrated by hand on one seed, results reported
+on a holdout seed].  This script does the same by measurement:
+
+  1. For every cell of a (B, N_max) grid it draws a batch with the calibration
+     seed 20260622: one row of the cell's representative length, the others
+     log-uniform between an eighth of it and it (H_q=32, H_kv=8, D=128,
+     16-token pages).
+  2. It times every candidate plan (no-split; split-S over several S with
+     and without the deep ring; the work queue over several chunk sizes; the
+     balanced grid at one and two blocks per SM) as the steady-state device
+     time of back-to-back steps over rotating pool copies.
+  3. The fastest plan of each cell becomes a rule; neighbouring cells of one B
+     with the same plan are merged.
+  4. Every cell is re-measured with the holdout seed 20260623; the report
+     lists the chosen plan's time against the best candidate (the regret).
+
+It writes the table as JSON (the library's build turns it into its built-in
+table) and a markdown report.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+B_EDGES = [1, 2, 4, 8, 16, 32, 2**31 - 1]          # rules cover [B_EDGES[i], B_EDGES[i+1])
+N_EDGES = [0, 1024, 4096, 16384, 65536, 2**31 - 1]  # and [N_EDGES[j], N_EDGES[j+1])
+N_REP = [512, 2048, 8192, 32768, 131072]            # representative N_max of each N range
+B_REP = [1, 2, 4, 8, 16, 64]                        # representative B of each B range
+MODE_NAMES = {0: "NO_SPLIT", 1: "SPLIT_S", 2: "WORK_QUEUE", 3: "BALANCED"}
+
+
+def candidates():
+    """(mode, num_splits, chunk_pages, flags) rules to try in every cell."""
+    out = [(0, 1, 0, 0)]
+    for S in (8, 16, 32, 37, 64):
+        out += [(1, S, 0, 0), (1, S, 0, 4)]
+    for C in (8, 16, 32, 64):
+        out.append((2, 1, C, 0))
+    out += [(3, 296, 0, 0), (3, 148, 0, 4)]
+    return out
+
+
+def cell_lengths(B: int, n_rep: int, seed: int):
+    import torch
+
+    g = torch.Generator().manual_seed(seed * 1000 + B * 7 + n_rep)
+    lo = max(16, n_rep // 8)
+    rest = torch.rand(max(0, B - 1), generator=g, dtype=torch.float64)
+    lens = [n_rep] + [int(math.exp(math.log(lo) + float(u) * (math.log(n_rep) - math.log(lo)))) for u in rest]
+    return lens
+
+
+def measure_cell(B, n_rep, seed, steps, cands, torch, bd, W, bench):
+    dev = torch.device("cuda")
+    w = W.make_custom(cell_lengths(B, n_rep, seed), 32, 8, 128, seed=seed, device=dev)
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    copies = bench.pool_copies(w, torch)
+    times = {}
+    for c in cands:
+        rule = bd.Rule(0, 2**31 - 1, 0, 2**31 - 1, *c)
+        dp = bd.plan_decode(w.seq_lens, shape, dev, rules=[rule])
+        times[c] = bench.time_steady(w, dp, steps, 3, torch, bd, copies) / steps * 1e3  # us per step
+    del copies, w
+    torch.cuda.empty_cache()
+    return times
+
+
+def build_rules(best):
+    """best[(bi, nj)] -> candidate; merge equal neighbours along N for each B range."""
+    rules = []
+    for bi in range(len(B_REP)):
+        nj = 0
+        while nj < len(N_REP):
+            c = best[(bi, nj)]
+            nk = nj
+            while nk + 1 < len(N_REP) and best[(bi, nk + 1)] == c:
+                nk += 1
+            mode, S, C, flags = c
+            r = {"b_lo": B_EDGES[bi], "b_hi": B_EDGES[bi + 1], "nmax_lo": N_EDGES[nj], "nmax_hi": N_EDGES[nk + 1],
+                 "mode": MODE_NAMES[mode]}
+            if mode in (1, 3):
+                r["num_splits"] = S
+            if mode == 2:
+                r["chunk_pages"] = C
+            if flags:
+                r["flags"] = flags
+            rules.append(r)
+            nj = nk + 1
+    return rules
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--out", default=os.path.join(HERE, "policy_b200.json"))
+    ap.add_argument("--report", default=os.path.join(ROOT, "profiles", "policy_calibration_b200.md"))
+    ap.add_argument("--steps", type=int, default=30)
+    args = ap.parse_args(argv)
+
+    import torch
+
+    from paged_kv_gqa_17_b200 import binding as bd
+    from paged_kv_gqa_17_b200 import timing as bench
+    from paged_kv_gqa_17_b200 import workloads as W
+
+    bd.lib()
+    cands = candidates()
+    best, calib = {}, {}
+    for bi, B in enumerate(B_REP):
+        for nj, n in enumerate(N_REP):
+            t = measure_cell(B, n, W.SEED_CALIBRATE, args.steps, cands, torch, bd, W, bench)
+            calib[(bi, nj)] = t
+            best[(bi, nj)] = min(t, key=t.get)
+            print(f"B={B:3d} N_max={n:6d} best {best[(bi, nj)]} {t[best[(bi, nj)]]:.2f} us", flush=True)
+    rules = build_rules(best)
+    doc = {
+        "name": "b200_calibrated",
+        "about": "Built-in policy table of libpkv.so (pkv_default_policy), written by "
+                 "paged_kv_gqa_17_b200/calibrate.py from steady-state timings on B200 with seed 20260622 "
+                 "(H_q=32, H_kv=8, D=128, 16-token pages). Rules are checked in order; the first whose "
+                 "half-open ranges hold (B, N_max) decides.",
+        "rules": rules,
+    }
+    with open(args.out, "w") as f:
+        json.dump(doc, f, indent=1)
+        f.write("\n")
+    # holdout check
+    lines = ["# Policy calibration on B200", "",
+             "Command: `python -m paged_kv_gqa_17_b200.calibrate` (writes paged_kv_gqa_17_b200/policy_b200.json).", "",
+             "Steady-state µs per decode step (back-to-back steps over rotating pool copies), H_q=32, H_kv=8, "
+             "D=128. Calibration seed 20260622 picks the plan; holdout seed 20260623 re-measures it.", "",
+             "| B | N_max | chosen plan (mode, S/T, C, flags) | calib µs | holdout µs | holdout best | best µs | regret |",
+             "|---|---|---|---|---|---|---|---|"]
+    for bi, B in enumerate(B_REP):
+        for nj, n in enumerate(N_REP):
+            c = best[(bi, nj)]
+            hold = measure_cell(B, n, W.SEED_REPORT, args.steps, cands, torch, bd, W, bench)
+            hb = min(hold, key=hold.get)
+            lines.append(f"| {B} | {n} | {MODE_NAMES[c[0]]} {c[1:]} | {calib[(bi, nj)][c]:.2f} | {hold[c]:.2f} | "
+                         f"{MODE_NAMES[hb[0]]} {hb[1:]} | {hold[hb]:.2f} | {100 * (hold[c] / hold[hb] - 1):.1f}% |")
+            print(lines[-1], flush=True)
+    os.makedirs(os.path.dirname(args.report), exist_ok=True)
+    with open(args.report, "w") as f:
+        f.write("\n".join(lines) + "\n")
+    print(f"wrote {args.out} and {args.report}")
+
+
+if __name__ == "__main__":
+    main()

@@ -30,14 +30,10 @@ int check_shape(const pkv_shape *s)
 
 namespace {
 
-// Built-in policy table, measured on B200 (seed 20260622, checked on 20260623).
-// It is the same table as paged_kv_gqa_17_b200/policy_b200.json.
+// Built-in policy table, measured on B200 by paged_kv_gqa_17_b200/calibrate.py
+// (seed 20260622, checked on 20260623); generated from policy_b200.json.
 const pkv_policy_rule kDefaultRules[] = {
-    // b_lo, b_hi, nmax_lo, nmax_hi, mode, num_splits, chunk_pages, flags
-    {1, 2, 0, 1024, PKV_NO_SPLIT, 1, 0, 0},
-    {1, 2, 1024, INT32_MAX, PKV_SPLIT_S, 37, 0, PKV_FLAG_DEEP_RING},
-    {2, INT32_MAX, 0, 1024, PKV_NO_SPLIT, 1, 0, 0},
-    {2, INT32_MAX, 1024, INT32_MAX, PKV_WORK_QUEUE, 1, 16, 0},
+#include "pkv_policy_table.inc"
 };
 constexpr int32_t kNumDefaultRules = (int32_t)(sizeof(kDefaultRules) / sizeof(kDefaultRules[0]));
 

@@ -1,0 +1,84 @@
+"""Device timing of decode steps (CUDA events on the launching stream).
+
+Two protocols:
+  time_steady    K steps queued back to back between one pair of events,
+                 consecutive steps reading different copies of the KV pool
+                 (pool_copies) so that no step finds its pages in L2;
+  time_isolated  single cold steps, L2 flushed (Flush) before each, events
+                 around the step alone.
+"""
+from __future__ import annotations
+
+FLUSH_BYTES = 256 << 20
+
+
+class Flush:
+    """Evicts L2: writes a buffer larger than L2, then reads another one, so
+    the next kernel finds neither its data nor dirty lines to write back."""
+
+    def __init__(self, torch, device):
+        self.a = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.b = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def __call__(self, i=0):
+        self.a.fill_(i & 255)
+        self.b.sum()
+
+
+def pool_copies(w, torch, l2_bytes=126 << 20):
+    """Copies of the KV pool so that >= 3 L2 sizes of step data separate two
+    reads of the same copy (at most 8 copies; 1 when one step already exceeds that)."""
+    per_step = w.kv_bytes()
+    n = 1 if per_step >= 3 * l2_bytes else min(8, -(-3 * l2_bytes // per_step) + 1)
+    return [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone()) for _ in range(n - 1)]
+
+
+def time_steady(w, dp, K, W, torch, bd, copies):
+    """Device time (ms) of K back-to-back steps, one event pair, rotating pool copies."""
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=w.q.device)
+    out = torch.empty_like(w.q)
+
+    def step(i):
+        k, v = copies[i % len(copies)]
+        bd.paged_decode(w.q, k, v, w.block_table, lens, w.P, w.scale, plan=dp, out=out)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for i in range(K):
+        step(W + i)
+    b.record(st)
+    torch.cuda.synchronize()
+    if bd.workspace_status(dp) != 0:
+        raise RuntimeError("device error during the timed steps")
+    return a.elapsed_time(b)
+
+
+def time_isolated(w, dp, K, W, torch, bd, flush):
+    """Per-step device times (ms) of single cold steps: L2 flushed, events around the step."""
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=w.q.device)
+    out = torch.empty_like(w.q)
+
+    def step():
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, w.P, w.scale, plan=dp, out=out)
+
+    for i in range(W):
+        flush(i)
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for i in range(K):
+        flush(i)
+        starts[i].record(st)
+        step()
+        ends[i].record(st)
+    torch.cuda.synchronize()
+    if bd.workspace_status(dp) != 0:
+        raise RuntimeError("device error during the timed steps")
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
