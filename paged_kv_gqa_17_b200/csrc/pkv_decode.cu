@@ -19,7 +19,8 @@
 //
 // B200 design (the pages' kernels were written for an RTX 3060):
 //   - one producer warp streams whole 16-token pages of K and V for one KV
-//     head (4 KiB each at D = 128) with TMA tensor copies into an NST-stage
+//     head (4 KiB each at D = 128) with TMA tensor copies (one rank-5 copy per
+//     page and tensor, four lanes issuing at once) into an NST-stage
 //     shared-memory ring, completion tracked by mbarriers; the copies use the
 //     128-byte swizzle so the tensor-core fragment loads below are free of
 //     bank conflicts;
@@ -215,6 +216,18 @@ __device__ __forceinline__ void named_barrier(int id, int threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// TMA tiled copy of a whole (page, head) block [d_hi][16 tokens][64 d] of a
+// rank-5 pool view (head_dim split as 64 x d_hi) in one instruction.
+__device__ __forceinline__ void tma_load_page(uint32_t dst, const CUtensorMap *tm, uint32_t bar, int head, int page,
+                                              uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(0), "r"(0), "r"(0), "r"(head), "r"(page), "r"(bar), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *tm)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
@@ -357,6 +370,59 @@ __device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslot
         const float inv = L > 0.f ? 1.f / L : 0.f;
         store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
     }
+}
+
+// The producer's issue rate bounds a block's bandwidth: one rank-5 TMA copy
+// per K (or V) page instead of one per 64-wide half, issued by several lanes
+// at once.
+#ifndef PKV_TMA_5D
+#define PKV_TMA_5D 1
+#endif
+#ifndef PKV_ISSUE_LANES
+#define PKV_ISSUE_LANES 4
+#endif
+
+// Producer: copy the K and V blocks of cnt consecutive pages of one KV head
+// into the ring, page j's physical id held by lane j of `e`; pages get ring
+// positions gp, gp+1, ... (stage = position % NST).  PKV_ISSUE_LANES lanes
+// issue in parallel, each waiting for its own stage to be released.
+// Returns false (after setting the error bit) when a wait timed out.
+template <int D, int NST>
+__device__ __forceinline__ bool issue_pages(const Params &p, int lane, int e, int cnt, int &gp, int head,
+                                            uint32_t k_ring, uint32_t v_ring, uint32_t bar_full, uint32_t bar_empty,
+                                            uint64_t policy)
+{
+    constexpr int kStage = D * kPage * 2;
+    bool ok = true;
+    for (int j0 = 0; j0 < cnt && ok; j0 += PKV_ISSUE_LANES) {
+        const int j = j0 + lane;
+        const int phys = __shfl_sync(0xffffffffu, e, j & 31);
+        bool my_ok = true;
+        if (lane < PKV_ISSUE_LANES && j < cnt) {
+            const int g = gp + j;
+            const int st = g % NST;
+            const int k = g / NST;
+            if (k > 0 && !mbar_wait(bar_empty + 8 * st, (k - 1) & 1, p.ws_error))
+                my_ok = false;
+            if (my_ok) {
+                const uint32_t fb = bar_full + 8 * st;
+                mbar_expect_tx(fb, 2 * kStage);
+#if PKV_TMA_5D
+                tma_load_page(k_ring + st * kStage, &p.tm_k, fb, head, phys, policy);
+                tma_load_page(v_ring + st * kStage, &p.tm_v, fb, head, phys, policy);
+#else
+#pragma unroll
+                for (int hf = 0; hf < D / kBoxD; ++hf) {
+                    tma_load_box(k_ring + st * kStage + hf * kBoxBytes, &p.tm_k, fb, hf * kBoxD, head, phys, policy);
+                    tma_load_box(v_ring + st * kStage + hf * kBoxBytes, &p.tm_v, fb, hf * kBoxD, head, phys, policy);
+                }
+#endif
+            }
+        }
+        ok = __all_sync(0xffffffffu, my_ok);
+    }
+    gp += cnt;
+    return ok;
 }
 
 // Attention over one 16-token page in ring stage (ks_base, vs_base) for the
@@ -721,6 +787,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
 #endif
         int e_next = lane < npages ? e_first : 0;
         bool ok = true;
+        int gp = 0;
         for (int base = 0; base < npages && ok; base += 32) {
             int e = e_next;
             e_next = base + 32 + lane < npages ? __ldg(bt + base + 32 + lane) : 0;
@@ -730,36 +797,13 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             if (bad)
                 e = 0;  // read a real page instead; the error bit reports the bad entry
             const int cnt = npages - base < 32 ? npages - base : 32;
-            for (int j = 0; j < cnt; ++j) {
-                const int phys = __shfl_sync(0xffffffffu, e, j);
-                const int pidx = base + j;
-                const int s = pidx % NST;
-                const int k = pidx / NST;
-                if (lane == 0) {
 #ifdef PKV_TRACE
-                    const long long tw0 = clock64();
+            const long long tw0 = clock64();
 #endif
-                    if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, p.ws_error))
-                        ok = false;
+            ok = issue_pages<D, NST>(p, lane, e, cnt, gp, h, k_ring, v_ring, bar_full, bar_empty, policy);
 #ifdef PKV_TRACE
-                    prod_wait += clock64() - tw0;
+            prod_wait += clock64() - tw0;
 #endif
-                    if (ok) {
-                        const uint32_t fb = bar_full + 8 * s;
-                        mbar_expect_tx(fb, 2 * C::kStageBytes);
-#pragma unroll
-                        for (int hf = 0; hf < C::kHalves; ++hf) {
-                            tma_load_box(k_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_k, fb, hf * kBoxD, h,
-                                         phys, policy);
-                            tma_load_box(v_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_v, fb, hf * kBoxD, h,
-                                         phys, policy);
-                        }
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok)
-                    break;
-            }
         }
 #ifdef PKV_TRACE
         if (lane == 0 && blockIdx.x < kTraceBlocks) {
@@ -1023,29 +1067,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
                 if (bad)
                     e = 0;
                 const int cnt = np - base < 32 ? np - base : 32;
-                for (int j = 0; j < cnt; ++j, ++gp) {
-                    const int phys = __shfl_sync(0xffffffffu, e, j);
-                    const int s = gp % NST;
-                    const int k = gp / NST;
-                    if (lane == 0) {
-                        if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, p.ws_error))
-                            ok = false;
-                        if (ok) {
-                            const uint32_t fb = bar_full + 8 * s;
-                            mbar_expect_tx(fb, 2 * C::kStageBytes);
-#pragma unroll
-                            for (int hf = 0; hf < D / kBoxD; ++hf) {
-                                tma_load_box(k_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_k, fb, hf * kBoxD,
-                                             item.y, phys, policy);
-                                tma_load_box(v_ring + s * C::kStageBytes + hf * kBoxBytes, &p.tm_v, fb, hf * kBoxD,
-                                             item.y, phys, policy);
-                            }
-                        }
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok)
-                        break;
-                }
+                ok = issue_pages<D, NST>(p, lane, e, cnt, gp, item.y, k_ring, v_ring, bar_full, bar_empty, policy);
             }
         }
     } else {
@@ -1312,6 +1334,20 @@ int pool_tensor_map(CUtensorMap *out, const void *base, const pkv_shape &s)
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc)
         return PKV_ERR_CUDA;
+    CUtensorMap tm;
+#if PKV_TMA_5D
+    // [pages][H_kv][d_hi][P][64] view: one box = one whole (page, head) block,
+    // laid out [d_hi][token][64 d] in shared memory like two rank-4 boxes.
+    cuuint64_t dims[5] = {(cuuint64_t)kBoxD, (cuuint64_t)s.page_size, (cuuint64_t)(s.head_dim / kBoxD),
+                          (cuuint64_t)s.H_kv, (cuuint64_t)s.num_pool_pages};
+    cuuint64_t strides[4] = {(cuuint64_t)key.strides[0], (cuuint64_t)(kBoxD * 2), (cuuint64_t)key.strides[1],
+                             (cuuint64_t)key.strides[2]};
+    cuuint32_t box[5] = {(cuuint32_t)kBoxD, (cuuint32_t)s.page_size, (cuuint32_t)(s.head_dim / kBoxD), 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult rc = enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+#else
     cuuint64_t dims[4], strides[3];
     for (int i = 0; i < 4; ++i)
         dims[i] = (cuuint64_t)key.dims[i];
@@ -1319,10 +1355,10 @@ int pool_tensor_map(CUtensorMap *out, const void *base, const pkv_shape &s)
         strides[i] = (cuuint64_t)key.strides[i];
     cuuint32_t box[4] = {(cuuint32_t)kBoxD, (cuuint32_t)s.page_size, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUtensorMap tm;
     CUresult rc = enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+#endif
     if (rc != CUDA_SUCCESS)
         return PKV_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(mu);
