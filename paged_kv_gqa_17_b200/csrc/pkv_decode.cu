@@ -75,6 +75,9 @@ struct __align__(64) Params {
     int32_t B, H_q, H_kv, G, max_pages, num_pool_pages;
     int32_t mode, num_splits, chunk_pages, separate_merge;
     int32_t n_items;
+#ifdef PKV_TRACE
+    int32_t trace_epoch;
+#endif
 };
 
 // ---------------------------------------------------------------------------
@@ -125,8 +128,10 @@ __device__ __forceinline__ uint64_t global_timer_ns()
 // Optional timeline tracing (build with -DPKV_TRACE): thread 0 of each block
 // records global-timer stamps at fixed points of the kernel.
 #ifdef PKV_TRACE
-constexpr int kTraceBlocks = 65536;
-__device__ unsigned long long g_pkv_trace[kTraceBlocks][16];
+// Two epochs (launch parity) so that consecutive launches can be compared.
+constexpr int kTraceBlocks = 16384;
+__device__ unsigned long long g_pkv_trace_buf[2][kTraceBlocks][16];
+#define g_pkv_trace (g_pkv_trace_buf[p.trace_epoch & 1])
 #define PKV_TRACE_POINT(slot)                                                  \
     do {                                                                       \
         if (threadIdx.x == 0 && blockIdx.x < kTraceBlocks)                     \
@@ -958,6 +963,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             PKV_TRACE_POINT(5);
         }
     }
+    PKV_TRACE_POINT(12);
 }
 
 // ---------------------------------------------------------------------------
@@ -1235,10 +1241,38 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
     }
 }
 
-// Separate merge: one block per (row, KV head); pairs with one slot were
-// finalized by the split kernel.
+// (M, L, O) <- (M, L, O) merged with the state (m2, l2, o2); neutral states
+// (max = -inf) carry no weight.
+__device__ __forceinline__ void merge_into(float &M, float &L, float4 &O, float m2, float l2, float4 o2)
+{
+    if (m2 == -INFINITY)
+        return;
+    if (M == -INFINITY) {
+        M = m2;
+        L = l2;
+        O = o2;
+        return;
+    }
+    const float Mn = fmaxf(M, m2);
+    const float a = exp2_approx(M - Mn);
+    const float b = exp2_approx(m2 - Mn);
+    L = fmaf(L, a, l2 * b);
+    O = fma4(O, a, scale4(o2, b));
+    M = Mn;
+}
+
+// Separate merge (chained to the split kernel by programmatic dependent
+// launch): one block per (row, KV head); pairs with one slot were finalized
+// by the split kernel.  Four threads share each (head, 4-column) task; a
+// thread loads the m, l and acc of its slots (every fourth one, 8 slots per
+// batch) all at once, so a pair of up to 32 slots costs one memory round
+// trip, then the four partial merges are combined by a fixed xor tree.
+constexpr int kMergeThreads = 512;
+constexpr int kMergeTPT = 4;
+constexpr int kMergeBatch = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Params p)
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ Params p)
 {
     grid_dependency_wait();  // the split kernel's partial states are complete and visible
     const int pair = blockIdx.x;
@@ -1259,7 +1293,50 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Para
     }
     if (nslots <= 1)
         return;
-    merge_pair<D>(p, row, h, slot0, nslots, threadIdx.x, blockDim.x);
+    const int G = p.G;
+    constexpr int D4 = D / 4;
+    const int sub = threadIdx.x % kMergeTPT;
+    for (int t = threadIdx.x / kMergeTPT; t < G * D4; t += kMergeThreads / kMergeTPT) {
+        const int g = t / D4;
+        const int d4 = (t % D4) * 4;
+        float M = -INFINITY, L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = sub; s0 < nslots; s0 += kMergeTPT * kMergeBatch) {
+            float ms[kMergeBatch], ls[kMergeBatch];
+            float4 as[kMergeBatch];
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u) {
+                const int s = s0 + u * kMergeTPT;
+                ms[u] = -INFINITY;
+                ls[u] = 0.f;
+                as[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s < nslots) {
+                    const int64_t idx = (int64_t)(slot0 + s) * G + g;
+                    ms[u] = __ldcg(p.ws_m + idx);
+                    ls[u] = __ldcg(p.ws_l + idx);
+                    as[u] = __ldcg(reinterpret_cast<const float4 *>(p.ws_acc + idx * D + d4));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kMergeBatch; ++u)
+                merge_into(M, L, O, ms[u], ls[u], as[u]);
+        }
+#pragma unroll
+        for (int off = 1; off < kMergeTPT; off <<= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, M, off);
+            const float l2 = __shfl_xor_sync(0xffffffffu, L, off);
+            float4 o2;
+            o2.x = __shfl_xor_sync(0xffffffffu, O.x, off);
+            o2.y = __shfl_xor_sync(0xffffffffu, O.y, off);
+            o2.z = __shfl_xor_sync(0xffffffffu, O.z, off);
+            o2.w = __shfl_xor_sync(0xffffffffu, O.w, off);
+            merge_into(M, L, O, m2, l2, o2);
+        }
+        if (sub == 0) {
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1543,6 +1620,10 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.chunk_pages = pl.chunk_pages;
     prm.separate_merge = (pl.flags & PKV_FLAG_SEPARATE_MERGE) ? 1 : 0;
     prm.n_items = n_items;
+#ifdef PKV_TRACE
+    static std::atomic<int32_t> trace_launches{0};
+    prm.trace_epoch = trace_launches.fetch_add(1);
+#endif
 
     const int64_t pairs = (int64_t)s.B * s.H_kv;
     const int64_t grid = pl.mode == PKV_NO_SPLIT ? pairs
@@ -1564,8 +1645,9 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         return PKV_ERR_CUDA;
     const bool need_merge = pl.mode != PKV_NO_SPLIT && prm.separate_merge;
     if (need_merge) {
-        cudaError_t e = s.head_dim == 128 ? launch_ex(merge_kernel<128>, (unsigned)pairs, 128, 0, st, pdl, prm)
-                                          : launch_ex(merge_kernel<64>, (unsigned)pairs, 128, 0, st, pdl, prm);
+        cudaError_t e = s.head_dim == 128
+                            ? launch_ex(merge_kernel<128>, (unsigned)pairs, kMergeThreads, 0, st, pdl, prm)
+                            : launch_ex(merge_kernel<64>, (unsigned)pairs, kMergeThreads, 0, st, pdl, prm);
         if (e != cudaSuccess || cudaGetLastError() != cudaSuccess)
             return PKV_ERR_CUDA;
     }
@@ -1600,7 +1682,7 @@ int pkv_paged_decode(const void *q, const void *k_pool, const void *v_pool, cons
 // Copy the timeline of the first blocks (16 uint64 per block) to the host.
 __attribute__((visibility("default"))) int pkv_trace_read(void *host, size_t bytes)
 {
-    return cudaMemcpyFromSymbol(host, g_pkv_trace, bytes) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cudaMemcpyFromSymbol(host, g_pkv_trace_buf, bytes) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 #endif
 
