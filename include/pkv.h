@@ -221,6 +221,16 @@ PKV_API int pkv_workspace_bytes(const pkv_shape *shape, const pkv_plan *plan, in
  * so later calls need no memset.  Also clears a recorded device error. */
 PKV_API int pkv_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
+/* Self-test of the device-side failure detection: every wait of the kernels
+ * on an mbarrier is bounded, and a wait that runs out sets the timeout bit in
+ * the workspace's error word instead of hanging.  This queues one small
+ * kernel on `stream` that waits on an mbarrier no thread ever arrives at;
+ * after limit_us microseconds (1 .. 1000000) the wait gives up and records
+ * the timeout, which pkv_workspace_status then reports as PKV_ERR_TIMEOUT
+ * (clear it with pkv_workspace_init).  No kernel of a decode runs. */
+PKV_API int pkv_selftest_wait_timeout(void *workspace, size_t workspace_bytes, uint32_t limit_us,
+                                      void *stream);
+
 /* Synchronize `stream`, then read the workspace's device error word:
  * PKV_OK, PKV_ERR_TIMEOUT or PKV_ERR_DEVICE_INPUT (also stored in
  * *device_error when not NULL, as the raw bit mask: 1 timeout, 2 seq_len out

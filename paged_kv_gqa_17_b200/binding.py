@@ -86,6 +86,7 @@ SIGNATURES = [
     ("pkv_workspace_bytes", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_workspace_init", ctypes.c_int, [c_p, c_sz, c_p]),
     ("pkv_workspace_status", ctypes.c_int, [c_p, c_p, c_p]),
+    ("pkv_selftest_wait_timeout", ctypes.c_int, [c_p, c_sz, ctypes.c_uint32, c_p]),
     ("pkv_paged_decode", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_i32, ctypes.c_float, c_p, c_p, c_p, c_p, c_p, c_i32, c_p, c_sz, c_p]),
     ("pkv_paged_decode_noalloc", ctypes.c_int,

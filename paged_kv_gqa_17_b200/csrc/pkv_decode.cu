@@ -145,7 +145,7 @@ __device__ unsigned long long g_pkv_trace_buf[2][kTraceBlocks][16];
 
 // Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs (or
 // kWaitLimitIters polls) with the timeout bit set in the error word.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err)
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err, uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -153,7 +153,7 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *
     for (uint32_t i = 1; i < kWaitLimitIters; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs)
+        if ((i & 255u) == 0 && global_timer_ns() - t0 > limit_ns)
             break;
     }
     atomicOr(err, kErrTimeout);
@@ -1339,6 +1339,19 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
     }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that no
+// one arrives at; the wait must give up after limit_ns and set the timeout bit.
+__global__ void wait_timeout_selftest_kernel(uint32_t *err, uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_wait(b, 0, err, limit_ns);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 
@@ -1685,6 +1698,15 @@ __attribute__((visibility("default"))) int pkv_trace_read(void *host, size_t byt
     return cudaMemcpyFromSymbol(host, g_pkv_trace_buf, bytes) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 #endif
+
+int pkv_selftest_wait_timeout(void *workspace, size_t workspace_bytes, uint32_t limit_us, void *stream)
+{
+    if (!workspace || workspace_bytes < kWsAlign || limit_us == 0 || limit_us > 1000000u)
+        return PKV_ERR_INVALID;
+    wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint32_t *>(workspace), (uint64_t)limit_us * 1000u);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
 
 int pkv_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
 {

@@ -16,6 +16,9 @@ drawn as fp32 N(0,1) and rounded to bf16, scale = 1/sqrt(head_dim)):
   prefix     B=64, H_q=64, H_kv=8, D=128, N_i = floor(exp(U[ln 256, ln 131072]));
              rows 0-15 share their first 128 physical pages (a 2048-token
              prefix) and have N_i >= 2049
+  bimodal, uniform, zipf
+             B=8, H_q=32, H_kv=8, D=128 traces in the style of the pages'
+             study (their parameters are not published; see make())
 
 For the last three the pool holds 1.25x the pages the rows need; a random
 permutation of the pool is dealt to the rows in order, so every row's pages
@@ -38,7 +41,7 @@ SEED_CALIBRATE = 20260622
 SEED_REPORT = 20260623
 PAGE = 16
 
-NAMES = ("tiny", "long", "crossover", "mixed", "prefix")
+NAMES = ("tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf")
 
 
 @dataclass
@@ -123,6 +126,24 @@ def make(name: str, seed: int = SEED_REPORT, device="cpu", poison: bool = False,
             lens = torch.randint(4096, 16384 + 1, (B,), generator=g).tolist()
         else:
             lens = [n - 1 if n % PAGE == 0 else n for n in _log_uniform(g, B, 512, 32768)]
+        return _finish(name, seed, device, poison, layout, q_scale, g, B, H_q, H_kv, D, lens)
+    elif name in ("bimodal", "uniform", "zipf"):
+        # B=8 traces shaped like the pages' study traces, whose parameters are
+        # not published; these are generated and stated here:
+        #   bimodal  4 rows U[256, 1024] and 4 rows U[16384, 32768], shuffled
+        #   uniform  8 rows U[512, 32768]
+        #   zipf     N_k = 32768 / k (k = 1..8) times U[0.9, 1.1]
+        B, H_q, H_kv, D = 8, 32, 8, 128
+        if name == "bimodal":
+            lens = (torch.randint(256, 1024 + 1, (4,), generator=g).tolist() +
+                    torch.randint(16384, 32768 + 1, (4,), generator=g).tolist())
+            order = torch.randperm(B, generator=g).tolist()
+            lens = [lens[k] for k in order]
+        elif name == "uniform":
+            lens = torch.randint(512, 32768 + 1, (B,), generator=g).tolist()
+        else:
+            jitter = (0.9 + 0.2 * torch.rand(B, generator=g, dtype=torch.float64)).tolist()
+            lens = [max(1, int(32768 / (k + 1) * jitter[k])) for k in range(B)]
         return _finish(name, seed, device, poison, layout, q_scale, g, B, H_q, H_kv, D, lens)
     elif name == "prefix":
         B, H_q, H_kv, D = 64, 64, 8, 128
