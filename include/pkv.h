@@ -75,6 +75,16 @@ typedef enum {
 #define PKV_FLAG_DEEP_RING 4      /* split kernel with a 12-page shared-memory ring (two blocks per
                                      SM) instead of 8 pages (three blocks per SM): more bytes in
                                      flight per block, for grids of about two blocks per SM */
+#define PKV_FLAG_PDL_EARLY 16     /* the caller promises that the kernel queued right before this call
+                                     writes neither seq_lens, block_table, the queue nor any K/V page
+                                     except each row's last one: the split kernel then reads those and
+                                     starts copying pages before waiting for that kernel (it still
+                                     waits before q, a row's last page and any write).  Ignored by the
+                                     balanced mode, which always waits first. */
+#define PKV_FLAG_CLUSTER_MERGE 8  /* SPLIT_S with S <= 16 only: the S blocks of each (row, KV head)
+                                     run as one thread-block cluster and merge their states through
+                                     distributed shared memory (no partial states in the workspace,
+                                     no merge launch); other modes return PKV_ERR_UNSUPPORTED */
 
 /* Problem shape and pool layout.  Pool element (page, kv_head, slot, d) of
  * k_pool / v_pool lives at  page*kv_stride_page + kv_head*kv_stride_head +

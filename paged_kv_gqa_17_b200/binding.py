@@ -19,7 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libpkv.so")
 
 NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED = 0, 1, 2, 3
-FLAG_SEPARATE_MERGE, FLAG_NO_PDL, FLAG_DEEP_RING = 1, 2, 4
+FLAG_SEPARATE_MERGE, FLAG_NO_PDL, FLAG_DEEP_RING, FLAG_CLUSTER_MERGE, FLAG_PDL_EARLY = 1, 2, 4, 8, 16
 INT32_MAX = 2**31 - 1
 _MODE_NAMES = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE, "BALANCED": BALANCED}
 

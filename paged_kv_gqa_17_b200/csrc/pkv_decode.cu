@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -74,6 +75,7 @@ struct __align__(64) Params {
     float scale_log2;  // scale * log2(e): logits are kept in the log2 domain
     int32_t B, H_q, H_kv, G, max_pages, num_pool_pages;
     int32_t mode, num_splits, chunk_pages, separate_merge;
+    int32_t pdl_early;  // may read lengths, table and KV pages (but a row's last) before the dependency wait
     int32_t n_items;
 #ifdef PKV_TRACE
     int32_t trace_epoch;
@@ -215,6 +217,44 @@ __device__ __forceinline__ void grid_launch_dependents()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Thread-block clusters: rank in the cluster, a full cluster barrier
+// (release / acquire), and loads from a peer block's shared memory.
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // Barrier among the first `threads` threads of the block (named barrier `id`).
 __device__ __forceinline__ void named_barrier(int id, int threads)
 {
@@ -331,6 +371,10 @@ struct Cfg {
     static constexpr int kMiscOff = kBarOff + 2 * NST * 8;  // int flag, then two merge mbarriers at +8, +16
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + slack to align the base to 1024
     static constexpr int kMaxMergeTasks = (kGP * (D / 4) + kThreads - 1) / kThreads;
+    // cluster merge: this block's final state [m: 16][l: 16][acc: kGP][D] in the idle ring
+    static constexpr int kClusterOff = (kCombineBytes + 127) / 128 * 128;
+    static constexpr int kClusterBytes = 128 + kGP * D * 4;
+    static_assert(kClusterOff + kClusterBytes <= kRingBytes, "cluster state must fit in the ring");
 };
 
 // Merge the nslots partial states of one (row, KV head) in ascending slot
@@ -395,11 +439,15 @@ __device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslot
 template <int D, int NST>
 __device__ __forceinline__ bool issue_pages(const Params &p, int lane, int e, int cnt, int &gp, int head,
                                             uint32_t k_ring, uint32_t v_ring, uint32_t bar_full, uint32_t bar_empty,
-                                            uint64_t policy)
+                                            uint64_t policy, int gate = INT_MAX)
 {
     constexpr int kStage = D * kPage * 2;
     bool ok = true;
     for (int j0 = 0; j0 < cnt && ok; j0 += PKV_ISSUE_LANES) {
+        // the page at ring position `gate` may be written by the previous
+        // kernel: wait for it (whole warp) before copying it
+        if (gp + j0 <= gate && gate < gp + j0 + PKV_ISSUE_LANES)
+            grid_dependency_wait();
         const int j = j0 + lane;
         const int phys = __shfl_sync(0xffffffffu, e, j & 31);
         bool my_ok = true;
@@ -533,6 +581,26 @@ __device__ __forceinline__ void attend_page(uint8_t *smem, uint32_t sbase, uint3
             mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
 }
 
+// (M, L, O) <- (M, L, O) merged with the state (m2, l2, o2); neutral states
+// (max = -inf) carry no weight.
+__device__ __forceinline__ void merge_into(float &M, float &L, float4 &O, float m2, float l2, float4 o2)
+{
+    if (m2 == -INFINITY)
+        return;
+    if (M == -INFINITY) {
+        M = m2;
+        L = l2;
+        O = o2;
+        return;
+    }
+    const float Mn = fmaxf(M, m2);
+    const float a = exp2_approx(M - Mn);
+    const float b = exp2_approx(m2 - Mn);
+    L = fmaf(L, a, l2 * b);
+    O = fma4(O, a, scale4(o2, b));
+    M = Mn;
+}
+
 // Merge of one (row, KV head)'s n partial states by the block that finished
 // it last, staged through the idle shared-memory ring.  The weights
 // w_s = 2^(m_s - M) (M = max_s m_s, 0 for a neutral state) and the
@@ -652,7 +720,7 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
 }
 
 // One block = one work item (row, KV head, token range) for all G query heads.
-template <int D, int NT, int NW, int NST>
+template <int D, int NT, int NW, int NST, bool CL>
 __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_constant__ Params p)
 {
     using C = Cfg<D, NT, NW, NST>;
@@ -672,8 +740,12 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     PKV_TRACE_POINT(0);
     // Under programmatic dependent launch this block may start while the
     // previous kernel on the stream is still running: wait before touching
-    // any global memory it may have written.
-    grid_dependency_wait();
+    // any global memory it may have written.  With pdl_early the caller
+    // promises that kernel writes neither the lengths, the table, the queue
+    // nor any KV page but a row's last, so those are read first and the wait
+    // comes before q, the last page and any global write.
+    if (!p.pdl_early)
+        grid_dependency_wait();
 
     // ---- which (row, KV head, token range) this block owns ----
     // The producer warp fetches the first 32 block-table entries of the
@@ -681,6 +753,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     // no-split and split-S grids is before the row length arrives.
     int row, h, tb, te, slot0 = 0, nslots = 1, my_slot = 0;
     int e_first = 0;
+    int row_len = -1;  // the row's length where known (for the early dependency gate)
     if (p.mode == PKV_WORK_QUEUE) {
         const int4 it = __ldg(p.items + blockIdx.x);
         row = it.x;
@@ -706,6 +779,8 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             const int idx = tb / kPage + lane;
             if (idx < p.max_pages)
                 e_first = __ldg(p.block_table + (int64_t)row * p.max_pages + idx);
+            if (p.pdl_early)
+                row_len = __ldg(p.seq_lens + row);
         }
     } else {
         const int S = p.mode == PKV_SPLIT_S ? p.num_splits : 1;
@@ -724,6 +799,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
                 atomicOr(p.ws_error, kErrSeqLen);
             N = N < 0 ? 0 : (int)row_cap;
         }
+        row_len = N;
         if (p.mode == PKV_SPLIT_S) {
             const int64_t span = (int64_t)p.chunk_pages * kPage;
             if (c == 0 && tid == 0 && (int64_t)S * span < N)
@@ -793,6 +869,15 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         int e_next = lane < npages ? e_first : 0;
         bool ok = true;
         int gp = 0;
+        // ring position of the row's last page, which the previous kernel may write
+        int gate = INT_MAX;
+        if (p.pdl_early) {
+            const int last = row_len > 0 ? (row_len - 1) / kPage : (row_len < 0 ? pg0 : -1);
+            if (last >= pg0 && last < pg0 + npages)
+                gate = last - pg0;
+            else if (row_len < 0 || row_len > row_cap)
+                gate = 0;  // unknown or invalid length: wait before the first copy
+        }
         for (int base = 0; base < npages && ok; base += 32) {
             int e = e_next;
             e_next = base + 32 + lane < npages ? __ldg(bt + base + 32 + lane) : 0;
@@ -805,11 +890,13 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
 #ifdef PKV_TRACE
             const long long tw0 = clock64();
 #endif
-            ok = issue_pages<D, NST>(p, lane, e, cnt, gp, h, k_ring, v_ring, bar_full, bar_empty, policy);
+            ok = issue_pages<D, NST>(p, lane, e, cnt, gp, h, k_ring, v_ring, bar_full, bar_empty, policy, gate);
 #ifdef PKV_TRACE
             prod_wait += clock64() - tw0;
 #endif
         }
+        if (p.pdl_early)
+            grid_dependency_wait();  // before this warp's share of the global writes below
 #ifdef PKV_TRACE
         if (lane == 0 && blockIdx.x < kTraceBlocks) {
             g_pkv_trace[blockIdx.x][10] = prod_wait;
@@ -819,6 +906,8 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     } else {
         // ================= consumers: tensor-core attention over pages =================
         // Q as the MMA's B operand (k = head_dim, n = query head), loaded once.
+        if (p.pdl_early)
+            grid_dependency_wait();  // q may come from the previous kernel
         uint32_t qf[D / 16][NT][2];
         const __nv_bfloat16 *qb = p.q + ((int64_t)row * p.H_q + (int64_t)h * p.G) * D;
 #pragma unroll
@@ -931,7 +1020,14 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
             L = fmaf(cb_l[w * C::kGP + g], sc, L);
             O = fma4(*reinterpret_cast<const float4 *>(cb_o + (w * C::kGP + g) * C::kOStride + d4), sc, O);
         }
-        if (nslots == 1) {
+        if (CL) {
+            float *cs = reinterpret_cast<float *>(smem + C::kClusterOff);
+            *reinterpret_cast<float4 *>(cs + 32 + g * D + d4) = O;
+            if (d4 == 0) {
+                cs[g] = M;
+                cs[16 + g] = L;
+            }
+        } else if (nslots == 1) {
             const float inv = L > 0.f ? 1.f / L : 0.f;
             store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
         } else {
@@ -945,8 +1041,46 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     }
 
     PKV_TRACE_POINT(4);
+    if (CL) {
+        // ---- cluster merge: the S blocks of this (row, KV head) form one
+        // cluster; each merges a slice of the (head, 4-column) tasks over all
+        // S states, read from the peers' shared memory in rank order ----
+        cluster_sync_all();
+        const uint32_t cs_addr = sbase + C::kClusterOff;
+        const int S = nslots;
+        const int T = G * D4;
+        const int per = (T + S - 1) / S;
+        const int e0 = (int)cluster_ctarank() * per;
+        const int e1 = e0 + per < T ? e0 + per : T;
+        for (int e = e0 + tid; e < e1; e += C::kThreads) {
+            const int g = e / D4;
+            const int d4 = (e % D4) * 4;
+            float ms[16], ls[16];
+            float4 as[16];
+#pragma unroll
+            for (int src = 0; src < 16; ++src) {
+                ms[src] = -INFINITY;
+                ls[src] = 0.f;
+                as[src] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (src < S) {
+                    const uint32_t base = map_shared_rank(cs_addr, (uint32_t)src);
+                    ms[src] = ld_cluster_f32(base + 4 * g);
+                    ls[src] = ld_cluster_f32(base + 64 + 4 * g);
+                    as[src] = ld_cluster_f32x4(base + 128 + 4 * (g * D + d4));
+                }
+            }
+            float M = -INFINITY, L = 0.f;
+            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int src = 0; src < 16; ++src)
+                merge_into(M, L, O, ms[src], ls[src], as[src]);
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+        }
+        cluster_sync_all();  // peers may still be reading this block's state
+    }
     // ---- the last block of a split (row, KV head) merges its states ----
-    if (nslots > 1 && !p.separate_merge) {
+    if (!CL && nslots > 1 && !p.separate_merge) {
         __syncthreads();
         if (tid == 0) {
             const uint32_t prev = ticket_acq_rel(p.ws_counters + pair);
@@ -1241,26 +1375,6 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
     }
 }
 
-// (M, L, O) <- (M, L, O) merged with the state (m2, l2, o2); neutral states
-// (max = -inf) carry no weight.
-__device__ __forceinline__ void merge_into(float &M, float &L, float4 &O, float m2, float l2, float4 o2)
-{
-    if (m2 == -INFINITY)
-        return;
-    if (M == -INFINITY) {
-        M = m2;
-        L = l2;
-        O = o2;
-        return;
-    }
-    const float Mn = fmaxf(M, m2);
-    const float a = exp2_approx(M - Mn);
-    const float b = exp2_approx(m2 - Mn);
-    L = fmaf(L, a, l2 * b);
-    O = fma4(O, a, scale4(o2, b));
-    M = Mn;
-}
-
 // Separate merge (chained to the split kernel by programmatic dependent
 // launch): one block per (row, KV head); pairs with one slot were finalized
 // by the split kernel.  Four threads share each (head, 4-column) task; a
@@ -1481,40 +1595,67 @@ cudaError_t set_smem(K kernel, int bytes, std::atomic<uint64_t> &done_mask)
 
 template <typename... Args>
 cudaError_t launch_ex(void (*kernel)(Args...), unsigned grid, unsigned block, size_t smem, cudaStream_t st, bool pdl,
-                      const Params &prm)
+                      const Params &prm, unsigned cluster = 0)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kernel, prm);
 }
 
-template <int D, int NT, int NST>
-cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+template <int D, int NT, int NST, bool CL>
+cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st, bool pdl, unsigned cluster)
 {
     using C = Cfg<D, NT, kNW, NST>;
     static std::atomic<uint64_t> configured{0};
-    auto kernel = split_kernel<D, NT, kNW, NST>;
+    auto kernel = split_kernel<D, NT, kNW, NST, CL>;
     cudaError_t e = set_smem(kernel, C::kSmemBytes, configured);
     if (e != cudaSuccess)
         return e;
-    e = launch_ex(kernel, (unsigned)grid, C::kThreads, C::kSmemBytes, st, pdl, prm);
+    if (CL && cluster > 8) {
+        static std::atomic<uint64_t> wide{0};
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess)
+            return e;
+        const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+        if (!(bit && (wide.load() & bit))) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess)
+                return e;
+            wide.fetch_or(bit);
+        }
+    }
+    e = launch_ex(kernel, (unsigned)grid, C::kThreads, C::kSmemBytes, st, pdl, prm, CL ? cluster : 0);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int NST>
-cudaError_t launch_split_nst(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+template <int NST, bool CL>
+cudaError_t launch_split_nst(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st, bool pdl,
+                             unsigned cluster)
 {
     if (D == 128)
-        return NT == 1 ? launch_split<128, 1, NST>(prm, grid, st, pdl) : launch_split<128, 2, NST>(prm, grid, st, pdl);
-    return NT == 1 ? launch_split<64, 1, NST>(prm, grid, st, pdl) : launch_split<64, 2, NST>(prm, grid, st, pdl);
+        return NT == 1 ? launch_split<128, 1, NST, CL>(prm, grid, st, pdl, cluster)
+                       : launch_split<128, 2, NST, CL>(prm, grid, st, pdl, cluster);
+    return NT == 1 ? launch_split<64, 1, NST, CL>(prm, grid, st, pdl, cluster)
+                   : launch_split<64, 2, NST, CL>(prm, grid, st, pdl, cluster);
 }
 
 #ifndef PKV_NST_BAL
@@ -1546,10 +1687,14 @@ cudaError_t launch_balanced_nst(int D, int NT, const Params &prm, int64_t grid, 
     return NT == 1 ? launch_balanced<64, 1, NST>(prm, grid, st, pdl) : launch_balanced<64, 2, NST>(prm, grid, st, pdl);
 }
 
-cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl,
+                             unsigned cluster)
 {
-    return deep ? launch_split_nst<kNSTDeep>(D, NT, prm, grid, st, pdl)
-                : launch_split_nst<kNST>(D, NT, prm, grid, st, pdl);
+    if (cluster > 0)
+        return deep ? launch_split_nst<kNSTDeep, true>(D, NT, prm, grid, st, pdl, cluster)
+                    : launch_split_nst<kNST, true>(D, NT, prm, grid, st, pdl, cluster);
+    return deep ? launch_split_nst<kNSTDeep, false>(D, NT, prm, grid, st, pdl, 0)
+                : launch_split_nst<kNST, false>(D, NT, prm, grid, st, pdl, 0);
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -1586,6 +1731,8 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         return PKV_ERR_INVALID;
     if (pl.mode == PKV_BALANCED && pl.num_splits < 1)
         return PKV_ERR_INVALID;
+    if ((pl.flags & PKV_FLAG_CLUSTER_MERGE) && (pl.mode != PKV_SPLIT_S || pl.num_splits > 16))
+        return PKV_ERR_UNSUPPORTED;
     int rc = check_fast_path(s);
     if (rc != PKV_OK)
         return rc;
@@ -1632,6 +1779,7 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.num_splits = pl.mode == PKV_SPLIT_S ? pl.num_splits : 1;
     prm.chunk_pages = pl.chunk_pages;
     prm.separate_merge = (pl.flags & PKV_FLAG_SEPARATE_MERGE) ? 1 : 0;
+    prm.pdl_early = (pl.flags & PKV_FLAG_PDL_EARLY) && !(pl.flags & PKV_FLAG_NO_PDL) ? 1 : 0;
     prm.n_items = n_items;
 #ifdef PKV_TRACE
     static std::atomic<int32_t> trace_launches{0};
@@ -1648,15 +1796,17 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     const int NT = prm.G <= 8 ? 1 : 2;
     const bool pdl = (pl.flags & PKV_FLAG_NO_PDL) == 0;
     const bool deep = (pl.flags & PKV_FLAG_DEEP_RING) != 0;
+    // cluster merge: the S blocks of each (row, KV head) form one cluster
+    const unsigned cluster = (pl.flags & PKV_FLAG_CLUSTER_MERGE) ? (unsigned)pl.num_splits : 0u;
     cudaError_t le;
     if (pl.mode == PKV_BALANCED)
         le = deep ? launch_balanced_nst<PKV_NST_BAL_DEEP>(s.head_dim, NT, prm, grid, st, pdl)
                   : launch_balanced_nst<PKV_NST_BAL>(s.head_dim, NT, prm, grid, st, pdl);
     else
-        le = launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl);
+        le = launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl, cluster);
     if (le != cudaSuccess)
         return PKV_ERR_CUDA;
-    const bool need_merge = pl.mode != PKV_NO_SPLIT && prm.separate_merge;
+    const bool need_merge = pl.mode != PKV_NO_SPLIT && prm.separate_merge && cluster == 0;
     if (need_merge) {
         cudaError_t e = s.head_dim == 128
                             ? launch_ex(merge_kernel<128>, (unsigned)pairs, kMergeThreads, 0, st, pdl, prm)

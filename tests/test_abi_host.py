@@ -166,6 +166,10 @@ def test_decode_rejects_unsupported_shapes_without_touching_the_gpu(L):
     rc = L.pkv_paged_decode(None, None, None, None, None, 16, 1.0, None, ctypes.byref(shape), ctypes.byref(wq),
                             None, None, 0, None, 0, None)
     assert rc == -1  # work queue without items
+    for bad_cluster in (bd.Plan(1, 17, 4, 8), bd.Plan(0, 1, 0, 8)):
+        rc = L.pkv_paged_decode(None, None, None, None, None, 16, 1.0, None, ctypes.byref(shape),
+                                ctypes.byref(bad_cluster), None, None, 0, None, 0, None)
+        assert rc == -2  # cluster merge only for split-S with S <= 16
 
 
 def test_host_pins_hold_for_the_c_planner(L):

@@ -40,6 +40,11 @@ MODES = {
     "bal296": rule(3, 296),
     "bal148_deep": rule(3, 148, 0, 4),
     "bal64_sep": rule(3, 64, 0, 1),
+    "split16_cl": rule(1, 16, 0, 8),
+    "split8_cl_deep": rule(1, 8, 0, 12),
+    "split3_cl": rule(1, 3, 0, 8),
+    "split1_cl": rule(1, 1, 0, 8),
+    "split12_cl_nopdl": rule(1, 12, 0, 10),
 }
 
 
@@ -76,7 +81,7 @@ CASES = {
 @pytest.mark.parametrize("case", sorted(CASES))
 @pytest.mark.parametrize("mode", ["nosplit", "split7", "split32", "split32_sep", "wq3", "wq3_sep", "split32_deep",
                                   "wq3_deep_sep", "split7_nopdl", "bal1", "bal7", "bal296", "bal148_deep",
-                                  "bal64_sep"])
+                                  "bal64_sep", "split16_cl", "split8_cl_deep", "split3_cl", "split12_cl_nopdl"])
 def test_ragged_shapes(case, mode):
     lens, H_q, H_kv, D = CASES[case]
     w = to_device(W.make_custom(lens, H_q, H_kv, D, seed=101, poison=True, q_scale=3.0))
@@ -94,7 +99,7 @@ def test_nhd_layout(mode):
     assert_close(got, ref, f"nhd/{mode}")
 
 
-@pytest.mark.parametrize("mode", ["nosplit", "split32", "wq3", "bal37"])
+@pytest.mark.parametrize("mode", ["nosplit", "split32", "wq3", "bal37", "split16_cl"])
 def test_peaked_logits(mode):
     """q scaled x8: logits ~ N(0, 64), a few tokens dominate; tests the
     running-max rescaling across pages and across splits."""
@@ -132,6 +137,9 @@ def test_deterministic_and_page_permutation_bit_identical():
     a, _ = run(w, mode_rule=MODES["split32"])
     b, _ = run(w, mode_rule=MODES["split32"])
     assert np.array_equal(a, b)
+    c1, _ = run(w, mode_rule=MODES["split16_cl"])
+    c2, _ = run(w, mode_rule=MODES["split16_cl"])
+    assert np.array_equal(c1, c2)
     perm = torch.randperm(w.num_pages, generator=torch.Generator().manual_seed(5)).cuda()
     inv = torch.empty_like(perm)
     inv[perm] = torch.arange(w.num_pages, device="cuda")
@@ -144,7 +152,8 @@ def test_deterministic_and_page_permutation_bit_identical():
 def test_split_counts_do_not_change_the_answer_beyond_rounding():
     w = to_device(W.make_custom([5000, 1234], 32, 8, 128, seed=108, poison=True))
     ref = oracle_full(w)
-    for mode in ("nosplit", "split2", "split7", "split32", "wq1", "wq16", "bal1", "bal7", "bal37", "bal296"):
+    for mode in ("nosplit", "split2", "split7", "split32", "wq1", "wq16", "bal1", "bal7", "bal37", "bal296",
+                 "split16_cl", "split1_cl"):
         got, _ = run(w, mode_rule=MODES[mode])
         assert_close(got, ref, mode)
 
@@ -211,7 +220,7 @@ def test_prefix_sharing_config_sampled():
 
 
 @pytest.mark.parametrize("name", ["long", "crossover", "mixed"])
-@pytest.mark.parametrize("mode", ["bal296", "bal148_deep"])
+@pytest.mark.parametrize("mode", ["bal296", "bal148_deep", "split16_cl"])
 def test_full_size_configs_balanced_sampled(name, mode):
     w = to_device(W.make(name, poison=True))
     got, dp = run(w, mode_rule=MODES[mode])
@@ -229,3 +238,27 @@ def test_balanced_deterministic_across_runs_and_deferred_merges():
     b, _ = run(w, mode_rule=rule(3, 24))
     assert np.array_equal(a, b)
     assert_close(a, oracle_full(w), "balanced B=40 T=24")
+
+
+@pytest.mark.parametrize("flags_rule", [rule(1, 32, 0, 4 | 16), rule(2, 1, 3, 16), rule(0, 1, 0, 16),
+                                        rule(1, 16, 0, 8 | 16), rule(1, 7, 0, 1 | 16)])
+def test_pdl_early_back_to_back_steps(flags_rule):
+    """Opt-in early start: consecutive decode steps on one stream, each allowed
+    to read the table, lengths and K/V before the previous one finishes.  The
+    previous kernel (a decode step) writes none of them, so every step must
+    still match the oracle."""
+    w = to_device(W.make_custom([3000, 77, 1999, 16], 32, 8, 128, seed=120, poison=True))
+    ref = oracle_full(w)
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", rules=[flags_rule])
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
+    outs = [torch.empty_like(w.q) for _ in range(6)]
+    torch.cuda.synchronize()
+    for out in outs:
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    torch.cuda.synchronize()
+    assert bd.workspace_status(dp) == 0
+    first = outs[0].float().cpu()
+    for out in outs:
+        assert torch.equal(out.float().cpu(), first)
+    assert_close(first.double().numpy(), ref, f"pdl early {dp.plan}")
