@@ -319,15 +319,19 @@ PKV_API int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape 
 
 /* One synchronous decode step from host buffers, the way a serving loop
  * calls it [PKV, Methodology 3 "Evaluation protocol": synchronized wall time
- * including host planning]: pick the plan (pkv_select_policy), build the
- * queue into host_staging (pkv_build_work_queue), copy q, block_table,
- * seq_lens and the queue host->device into device_buffer, zero the
- * completion counters, run pkv_paged_decode, copy out device->host and
- * synchronize `stream`.  q_host, block_table_host, seq_lens_host, out_host
- * are host pointers with the layouts of pkv_paged_decode; k_pool / v_pool
- * are device pools (the cache stays resident on the device).  The plan used
- * is written to *plan_out when not NULL.  Returns the device error status
- * like pkv_workspace_status when the kernels ran. */
+ * including host planning]: pick the plan (pkv_select_policy), build its
+ * queue into host_staging (pkv_build_work_queue or pkv_build_balanced_queue),
+ * move q, seq_lens, block_table, the queue and the zeroed completion
+ * counters and error word host->device in ONE copy, run pkv_paged_decode,
+ * move the error word and out device->host in ONE copy and synchronize
+ * `stream`.  q, block_table and out larger than 64 KiB each get a copy of
+ * their own instead of travelling through the staging buffer.  q_host,
+ * block_table_host, seq_lens_host, out_host are host pointers with the
+ * layouts of pkv_paged_decode; k_pool / v_pool are device pools (the cache
+ * stays resident on the device).  device_buffer must be 256-byte aligned
+ * (PKV_ERR_UNSUPPORTED otherwise); it needs no zeroing.  The plan used is
+ * written to *plan_out when not NULL.  Returns the device error status like
+ * pkv_workspace_status when the kernels ran. */
 PKV_API int pkv_decode_host(const void *q_host, const int32_t *block_table_host,
                             const int32_t *seq_lens_host, void *out_host, const void *k_pool,
                             const void *v_pool, float scale, const pkv_shape *shape,

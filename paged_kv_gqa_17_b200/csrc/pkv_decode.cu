@@ -51,6 +51,17 @@
 
 #include "pkv_internal.h"
 
+// One rank-5 TMA copy per K (or V) page; 0 selects one rank-4 copy per
+// 64-wide half of head_dim.
+#ifndef PKV_TMA_5D
+#define PKV_TMA_5D 1
+#endif
+// Pages per block that the split kernel prefetches into L2 while it waits for
+// the kernel before it (0 turns the prefetch off).
+#ifndef PKV_L2_PREFETCH_PAGES
+#define PKV_L2_PREFETCH_PAGES 8
+#endif
+
 namespace pkv {
 
 constexpr int kBoxD = 64;                   // head-dim elements per TMA box row (128 bytes)
@@ -273,6 +284,44 @@ __device__ __forceinline__ void tma_load_page(uint32_t dst, const CUtensorMap *t
         : "memory");
 }
 
+// L2 prefetch of one (page, head) block through the same tensor map: no
+// shared memory, no barrier; coordinates outside the tensor fetch nothing.
+template <int D>
+__device__ __forceinline__ void tma_prefetch_page_l2(const CUtensorMap *tm, int head, int page)
+{
+#if PKV_TMA_5D
+    asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(0), "r"(0), "r"(0), "r"(head), "r"(page)
+                 : "memory");
+#else
+    for (int d0 = 0; d0 < D; d0 += kBoxD)
+        asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                         reinterpret_cast<uint64_t>(tm)),
+                     "r"(d0), "r"(0), "r"(head), "r"(page)
+                     : "memory");
+#endif
+}
+
+// Loads that are cached in L2 only (never in L1), for reads of data that a
+// kernel still running may be writing: a later load of the same address
+// after the dependency wait cannot hit a stale L1 line.
+__device__ __forceinline__ int ld_l2_only(const int32_t *ptr)
+{
+    int v;
+    asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(ptr));
+    return v;
+}
+
+__device__ __forceinline__ int4 ld_l2_only(const int4 *ptr)
+{
+    int4 v;
+    asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(ptr));
+    return v;
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *tm)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
@@ -422,11 +471,8 @@ __device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslot
 }
 
 // The producer's issue rate bounds a block's bandwidth: one rank-5 TMA copy
-// per K (or V) page instead of one per 64-wide half, issued by several lanes
-// at once.
-#ifndef PKV_TMA_5D
-#define PKV_TMA_5D 1
-#endif
+// per K (or V) page instead of one per 64-wide half (PKV_TMA_5D, defined
+// above), issued by several lanes at once.
 #ifndef PKV_ISSUE_LANES
 #define PKV_ISSUE_LANES 4
 #endif
@@ -719,6 +765,55 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
     return true;
 }
 
+// Before its dependency wait the split kernel may read nothing that the
+// kernel before it might still be writing.  What it may do is warm L2: the
+// producer warp reads its range (work item or row length) and the first
+// block-table entries speculatively, through L2 only, and asks the TMA unit to
+// prefetch the first PKV_L2_PREFETCH_PAGES K/V pages of the range into L2.
+// A stale or torn value costs only a useless prefetch (page ids are range
+// checked, and a prefetch moves no data into the block); everything the block
+// uses is read again after the wait, and L2 is coherent with the writes of
+// the kernel before.  In a back-to-back decode loop this streams the first
+// pages while the previous step finishes its merges.
+template <int D>
+__device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lane, int64_t row_cap)
+{
+#if PKV_L2_PREFETCH_PAGES > 0
+    int row, h;
+    int64_t pg0, pg_end;
+    if (p.mode == PKV_WORK_QUEUE) {
+        const int4 it = ld_l2_only(p.items + blockIdx.x);
+        if (!(it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w && it.w <= row_cap))
+            return;
+        row = it.x;
+        h = it.y;
+        pg0 = it.z / kPage;
+        pg_end = (it.w + kPage - 1) / kPage;
+    } else {
+        const int S = p.mode == PKV_SPLIT_S ? p.num_splits : 1;
+        const int pair = blockIdx.x / S;
+        row = pair / p.H_kv;
+        h = pair % p.H_kv;
+        int64_t N = ld_l2_only(p.seq_lens + row);
+        N = N < 0 ? 0 : (N > row_cap ? row_cap : N);
+        pg_end = (N + kPage - 1) / kPage;
+        pg0 = 0;
+        if (p.mode == PKV_SPLIT_S) {
+            pg0 = (int64_t)(blockIdx.x % S) * p.chunk_pages;
+            pg_end = pg_end < pg0 + p.chunk_pages ? pg_end : pg0 + p.chunk_pages;
+        }
+    }
+    const int64_t j = pg0 + lane;
+    if (lane < PKV_L2_PREFETCH_PAGES && j < pg_end) {
+        const int e = ld_l2_only(p.block_table + (int64_t)row * p.max_pages + j);
+        if (e >= 0 && e < p.num_pool_pages) {
+            tma_prefetch_page_l2<D>(&p.tm_k, h, e);
+            tma_prefetch_page_l2<D>(&p.tm_v, h, e);
+        }
+    }
+#endif
+}
+
 // One block = one work item (row, KV head, token range) for all G query heads.
 template <int D, int NT, int NW, int NST, bool CL>
 __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_constant__ Params p)
@@ -738,14 +833,34 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     const int lane = tid & 31;
     const int64_t row_cap = (int64_t)p.max_pages * kPage;
     PKV_TRACE_POINT(0);
+    // Set-up that reads no global data comes first: the ring's barriers and
+    // the tensor maps (kernel parameters).
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(sbase + C::kMiscOff + 8, 1);
+        mbar_init(sbase + C::kMiscOff + 16, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+    }
     // Under programmatic dependent launch this block may start while the
-    // previous kernel on the stream is still running: wait before touching
-    // any global memory it may have written.  With pdl_early the caller
+    // previous kernel on the stream is still running: wait before reading
+    // any global memory it may have written (after warming L2 with the
+    // first pages, see l2_prefetch_first_pages).  With pdl_early the caller
     // promises that kernel writes neither the lengths, the table, the queue
     // nor any KV page but a row's last, so those are read first and the wait
     // comes before q, the last page and any global write.
-    if (!p.pdl_early)
+    if (!p.pdl_early) {
+        if (warp == NW)
+            l2_prefetch_first_pages<D>(p, lane, row_cap);
         grid_dependency_wait();
+    }
 
     // ---- which (row, KV head, token range) this block owns ----
     // The producer warp fetches the first 32 block-table entries of the
@@ -819,21 +934,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
     const int pg0 = tb / kPage;
     const int npages = te > tb ? (te + kPage - 1) / kPage - pg0 : 0;
 
-    if (tid == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1);
-        }
-        mbar_init(sbase + C::kMiscOff + 8, 1);
-        mbar_init(sbase + C::kMiscOff + 16, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        fence_proxy_async_smem();
-    }
-    if (warp == NW && lane == 0) {
-        prefetch_tensormap(&p.tm_k);
-        prefetch_tensormap(&p.tm_v);
-    }
-    __syncthreads();
+    __syncthreads();  // the barriers' initialisation is visible to all warps
     PKV_TRACE_POINT(1);
 #ifdef PKV_TRACE
     if (tid == 0 && blockIdx.x < kTraceBlocks) {
@@ -1712,11 +1813,23 @@ int check_fast_path(const pkv_shape &s)
 
 }  // namespace
 
-// Internal entry shared by pkv_paged_decode and pkv_decode_host.
+// Device addresses of the workspace sections (error word, completion
+// counters, partial states); normally carved out of one workspace by
+// ws_layout, placed one by one by pkv_decode_host.
+struct WsPtrs {
+    uint32_t *error;
+    uint32_t *counters;
+    float *m, *l, *acc;
+};
+
+// Internal entry shared by pkv_paged_decode, pkv_paged_decode_noalloc and
+// pkv_decode_host.  With `sections` NULL the workspace sections are carved
+// out of `workspace` (checked against workspace_bytes); otherwise they are
+// taken from `sections` and workspace/workspace_bytes are ignored.
 int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, const int32_t *block_table,
                       const int32_t *seq_lens, int32_t page_size, float scale, void *out, const pkv_shape *shape,
                       const pkv_plan *plan, const pkv_work_item *items, const int32_t *indptr, int32_t n_items,
-                      void *workspace, size_t workspace_bytes, cudaStream_t st)
+                      void *workspace, size_t workspace_bytes, cudaStream_t st, const WsPtrs *sections = nullptr)
 {
     if (check_shape(shape) != PKV_OK || !plan || page_size != shape->page_size)
         return PKV_ERR_INVALID;
@@ -1738,17 +1851,29 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         return rc;
     if (s.B == 0)
         return PKV_OK;
-    if (!q || !k_pool || !v_pool || !seq_lens || !out || !workspace || (!block_table && s.max_pages_per_seq > 0))
+    if (!q || !k_pool || !v_pool || !seq_lens || !out || (!workspace && !sections) ||
+        (!block_table && s.max_pages_per_seq > 0))
         return PKV_ERR_INVALID;
     if (s.num_pool_pages < 1 || s.max_pages_per_seq < 1)
         return PKV_ERR_INVALID;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
-        !aligned(workspace, 256) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+        (!sections && !aligned(workspace, 256)) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
         (items && !aligned(items, 16)) || (indptr && !aligned(indptr, 4)))
         return PKV_ERR_UNSUPPORTED;
-    const WsLayout ws = ws_layout(s, pl, n_items);
-    if (workspace_bytes < ws.total)
-        return PKV_ERR_CAPACITY;
+    WsPtrs wp;
+    if (sections) {
+        wp = *sections;
+    } else {
+        const WsLayout ws = ws_layout(s, pl, n_items);
+        if (workspace_bytes < ws.total)
+            return PKV_ERR_CAPACITY;
+        uint8_t *wsb = static_cast<uint8_t *>(workspace);
+        wp.error = reinterpret_cast<uint32_t *>(wsb + ws.error_off);
+        wp.counters = reinterpret_cast<uint32_t *>(wsb + ws.counters_off);
+        wp.m = reinterpret_cast<float *>(wsb + ws.m_off);
+        wp.l = reinterpret_cast<float *>(wsb + ws.l_off);
+        wp.acc = reinterpret_cast<float *>(wsb + ws.acc_off);
+    }
 
     Params prm;
     std::memset(&prm, 0, sizeof prm);
@@ -1756,18 +1881,17 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         return rc;
     if ((rc = pool_tensor_map(&prm.tm_v, v_pool, s)) != PKV_OK)
         return rc;
-    uint8_t *wsb = static_cast<uint8_t *>(workspace);
     prm.q = static_cast<const __nv_bfloat16 *>(q);
     prm.out = static_cast<__nv_bfloat16 *>(out);
     prm.block_table = block_table;
     prm.seq_lens = seq_lens;
     prm.items = reinterpret_cast<const int4 *>(items);
     prm.indptr = indptr;
-    prm.ws_error = reinterpret_cast<uint32_t *>(wsb + ws.error_off);
-    prm.ws_counters = reinterpret_cast<uint32_t *>(wsb + ws.counters_off);
-    prm.ws_m = reinterpret_cast<float *>(wsb + ws.m_off);
-    prm.ws_l = reinterpret_cast<float *>(wsb + ws.l_off);
-    prm.ws_acc = reinterpret_cast<float *>(wsb + ws.acc_off);
+    prm.ws_error = wp.error;
+    prm.ws_counters = wp.counters;
+    prm.ws_m = wp.m;
+    prm.ws_l = wp.l;
+    prm.ws_acc = wp.acc;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.B = s.B;
     prm.H_q = s.H_q;
@@ -1911,12 +2035,30 @@ void *noalloc_scratch_address()
     return addr[dev];
 }
 
+// pkv_decode_host moves a step's inputs in one host->device copy and its
+// result in one device->host copy.  The device buffer is laid out so that the
+// inputs and the zeroed error word / completion counters form one contiguous
+// upload, and the error word and `out` one contiguous download:
+//
+//   [q*] [seq_lens] [items] [indptr] [block_table*] [counters] [error] [out*] [m] [l] [acc] [q**] [block_table**]
+//   '------------------------ upload --------------------------------'
+//                                                           '-- download --'
+//
+// The host staging buffer holds the same upload image, then the download.
+// q, block_table and out travel inside the packed copies (*) up to
+// kInlineBytes each; larger ones are copied straight from / to the caller's
+// buffers with their own copy (**), where a host-side memcpy into the
+// staging buffer would cost more than one extra copy command.
+constexpr size_t kInlineBytes = size_t(64) << 10;
+
 struct HostLayout {
     pkv_plan plan;
-    int32_t n_items = 0;
-    WsLayout ws;
-    size_t q_off, bt_off, lens_off, out_off, items_off, indptr_off, dev_total;
-    size_t h_items_off, h_indptr_off, h_err_off, host_total;
+    int32_t n_items = 0, n_indptr = 0;
+    bool q_inline, bt_inline, out_inline;
+    size_t q_bytes, bt_bytes;
+    size_t q_off, lens_off, items_off, indptr_off, bt_off, counters_off, err_off, out_off, m_off, l_off, acc_off;
+    size_t up_bytes, down_bytes, dev_total;
+    size_t h_down_off, host_total;
 };
 
 int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_rule *rules, int32_t n_rules,
@@ -1925,36 +2067,53 @@ int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_ru
     int rc = pkv_select_policy(lens, shape, rules, n_rules, &L->plan);
     if (rc != PKV_OK)
         return rc;
+    const pkv_shape &s = *shape;
+    const size_t pairs = (size_t)s.B * s.H_kv;
     L->n_items = 0;
+    L->n_indptr = 0;
     if (L->plan.mode == PKV_WORK_QUEUE) {
         rc = pkv_work_queue_size(lens, shape, L->plan.chunk_pages, &L->n_items);
-        if (rc != PKV_OK)
-            return rc;
+        L->n_indptr = (int32_t)pairs + 1;
+    } else if (L->plan.mode == PKV_BALANCED) {
+        rc = pkv_balanced_queue_size(lens, shape, L->plan.num_splits, &L->n_items);
+        L->n_indptr = (int32_t)pairs + 2 + L->plan.num_splits;
     }
-    const pkv_shape &s = *shape;
-    L->ws = ws_layout(s, L->plan, L->n_items);
-    const size_t pairs = (size_t)s.B * s.H_kv;
-    size_t off = L->ws.total;
-    L->q_off = off;
-    off += round_up((size_t)s.B * s.H_q * s.head_dim * 2, kWsAlign);
-    L->bt_off = off;
-    off += round_up((size_t)s.B * s.max_pages_per_seq * 4, kWsAlign);
-    L->lens_off = off;
-    off += round_up((size_t)s.B * 4, kWsAlign);
-    L->out_off = off;
-    off += round_up((size_t)s.B * s.H_q * s.head_dim * 2, kWsAlign);
-    L->items_off = off;
-    off += round_up((size_t)L->n_items * sizeof(pkv_work_item), kWsAlign);
-    L->indptr_off = off;
-    off += round_up((pairs + 1) * 4, kWsAlign);
+    if (rc != PKV_OK)
+        return rc;
+    const WsLayout ws = ws_layout(s, L->plan, L->n_items);
+    L->q_bytes = (size_t)s.B * s.H_q * s.head_dim * 2;
+    L->bt_bytes = (size_t)s.B * s.max_pages_per_seq * 4;
+    L->q_inline = L->q_bytes <= kInlineBytes;
+    L->out_inline = L->q_inline;
+    L->bt_inline = L->bt_bytes <= kInlineBytes;
+    size_t off = 0;
+    auto take = [&off](size_t bytes) {
+        const size_t at = off;
+        off += round_up(bytes, kWsAlign);
+        return at;
+    };
+    L->q_off = L->q_inline ? take(L->q_bytes) : 0;
+    L->lens_off = take((size_t)s.B * 4);
+    L->items_off = take((size_t)L->n_items * sizeof(pkv_work_item));
+    L->indptr_off = take((size_t)L->n_indptr * 4);
+    L->bt_off = L->bt_inline ? take(L->bt_bytes) : 0;
+    L->counters_off = take(ws.m_off - ws.counters_off);
+    L->err_off = take(kWsAlign);
+    L->up_bytes = L->err_off + 16;
+    L->out_off = take(L->q_bytes);
+    L->down_bytes = L->out_inline ? L->out_off + L->q_bytes - L->err_off : 16;
+    L->m_off = take(ws.l_off - ws.m_off);
+    L->l_off = take(ws.acc_off - ws.l_off);
+    L->acc_off = take(ws.total - ws.acc_off);
+    if (!L->q_inline)
+        L->q_off = take(L->q_bytes);
+    if (!L->bt_inline)
+        L->bt_off = take(L->bt_bytes);
     L->dev_total = off;
-    L->h_items_off = 0;
-    L->h_indptr_off = round_up((size_t)L->n_items * sizeof(pkv_work_item), 64);
-    L->h_err_off = L->h_indptr_off + round_up((pairs + 1) * 4, 64);
-    L->host_total = L->h_err_off + 64;
+    L->h_down_off = round_up(L->up_bytes, kWsAlign);
+    L->host_total = L->h_down_off + round_up(L->down_bytes, kWsAlign);
     return PKV_OK;
 }
-
 }  // namespace
 
 int pkv_paged_decode_noalloc(const void *q, const void *k_pool, const void *v_pool, const int32_t *block_table,
@@ -2013,45 +2172,55 @@ int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const i
         return PKV_ERR_INVALID;
     if (device_buffer_bytes < L.dev_total || host_staging_bytes < L.host_total)
         return PKV_ERR_CAPACITY;
+    if (!aligned(device_buffer, kWsAlign))
+        return PKV_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *dev = static_cast<uint8_t *>(device_buffer);
     uint8_t *hst = static_cast<uint8_t *>(host_staging);
-    pkv_work_item *h_items = reinterpret_cast<pkv_work_item *>(hst + L.h_items_off);
-    int32_t *h_indptr = reinterpret_cast<int32_t *>(hst + L.h_indptr_off);
-    uint32_t *h_err = reinterpret_cast<uint32_t *>(hst + L.h_err_off);
-    if (L.plan.mode == PKV_WORK_QUEUE) {
-        int32_t n = 0;
+    // upload image: inputs, queue, zeroed counters and error word
+    if (L.q_inline)
+        std::memcpy(hst + L.q_off, q_host, L.q_bytes);
+    std::memcpy(hst + L.lens_off, seq_lens_host, (size_t)s.B * 4);
+    if (L.bt_inline)
+        std::memcpy(hst + L.bt_off, block_table_host, L.bt_bytes);
+    std::memset(hst + L.counters_off, 0, L.up_bytes - L.counters_off);
+    pkv_work_item *h_items = reinterpret_cast<pkv_work_item *>(hst + L.items_off);
+    int32_t *h_indptr = reinterpret_cast<int32_t *>(hst + L.indptr_off);
+    int32_t n = 0;
+    if (L.plan.mode == PKV_WORK_QUEUE)
         rc = pkv_build_work_queue(seq_lens_host, shape, L.plan.chunk_pages, h_items, L.n_items, h_indptr, &n);
-        if (rc != PKV_OK)
-            return rc;
-    }
-    const size_t q_bytes = (size_t)s.B * s.H_q * s.head_dim * 2;
-    const size_t bt_bytes = (size_t)s.B * s.max_pages_per_seq * 4;
-    const size_t pairs = (size_t)s.B * s.H_kv;
-    bool ok = cudaMemcpyAsync(dev + L.q_off, q_host, q_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-              cudaMemcpyAsync(dev + L.bt_off, block_table_host, bt_bytes, cudaMemcpyHostToDevice, st) ==
-                  cudaSuccess &&
-              cudaMemcpyAsync(dev + L.lens_off, seq_lens_host, (size_t)s.B * 4, cudaMemcpyHostToDevice, st) ==
-                  cudaSuccess &&
-              cudaMemsetAsync(dev, 0, L.ws.m_off, st) == cudaSuccess;  // error word + completion counters
-    if (ok && L.plan.mode == PKV_WORK_QUEUE)
-        ok = cudaMemcpyAsync(dev + L.items_off, h_items, (size_t)L.n_items * sizeof(pkv_work_item),
-                             cudaMemcpyHostToDevice, st) == cudaSuccess &&
-             cudaMemcpyAsync(dev + L.indptr_off, h_indptr, (pairs + 1) * 4, cudaMemcpyHostToDevice, st) ==
-                 cudaSuccess;
+    else if (L.plan.mode == PKV_BALANCED)
+        rc = pkv_build_balanced_queue(seq_lens_host, shape, L.plan.num_splits, h_items, L.n_items, h_indptr, &n);
+    if (rc != PKV_OK)
+        return rc;
+    bool ok = cudaMemcpyAsync(dev, hst, L.up_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    if (ok && !L.q_inline)
+        ok = cudaMemcpyAsync(dev + L.q_off, q_host, L.q_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    if (ok && !L.bt_inline)
+        ok = cudaMemcpyAsync(dev + L.bt_off, block_table_host, L.bt_bytes, cudaMemcpyHostToDevice, st) ==
+             cudaSuccess;
     if (!ok)
         return PKV_ERR_CUDA;
+    const WsPtrs wp{reinterpret_cast<uint32_t *>(dev + L.err_off), reinterpret_cast<uint32_t *>(dev + L.counters_off),
+                    reinterpret_cast<float *>(dev + L.m_off), reinterpret_cast<float *>(dev + L.l_off),
+                    reinterpret_cast<float *>(dev + L.acc_off)};
     rc = paged_decode_impl(dev + L.q_off, k_pool, v_pool, reinterpret_cast<const int32_t *>(dev + L.bt_off),
                            reinterpret_cast<const int32_t *>(dev + L.lens_off), s.page_size, scale, dev + L.out_off,
                            shape, &L.plan, reinterpret_cast<const pkv_work_item *>(dev + L.items_off),
-                           reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, dev, L.ws.total, st);
+                           reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, nullptr, 0, st, &wp);
     if (rc != PKV_OK)
         return rc;
-    if (cudaMemcpyAsync(out_host, dev + L.out_off, q_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaMemcpyAsync(h_err, dev, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaStreamSynchronize(st) != cudaSuccess)
+    uint8_t *h_down = hst + L.h_down_off;
+    ok = cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    if (ok && !L.out_inline)
+        ok = cudaMemcpyAsync(out_host, dev + L.out_off, L.q_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    if (!ok || cudaStreamSynchronize(st) != cudaSuccess)
         return PKV_ERR_CUDA;
-    return status_from_error_word(*h_err);
+    if (L.out_inline)
+        std::memcpy(out_host, h_down + (L.out_off - L.err_off), L.q_bytes);
+    uint32_t err;
+    std::memcpy(&err, h_down, 4);
+    return status_from_error_word(err);
 }
 
 }  // extern "C"

@@ -1,0 +1,132 @@
+"""pkv_decode_host (host buffers in, host buffer out, one packed copy each
+way) against the oracle and against pkv_paged_decode with the same plan.
+
+Both paths run the same kernels on the same plan, so their outputs must be
+bit-identical; the oracle comparison uses the tolerance of the other parity
+tests.  Covers every plan family the policy can pick (the balanced one
+included), inputs that travel inside the packed copies and inputs too large
+for them (q, block table, out above 64 KiB), and buffer reuse after a call
+that the kernels reported a device-input error on."""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_gqa_17_b200 import binding as bd
+from paged_kv_gqa_17_b200 import workloads as W
+
+from .gpu_util import assert_close, oracle_full, oracle_sampled, run, to_device
+
+pytestmark = pytest.mark.gpu
+
+ANY = (0, 2**31 - 1, 0, 2**31 - 1)
+
+
+def rule(mode, S=1, C=0, flags=0):
+    return bd.Rule(*ANY, mode, S, C, flags)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_gqa_17_b200 import build
+
+    build.build()
+    bd.lib()
+
+
+def host_inputs(w):
+    q_h = w.q.cpu().pin_memory()
+    bt_h = w.block_table.cpu().pin_memory()
+    lens_h = torch.tensor(w.seq_lens, dtype=torch.int32).pin_memory()
+    out_h = torch.full_like(q_h, float("nan")).pin_memory()
+    return q_h, bt_h, lens_h, out_h
+
+
+def host_decode(w, rules=None, dec=None):
+    q_h, bt_h, lens_h, out_h = host_inputs(w)
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table, w.layout)
+    dec = dec or bd.HostDecoder(w.q.device)
+    dec.ensure(lens_h, shape, rules)
+    plan = dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
+    return out_h.float().double().numpy(), plan
+
+
+PLANS = {
+    "nosplit": rule(0),
+    "split7": rule(1, 7),
+    "split32_deep_sep": rule(1, 32, 0, 5),
+    "wq3": rule(2, 1, 3),
+    "wq16_sep": rule(2, 1, 16, 1),
+    "bal37": rule(3, 37),
+    "bal296": rule(3, 296),
+    "split16_cl": rule(1, 16, 0, 8),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PLANS))
+def test_host_path_matches_oracle_and_device_path(name):
+    w = to_device(W.make_custom([1000, 4097, 2500, 17, 0], 32, 8, 128, seed=130, poison=True))
+    got, plan = host_decode(w, rules=[PLANS[name]])
+    assert plan.tuple()[0] == PLANS[name].mode
+    assert_close(got, oracle_full(w), f"host/{name}")
+    dev, dp = run(w, mode_rule=PLANS[name])
+    assert dp.plan.tuple() == plan.tuple()
+    assert np.array_equal(got, dev), name
+
+
+def test_host_path_default_policy_picks_balanced():
+    """B=8 with N_max in [16384, 65536): the built-in table picks the balanced
+    grid, whose queue the host path builds and uploads itself."""
+    lens = [20000, 300, 9000, 17000, 64, 5000, 12345, 1]
+    w = to_device(W.make_custom(lens, 32, 8, 128, seed=131, poison=True))
+    got, plan = host_decode(w)
+    assert plan.mode == bd.BALANCED, plan.tuple()
+    dev, dp = run(w)
+    assert dp.plan.tuple() == plan.tuple()
+    assert np.array_equal(got, dev)
+    pairs = [(0, 0), (0, 31), (3, 17), (7, 5), (4, 9), (6, 30)]
+    assert_close(np.stack([got[r, h] for r, h in pairs]), oracle_sampled(w, pairs), "host/balanced")
+
+
+@pytest.mark.parametrize("rules", [None, [rule(2, 1, 8)]])
+def test_host_path_large_inputs_use_their_own_copies(rules):
+    """B=64, H_q=64: q and out are 1 MiB and the block table 64 x 350 x 4 B,
+    all above the 64 KiB that travel inside the packed copies."""
+    rng = np.random.default_rng(11)
+    lens = [int(x) for x in rng.integers(1, 5600, 64)]
+    lens[5] = 350 * 16
+    w = W.make_custom(lens, 64, 8, 128, seed=132, poison=True, device="cuda")
+    assert w.q.numel() * 2 > 64 * 1024 and w.block_table.numel() * 4 > 64 * 1024
+    got, plan = host_decode(w, rules=rules)
+    dev, dp = run(w, rules=rules)
+    assert dp.plan.tuple() == plan.tuple()
+    assert np.array_equal(got, dev)
+    pairs = [(0, 0), (5, 63), (63, 1), (31, 40)]
+    assert_close(np.stack([got[r, h] for r, h in pairs]), oracle_sampled(w, pairs), "host/large")
+
+
+def test_host_path_reuses_buffers_after_a_device_input_error():
+    """The upload zeroes the error word and counters every call: a call that
+    the kernels flagged (page id out of range) leaves nothing behind for the
+    next call on the same buffers."""
+    w = to_device(W.make_custom([700, 1500, 33], 16, 4, 128, seed=133, poison=True))
+    ref = oracle_full(w)
+    dec = bd.HostDecoder("cuda")
+    for r in ([rule(1, 7)], [rule(2, 1, 3)], [rule(3, 11)]):
+        got, _ = host_decode(w, rules=r, dec=dec)
+        assert_close(got, ref, f"host/{r[0].mode} first")
+        q_h, bt_h, lens_h, out_h = host_inputs(w)
+        bt_h[1, 2] = w.num_pages + 9
+        shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+        with pytest.raises(bd.PkvError) as e:
+            dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=r)
+        assert e.value.status == -6  # PKV_ERR_DEVICE_INPUT
+        got, _ = host_decode(w, rules=r, dec=dec)
+        assert_close(got, ref, f"host/{r[0].mode} after error")
+
+
+def test_host_path_empty_rows():
+    w = to_device(W.make_custom([0, 0], 8, 2, 64, seed=134, poison=True))
+    got, _ = host_decode(w)
+    assert (got == 0).all()
