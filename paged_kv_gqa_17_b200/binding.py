@@ -98,7 +98,8 @@ SIGNATURES = [
 
 
 def lib(path: Optional[str] = None):
-    """Load libpkv.so (built by paged_kv_gqa_17_b200.build); raise if it is missing."""
+    """Load libpkv.so (built by paged_kv_gqa_17_b200.build); raise if it is missing.
+    With `path`, load that build instead and make it the one every later call uses."""
     global _lib
     if _lib is not None and path is None:
         return _lib
@@ -110,8 +111,7 @@ def lib(path: Optional[str] = None):
         fn = getattr(handle, name)
         fn.restype = res
         fn.argtypes = args
-    if path is None:
-        _lib = handle
+    _lib = handle
     return handle
 
 

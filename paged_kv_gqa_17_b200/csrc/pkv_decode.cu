@@ -59,8 +59,9 @@
 // Pages per block that the split kernel prefetches into L2 while it waits for
 // the kernel before it (0 turns the prefetch off).
 #ifndef PKV_L2_PREFETCH_PAGES
-#define PKV_L2_PREFETCH_PAGES 8
+#define PKV_L2_PREFETCH_PAGES 16
 #endif
+static_assert(PKV_L2_PREFETCH_PAGES >= 0 && PKV_L2_PREFETCH_PAGES <= 32, "one page per lane of the producer warp");
 
 namespace pkv {
 
@@ -1237,6 +1238,37 @@ __device__ __forceinline__ bool item_pages(const Params &p, const int4 &it, int 
     return ok;
 }
 
+// The balanced grid's counterpart of l2_prefetch_first_pages: the first
+// PKV_L2_PREFETCH_PAGES pages of this block's share, walked through its first
+// work items, all read speculatively through L2 before the dependency wait.
+template <int D>
+__device__ __forceinline__ void l2_prefetch_block_share(const Params &p, int lane)
+{
+#if PKV_L2_PREFETCH_PAGES > 0
+    const int32_t *block_ptr = p.indptr + p.B * p.H_kv + 1;
+    const int it0 = ld_l2_only(block_ptr + blockIdx.x);
+    const int it1 = ld_l2_only(block_ptr + blockIdx.x + 1);
+    if (it0 < 0 || it1 < it0 || it1 > p.n_items)
+        return;
+    int got = 0;
+    for (int it = it0; it < it1 && it < it0 + PKV_L2_PREFETCH_PAGES && got < PKV_L2_PREFETCH_PAGES; ++it) {
+        const int4 item = ld_l2_only(p.items + it);
+        int pg0, np;
+        if (!item_pages(p, item, pg0, np))
+            return;
+        const int cnt = np < PKV_L2_PREFETCH_PAGES - got ? np : PKV_L2_PREFETCH_PAGES - got;
+        if (lane >= got && lane < got + cnt) {
+            const int e = ld_l2_only(p.block_table + (int64_t)item.x * p.max_pages + pg0 + (lane - got));
+            if (e >= 0 && e < p.num_pool_pages) {
+                tma_prefetch_page_l2<D>(&p.tm_k, item.y, e);
+                tma_prefetch_page_l2<D>(&p.tm_v, item.y, e);
+            }
+        }
+        got += cnt;
+    }
+#endif
+}
+
 template <int D, int NT, int NW, int NST>
 __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_constant__ Params p)
 {
@@ -1258,17 +1290,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
     const int warp = tid >> 5;
     const int lane = tid & 31;
     constexpr int kConsumers = NW * 32;
-    grid_dependency_wait();
-
-    const int pairs = p.B * p.H_kv;
-    const int32_t *block_ptr = p.indptr + pairs + 1;
-    const int it0 = __ldg(block_ptr + blockIdx.x);
-    const int it1 = __ldg(block_ptr + blockIdx.x + 1);
-    if (it0 < 0 || it1 < it0 || it1 > p.n_items) {
-        if (tid == 0)
-            atomicOr(p.ws_error, kErrItem);
-        return;
-    }
+    // set-up that reads no global data, then the dependency wait (see split_kernel)
     if (tid == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(bar_full + 8 * s, 1);
@@ -1285,7 +1307,20 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
         prefetch_tensormap(&p.tm_k);
         prefetch_tensormap(&p.tm_v);
     }
-    __syncthreads();
+    if (warp == NW)
+        l2_prefetch_block_share<D>(p, lane);
+    grid_dependency_wait();
+
+    const int pairs = p.B * p.H_kv;
+    const int32_t *block_ptr = p.indptr + pairs + 1;
+    const int it0 = __ldg(block_ptr + blockIdx.x);
+    const int it1 = __ldg(block_ptr + blockIdx.x + 1);
+    if (it0 < 0 || it1 < it0 || it1 > p.n_items) {
+        if (tid == 0)
+            atomicOr(p.ws_error, kErrItem);
+        return;
+    }
+    __syncthreads();  // the barriers' initialisation is visible to all warps
 
     const int r = lane >> 2;
     const int c4 = lane & 3;
