@@ -427,50 +427,6 @@ struct Cfg {
     static_assert(kClusterOff + kClusterBytes <= kRingBytes, "cluster state must fit in the ring");
 };
 
-// Merge the nslots partial states of one (row, KV head) in ascending slot
-// order and write the bf16 output of its G query heads.
-template <int D>
-__device__ void merge_pair(const Params &p, int row, int h, int slot0, int nslots, int tid, int nthreads)
-{
-    const int G = p.G;
-    constexpr int D4 = D / 4;
-    for (int e = tid; e < G * D4; e += nthreads) {
-        const int g = e / D4;
-        const int d4 = (e % D4) * 4;
-        float M = -INFINITY, L = 0.f;
-        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < nslots; s0 += 8) {
-            float ms[8], ls[8];
-            float4 as[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                ms[u] = -INFINITY;
-                ls[u] = 0.f;
-                as[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (s0 + u < nslots) {
-                    const int64_t idx = (int64_t)(slot0 + s0 + u) * G + g;
-                    ms[u] = __ldcg(p.ws_m + idx);
-                    ls[u] = __ldcg(p.ws_l + idx);
-                    as[u] = __ldcg(reinterpret_cast<const float4 *>(p.ws_acc + idx * D + d4));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (ms[u] == -INFINITY)
-                    continue;  // neutral state: weight 0
-                const float Mn = fmaxf(M, ms[u]);
-                const float a = exp2_approx(M - Mn);
-                const float b = exp2_approx(ms[u] - Mn);
-                L = fmaf(L, a, ls[u] * b);
-                O = fma4(O, a, scale4(as[u], b));
-                M = Mn;
-            }
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
-    }
-}
-
 // The producer's issue rate bounds a block's bandwidth: one rank-5 TMA copy
 // per K (or V) page instead of one per 64-wide half (PKV_TMA_5D, defined
 // above), issued by several lanes at once.
@@ -648,13 +604,75 @@ __device__ __forceinline__ void merge_into(float &M, float &L, float4 &O, float 
     M = Mn;
 }
 
+// The same merge straight from L2 into registers: each thread owns (head g,
+// 4 columns) tasks and walks the slots in batches of 8, the loads of batch
+// k+1 in flight while batch k is merged (online: running max M, the sum L
+// and the accumulator O rescaled as the max grows), in ascending slot order.
+template <int D>
+__device__ void merge_pair_direct(const Params &p, int row, int h, int slot0, int nslots, int tid, int nthreads)
+{
+    constexpr int kB = 8;
+    const int G = p.G;
+    constexpr int D4 = D / 4;
+    for (int e = tid; e < G * D4; e += nthreads) {
+        const int g = e / D4;
+        const int d4 = (e % D4) * 4;
+        float M = -INFINITY, L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        float ms[2][kB], ls[2][kB];
+        float4 as[2][kB];
+        auto load = [&](int buf, int s0) {
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                ms[buf][u] = -INFINITY;
+                ls[buf][u] = 0.f;
+                as[buf][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s0 + u < nslots) {
+                    const int64_t idx = (int64_t)(slot0 + s0 + u) * G + g;
+                    ms[buf][u] = __ldcg(p.ws_m + idx);
+                    ls[buf][u] = __ldcg(p.ws_l + idx);
+                    as[buf][u] = __ldcg(reinterpret_cast<const float4 *>(p.ws_acc + idx * D + d4));
+                }
+            }
+        };
+        load(0, 0);
+        for (int s0 = 0, buf = 0; s0 < nslots; s0 += kB, buf ^= 1) {
+            if (s0 + kB < nslots) {
+                if (buf == 0)
+                    load(1, s0 + kB);
+                else
+                    load(0, s0 + kB);
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const float mu = buf == 0 ? ms[0][u] : ms[1][u];
+                const float lu = buf == 0 ? ls[0][u] : ls[1][u];
+                const float4 au = buf == 0 ? as[0][u] : as[1][u];
+                if (mu == -INFINITY)
+                    continue;  // neutral state: weight 0
+                const float Mn = fmaxf(M, mu);
+                const float a = exp2_approx(M - Mn);
+                const float b = exp2_approx(mu - Mn);
+                L = fmaf(L, a, lu * b);
+                O = fma4(O, a, scale4(au, b));
+                M = Mn;
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+    }
+}
+
 // Merge of one (row, KV head)'s n partial states by the block that finished
-// it last, staged through the idle shared-memory ring.  The weights
-// w_s = 2^(m_s - M) (M = max_s m_s, 0 for a neutral state) and the
-// denominator L = sum_s w_s l_s are computed once per head; the fp32
-// accumulators arrive in chunks by bulk async copies (double buffered), and
-// out = sum_s w_s acc_s / L is accumulated in ascending slot order.
-// Returns false when the ring cannot hold the weights plus two slots.
+// it last, staged through the idle shared-memory ring.  The fp32
+// accumulators arrive by bulk async copies, in chunks of hs slots: all of
+// them in two chunks on the two merge barriers when the ring holds them,
+// else double buffered.  While they land, the block loads the (m, l) pairs
+// into shared memory.  Each thread then owns (head g, 4 columns) tasks and
+// does the whole merge for them on its own, with no further block-wide
+// step: M = max_s m_s, and in ascending slot order w_s = 2^(m_s - M) (0 for
+// a neutral state), L += w_s l_s, O += w_s acc_s; out = O / L.
+// Returns false when the ring cannot hold the (m, l) pairs plus two slots.
 template <int D, int NT, int NW, int NST>
 __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0, int row, int h, int slot0, int n,
                                   int tid, uint32_t (&uses)[2])
@@ -663,61 +681,48 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
     const int G = p.G;
     constexpr int D4 = D / 4;
     const int slot_bytes = G * D * 4;
-    const int wbytes = ((2 * n * G + 32) * 4 + 1023) / 1024 * 1024;
-    const int half = (C::kRingBytes - wbytes) / 2 / 1024 * 1024;
-    const int hs = half > 0 ? half / slot_bytes : 0;  // slots per buffer
-    if (hs < 1)
+    const int mlbytes = (2 * n * G * 4 + 1023) / 1024 * 1024;
+    const int cap = (C::kRingBytes - mlbytes) / slot_bytes;  // slots the ring holds besides (m, l)
+    if (cap < 2)
         return false;
-    float *w_s = reinterpret_cast<float *>(smem);  // [n][G]: m, then the weights
-    float *l_s = w_s + n * G;                      // [n][G]
-    float *ML = l_s + n * G;                       // M[16], L[16]
-    const uint32_t stage0 = smem_addr(smem) + wbytes;
+    const int hs = (n + 1) / 2 < cap / 2 ? (n + 1) / 2 : cap / 2;  // slots per chunk (and per buffer)
     const int nch = (n + hs - 1) / hs;
+    float *m_s = reinterpret_cast<float *>(smem);  // [n][G]
+    float *l_s = m_s + n * G;                      // [n][G]
+    const uint32_t stage0 = smem_addr(smem) + mlbytes;
+    const int buf_bytes = hs * slot_bytes;
     if (tid == 0) {
+        fence_proxy_async_smem();    // earlier generic accesses to the ring precede the copies
         fence_proxy_async_global();  // the states were written by other blocks' generic stores
         for (int ch = 0; ch < 2 && ch < nch; ++ch) {
             const int cnt = min(hs, n - ch * hs);
             mbar_expect_tx(mbar0 + 8 * ch, cnt * slot_bytes);
-            bulk_g2s(stage0 + ch * half, p.ws_acc + (int64_t)(slot0 + ch * hs) * G * D, cnt * slot_bytes,
+            bulk_g2s(stage0 + ch * buf_bytes, p.ws_acc + (int64_t)(slot0 + ch * hs) * G * D, cnt * slot_bytes,
                      mbar0 + 8 * ch);
         }
     }
     for (int i = tid; i < n * G; i += C::kThreads) {
-        w_s[i] = __ldcg(p.ws_m + (int64_t)slot0 * G + i);
+        m_s[i] = __ldcg(p.ws_m + (int64_t)slot0 * G + i);
         l_s[i] = __ldcg(p.ws_l + (int64_t)slot0 * G + i);
     }
     __syncthreads();
-    // One warp per head: M = max_s m_s, the weights, and L = sum_s w_s l_s,
-    // each reduced over the lanes by a fixed xor-shuffle tree.
-    const int lane = tid & 31;
-    for (int g = tid >> 5; g < G; g += C::kThreads / 32) {
-        float M = -INFINITY;
-        for (int s = lane; s < n; s += 32)
-            M = fmaxf(M, w_s[s * G + g]);
-#pragma unroll
-        for (int sh = 16; sh > 0; sh >>= 1)
-            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
-        float L = 0.f;
-        for (int s = lane; s < n; s += 32) {
-            const float m = w_s[s * G + g];
-            const float wgt = m == -INFINITY ? 0.f : exp2_approx(m - M);
-            w_s[s * G + g] = wgt;
-            L = fmaf(wgt, l_s[s * G + g], L);
-        }
-#pragma unroll
-        for (int sh = 16; sh > 0; sh >>= 1)
-            L += __shfl_xor_sync(0xffffffffu, L, sh);
-        if (lane == 0)
-            ML[16 + g] = L;
-    }
-    __syncthreads();
+    float M[C::kMaxMergeTasks], L[C::kMaxMergeTasks];
     float4 O[C::kMaxMergeTasks];
 #pragma unroll
-    for (int k = 0; k < C::kMaxMergeTasks; ++k)
+    for (int k = 0; k < C::kMaxMergeTasks; ++k) {
+        const int e = tid + k * C::kThreads;
+        M[k] = -INFINITY;
+        L[k] = 0.f;
         O[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < G * D4) {
+            const int g = e / D4;
+            for (int s = 0; s < n; ++s)
+                M[k] = fmaxf(M[k], m_s[s * G + g]);
+        }
+    }
     for (int ch = 0; ch < nch; ++ch) {
         mbar_wait(mbar0 + 8 * (ch & 1), (uses[ch & 1] + (ch >> 1)) & 1, p.ws_error);
-        const float *st = reinterpret_cast<const float *>(smem + wbytes + (ch & 1) * half);
+        const float *st = reinterpret_cast<const float *>(smem + mlbytes + (ch & 1) * buf_bytes);
         const int first = ch * hs;
         const int cnt = min(hs, n - first);
 #pragma unroll
@@ -729,25 +734,34 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
                 float4 O2 = make_float4(0.f, 0.f, 0.f, 0.f);  // second chain for ILP
                 int s = 0;
                 for (; s + 1 < cnt; s += 2) {
-                    O[k] = fma4(*reinterpret_cast<const float4 *>(st + (s * G + g) * D + d4),
-                                w_s[(first + s) * G + g], O[k]);
-                    O2 = fma4(*reinterpret_cast<const float4 *>(st + ((s + 1) * G + g) * D + d4),
-                              w_s[(first + s + 1) * G + g], O2);
+                    const float ma = m_s[(first + s) * G + g];
+                    const float mb = m_s[(first + s + 1) * G + g];
+                    const float wa = ma == -INFINITY ? 0.f : exp2_approx(ma - M[k]);
+                    const float wb = mb == -INFINITY ? 0.f : exp2_approx(mb - M[k]);
+                    L[k] = fmaf(wa, l_s[(first + s) * G + g], L[k]);
+                    L[k] = fmaf(wb, l_s[(first + s + 1) * G + g], L[k]);
+                    O[k] = fma4(*reinterpret_cast<const float4 *>(st + (s * G + g) * D + d4), wa, O[k]);
+                    O2 = fma4(*reinterpret_cast<const float4 *>(st + ((s + 1) * G + g) * D + d4), wb, O2);
                 }
-                if (s < cnt)
-                    O[k] = fma4(*reinterpret_cast<const float4 *>(st + (s * G + g) * D + d4), w_s[(first + s) * G + g],
-                                O[k]);
+                if (s < cnt) {
+                    const float ma = m_s[(first + s) * G + g];
+                    const float wa = ma == -INFINITY ? 0.f : exp2_approx(ma - M[k]);
+                    L[k] = fmaf(wa, l_s[(first + s) * G + g], L[k]);
+                    O[k] = fma4(*reinterpret_cast<const float4 *>(st + (s * G + g) * D + d4), wa, O[k]);
+                }
                 O[k] = make_float4(O[k].x + O2.x, O[k].y + O2.y, O[k].z + O2.z, O[k].w + O2.w);
             }
         }
-        __syncthreads();
-        if (tid == 0 && ch + 2 < nch) {
-            fence_proxy_async_smem();  // our reads of this buffer precede its refill
-            const int c2 = ch + 2;
-            const int cnt2 = min(hs, n - c2 * hs);
-            mbar_expect_tx(mbar0 + 8 * (c2 & 1), cnt2 * slot_bytes);
-            bulk_g2s(stage0 + (c2 & 1) * half, p.ws_acc + (int64_t)(slot0 + c2 * hs) * G * D, cnt2 * slot_bytes,
-                     mbar0 + 8 * (c2 & 1));
+        if (ch + 2 < nch) {
+            __syncthreads();  // every thread is done with this buffer
+            if (tid == 0) {
+                fence_proxy_async_smem();  // our reads of this buffer precede its refill
+                const int c2 = ch + 2;
+                const int cnt2 = min(hs, n - c2 * hs);
+                mbar_expect_tx(mbar0 + 8 * (c2 & 1), cnt2 * slot_bytes);
+                bulk_g2s(stage0 + (c2 & 1) * buf_bytes, p.ws_acc + (int64_t)(slot0 + c2 * hs) * G * D,
+                         cnt2 * slot_bytes, mbar0 + 8 * (c2 & 1));
+            }
         }
     }
 #pragma unroll
@@ -756,14 +770,31 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
         if (e < G * D4) {
             const int g = e / D4;
             const int d4 = (e % D4) * 4;
-            const float L = ML[16 + g];
-            const float inv = L > 0.f ? 1.f / L : 0.f;
+            const float inv = L[k] > 0.f ? 1.f / L[k] : 0.f;
             store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O[k], inv));
         }
     }
     uses[0] += (nch + 1) / 2;  // barrier 0 carried the even chunks, barrier 1 the odd ones
     uses[1] += nch / 2;
+    __syncthreads();  // the ring is free again once every thread has left it
     return true;
+}
+
+// The last block's merge of a pair: up to kDirectMergeSlots states straight
+// into registers (one batch of L2 loads in flight per thread, or two), more
+// through the ring, whose bulk copies keep all of them in flight at once.
+// Both were timed on B200 with the step's own blocks as the merging blocks:
+// the direct path wins at 8-12 states (by about 1-2 us per step), the
+// staged one at 32.
+constexpr int kDirectMergeSlots = 16;
+
+template <int D, int NT, int NW, int NST>
+__device__ void merge_pair_last_block(const Params &p, uint8_t *smem, uint32_t mbar0, int row, int h, int slot0,
+                                      int n, int tid, uint32_t (&uses)[2])
+{
+    using C = Cfg<D, NT, NW, NST>;
+    if (n <= kDirectMergeSlots || !merge_pair_staged<D, NT, NW, NST>(p, smem, mbar0, row, h, slot0, n, tid, uses))
+        merge_pair_direct<D>(p, row, h, slot0, n, tid, C::kThreads);
 }
 
 // Before its dependency wait the split kernel may read nothing that the
@@ -1191,9 +1222,8 @@ __global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_const
         __syncthreads();
         if (misc[0]) {
             uint32_t uses[2] = {0, 0};
-            if (!merge_pair_staged<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid,
-                                                   uses))
-                merge_pair<D>(p, row, h, slot0, nslots, tid, C::kThreads);
+            merge_pair_last_block<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid,
+                                                  uses);
             if (tid == 0)
                 p.ws_counters[pair] = 0u;  // ready for the next call
             PKV_TRACE_POINT(5);
@@ -1484,7 +1514,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
                 }
                 named_barrier(1, kConsumers);
                 if (misc[1]) {
-                    merge_pair<D>(p, row, h, slot0, nslots, tid, kConsumers);
+                    merge_pair_direct<D>(p, row, h, slot0, nslots, tid, kConsumers);
                     named_barrier(1, kConsumers);
                     if (tid == 0) {
                         p.ws_counters[pair] = 0u;
@@ -1503,8 +1533,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
     uint32_t uses[2] = {0, 0};
     for (int k = 0; k < nd; ++k) {
         const int4 d = deferred[k];
-        if (!merge_pair_staged<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, d.x, d.y, d.z, d.w, tid, uses))
-            merge_pair<D>(p, d.x, d.y, d.z, d.w, tid, C::kThreads);
+        merge_pair_last_block<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, d.x, d.y, d.z, d.w, tid, uses);
         __syncthreads();
         if (tid == 0)
             p.ws_counters[d.x * p.H_kv + d.y] = 0u;  // ready for the next call
