@@ -13,9 +13,11 @@ Metric: KV GB/s = (K+V bytes of the valid tokens + q + out) / step time, and
 its fraction of the measured HBM copy bandwidth; also us/step.
   value  steady-state device time: K steps queued back to back on one
          stream between one pair of CUDA events, inputs resident in HBM.
-         Consecutive steps read different copies of the KV pool (enough
-         copies that three L2 sizes of data lie between two reads of the
-         same copy), so no step finds its pages in L2.
+         The K steps are captured once in a CUDA graph and replayed (as a
+         serving loop replays its decode step; --no-graph queues them from
+         Python instead).  Consecutive steps read different copies of the KV
+         pool (enough copies that three L2 sizes of data lie between two
+         reads of the same copy), so no step finds its pages in L2.
   latency_us  one isolated step, cold: L2 flushed (a 256 MiB write, then a
          256 MiB read so no dirty lines are left) before each step, CUDA
          events around the step alone.
@@ -63,6 +65,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines in 'all_workloads'")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=8.0, help="target CPU time of the cpu_baseline sample")
+    ap.add_argument("--no-graph", action="store_true", help="queue the timed steps from Python, not a CUDA graph")
     return ap.parse_args(argv)
 
 
@@ -330,7 +333,7 @@ def run_ours(args):
     barrier(dist, device)
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
-        steady_ms = time_steady(w, dp, args.steps, args.warmup, torch, bd, copies)
+        steady_ms = time_steady(w, dp, args.steps, args.warmup, torch, bd, copies, graph=not args.no_graph)
     torch.cuda.synchronize()
     barrier(dist, device)
     n_copies = len(copies)
@@ -344,7 +347,8 @@ def run_ours(args):
     early_plan = bd.Plan(dp.plan.mode, dp.plan.num_splits, dp.plan.chunk_pages, dp.plan.flags | bd.FLAG_PDL_EARLY)
     dp_early = bd.plan_decode(w.seq_lens, shape, device, plan=early_plan)
     copies = pool_copies(w, torch)
-    early_ms = time_steady(w, dp_early, args.steps, args.warmup, torch, bd, copies) / args.steps
+    early_ms = time_steady(w, dp_early, args.steps, args.warmup, torch, bd, copies,
+                           graph=not args.no_graph) / args.steps
     del copies, dp_early
     e2e_ms, h2d, d2h, _ = time_e2e(w, args.e2e_steps or args.steps, min(args.warmup, 3), torch, bd, flush)
     e2e_total = max_over_ranks(sum(e2e_ms), dist, device)
@@ -379,6 +383,8 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded bf16 N(0,1) q/K/V, random page placement)",
         "config": dict(_describe(w, dp.plan), parallelism=f"replicas x{world} (one workload per GPU)",
+                       timed_steps="one CUDA graph of the K steps, replayed" if not args.no_graph
+                       else "K steps queued from Python",
                        l2=f"inputs larger than L2: back-to-back steps rotate over {n_copies} copies of the KV pool "
                           f"({n_copies * w.kv_bytes() / 2**20:.0f} MiB of step data); latency_us is flushed per step"),
         "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4),

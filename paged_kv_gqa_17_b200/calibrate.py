@@ -12,9 +12,10 @@ on a holdout seed].  This script does the same by measurement:
      log-uniform between an eighth of it and it (H_q=32, H_kv=8, D=128,
      16-token pages).
   2. It times every candidate plan (no-split; split-S over several S with
-     and without the deep ring; the work queue over several chunk sizes; the
-     balanced grid at one and two blocks per SM) as the steady-state device
-     time of back-to-back steps over rotating pool copies.
+     and without the deep ring, and with the cluster merge at S = 8 and 16;
+     the work queue over several chunk sizes; the balanced grid at one and
+     two blocks per SM) as the steady-state device time of back-to-back
+     steps over rotating pool copies.
   3. The fastest plan of each cell becomes a rule; neighbouring cells of one B
      with the same plan are merged.
   4. Every cell is re-measured with the holdout seed 20260623; the report
@@ -48,6 +49,8 @@ def candidates():
     out = [(0, 1, 0, 0)]
     for S in (8, 16, 32, 37, 64):
         out += [(1, S, 0, 0), (1, S, 0, 4)]
+    for S in (8, 16):
+        out.append((1, S, 0, 12))  # cluster merge, deep ring
     for C in (8, 16, 32, 64):
         out.append((2, 1, C, 0))
     out += [(3, 296, 0, 0), (3, 148, 0, 4)]

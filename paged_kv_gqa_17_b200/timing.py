@@ -3,7 +3,10 @@
 Two protocols:
   time_steady    K steps queued back to back between one pair of events,
                  consecutive steps reading different copies of the KV pool
-                 (pool_copies) so that no step finds its pages in L2;
+                 (pool_copies) so that no step finds its pages in L2.  The K
+                 steps are captured once in a CUDA graph and replayed, as a
+                 serving loop replays its decode step, so that the host's
+                 launch rate never paces the device;
   time_isolated  single cold steps, L2 flushed (Flush) before each, events
                  around the step alone.
 """
@@ -33,8 +36,9 @@ def pool_copies(w, torch, l2_bytes=126 << 20):
     return [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone()) for _ in range(n - 1)]
 
 
-def time_steady(w, dp, K, W, torch, bd, copies):
-    """Device time (ms) of K back-to-back steps, one event pair, rotating pool copies."""
+def time_steady(w, dp, K, W, torch, bd, copies, graph=True):
+    """Device time (ms) of K back-to-back steps, one event pair, rotating pool
+    copies; the steps are replayed from a CUDA graph unless graph=False."""
     lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=w.q.device)
     out = torch.empty_like(w.q)
 
@@ -45,14 +49,26 @@ def time_steady(w, dp, K, W, torch, bd, copies):
     for i in range(W):
         step(i)
     torch.cuda.synchronize()
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(K):
+                step(W + i)
+        g.replay()  # untimed: the first replay also uploads the graph
+        torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(st)
-    for i in range(K):
-        step(W + i)
+    if graph:
+        g.replay()
+    else:
+        for i in range(K):
+            step(W + i)
     b.record(st)
     torch.cuda.synchronize()
+    del g
     if bd.workspace_status(dp) != 0:
         raise RuntimeError("device error during the timed steps")
     return a.elapsed_time(b)
