@@ -58,7 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="long", choices=["tiny", "long", "crossover", "mixed", "prefix"])
+    ap.add_argument("--workload", default="long",
+                    choices=["tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=None)
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end timing (default: --steps)")
@@ -235,7 +236,7 @@ class ClockSampler:
 # the GPU arm
 
 def _describe(w, plan):
-    names = {0: "NO_SPLIT", 1: "SPLIT_S", 2: "WORK_QUEUE"}
+    names = {0: "NO_SPLIT", 1: "SPLIT_S", 2: "WORK_QUEUE", 3: "BALANCED"}
     lens = w.seq_lens
     return {
         "workload": f"{w.name}: B={w.B} H_q={w.H_q} H_kv={w.H_kv} D={w.D} P={w.P} "

@@ -1,0 +1,50 @@
+"""Host-side pieces of bench.py, without a GPU: the JSON description of
+every plan family, the argument parser, and the reference arm's JSON line
+(the oracle on the tiny workload)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from paged_kv_gqa_17_b200 import workloads as W  # noqa: E402
+
+
+class _Plan:
+    def __init__(self, mode, S, C, flags):
+        self.mode, self.num_splits, self.chunk_pages, self.flags = mode, S, C, flags
+
+
+@pytest.mark.parametrize("mode,name", [(0, "NO_SPLIT"), (1, "SPLIT_S"), (2, "WORK_QUEUE"), (3, "BALANCED")])
+def test_describe_names_every_plan_family(mode, name):
+    w = W.make("tiny")
+    d = bench._describe(w, _Plan(mode, 4, 2, 0))
+    assert d["plan"]["mode"] == name
+    assert d["batch"] == 1 and d["tokens"] == 512
+    json.dumps(d)
+
+
+def test_parser_accepts_every_named_workload():
+    for name in ("tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf"):
+        assert bench.parse_args(["--workload", name]).workload == name
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.workload == "long" and not a.no_graph
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "impl"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["unit"] == d["unit"]
