@@ -1,6 +1,6 @@
 """Calibrate the built-in policy table on the GPU from measured timings.
 
-    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--steps 30]
+    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--steps 100]
 
 The policy maps (batch size B, longest row N_max) to an execution plan
 [PersistentKV explainer, Technical summary > Methodology > 2 "Calibrated
@@ -110,7 +110,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--out", default=os.path.join(HERE, "policy_b200.json"))
     ap.add_argument("--report", default=os.path.join(ROOT, "profiles", "policy_calibration_b200.md"))
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     args = ap.parse_args(argv)
 
     import torch
