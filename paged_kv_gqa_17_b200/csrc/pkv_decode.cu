@@ -936,8 +936,14 @@ __device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lan
 }
 
 // One block = one work item (row, KV head, token range) for all G query heads.
+// The deep-ring variants (two blocks per SM at most, by shared memory) tell
+// the compiler so.  With that hint the D = 128, G <= 8 variants come out at
+// 128 registers, which still lets the 8-stage ones run three blocks per SM,
+// and they measured faster on B200 than the unhinted allocation (115
+// registers) at every timed configuration (long context, crossover, mixed,
+// many-wave queues).
 template <int D, int NT, int NW, int NST, bool CL>
-__global__ void __launch_bounds__((NW + 1) * 32) split_kernel(const __grid_constant__ Params p)
+__global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kernel(const __grid_constant__ Params p)
 {
     using C = Cfg<D, NT, NW, NST>;
     extern __shared__ uint8_t smem_raw[];
