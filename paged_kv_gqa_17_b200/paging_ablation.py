@@ -15,7 +15,8 @@ contiguous ("slab") cache.  This script measures it for this library:
   - NHD: the permuted workload with the pool laid out [pages][16][H_kv][D]
     instead of [pages][H_kv][16][D].
 
-Same plan (the built-in policy's) for all three; steady-state µs per step.
+Same plan (the built-in policy's) for all three; steady-state µs per step
+(back-to-back steps replayed from a CUDA graph, rotating pool copies).
 """
 from __future__ import annotations
 
@@ -64,7 +65,7 @@ def main(argv=None):
     dev = torch.device("cuda")
     lines = ["# Paging-overhead ablation (B200)", "",
              "Command: `python -m paged_kv_gqa_17_b200.paging_ablation`. Same values, same plan (built-in policy); "
-             "steady-state µs per step over rotating pool copies.", "",
+             "steady-state µs per step (CUDA-graph replay of back-to-back steps over rotating pool copies).", "",
              "| workload | plan | permuted HND | identity HND | permuted NHD | identity / permuted |",
              "|---|---|---|---|---|---|"]
     for name in ("long", "crossover", "mixed"):
@@ -78,26 +79,9 @@ def main(argv=None):
             vshape = bd.shape_of(v.q, v.k_pool, v.block_table, v.layout)
             dp = bd.plan_decode(v.seq_lens, vshape, dev, plan=plan)
             copies = T.pool_copies(v, torch)
-            lens = torch.tensor(v.seq_lens, dtype=torch.int32, device=dev)
-            out = torch.empty_like(v.q)
-
-            def step(i, v=v, dp=dp, copies=copies, lens=lens, out=out):
-                k, vv = copies[i % len(copies)]
-                bd.paged_decode(v.q, k, vv, v.block_table, lens, v.P, v.scale, plan=dp, out=out, layout=v.layout)
-
-            for i in range(5):
-                step(i)
-            torch.cuda.synchronize()
-            st = torch.cuda.current_stream()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(st)
-            for i in range(args.steps):
-                step(i)
-            b.record(st)
-            torch.cuda.synchronize()
-            res[label] = a.elapsed_time(b) / args.steps * 1e3
-            print(name, label, f"{res[label]:.2f} us", flush=True)
+            res[label] = T.time_steady(v, dp, args.steps, 5, torch, bd, copies) / args.steps * 1e3
             del copies
+            print(name, label, f"{res[label]:.2f} us", flush=True)
         lines.append(f"| {name} | {plan.tuple()} | {res['permuted HND']:.2f} | {res['identity HND']:.2f} | "
                      f"{res['permuted NHD']:.2f} | {res['identity HND'] / res['permuted HND']:.3f} |")
         torch.cuda.empty_cache()
