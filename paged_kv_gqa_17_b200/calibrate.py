@@ -13,8 +13,8 @@ on a holdout seed].  This script does the same by measurement:
      16-token pages).
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
-     the work queue over several chunk sizes; the balanced grid at one and
-     two blocks per SM) as the steady-state device time of back-to-back
+     the work queue over seven chunk sizes, with and without the deep ring;
+     the balanced grid at one and two blocks per SM) as the steady-state device time of back-to-back
      steps over rotating pool copies.
   3. The fastest plan of each cell becomes a rule; neighbouring cells of one B
      with the same plan are merged.
@@ -51,8 +51,8 @@ def candidates():
         out += [(1, S, 0, 0), (1, S, 0, 4)]
     for S in (8, 16):
         out.append((1, S, 0, 12))  # cluster merge, deep ring
-    for C in (8, 16, 32, 64):
-        out.append((2, 1, C, 0))
+    for C in (8, 16, 24, 32, 48, 64, 96):
+        out += [(2, 1, C, 0), (2, 1, C, 4)]
     out += [(3, 296, 0, 0), (3, 148, 0, 4)]
     return out
 
