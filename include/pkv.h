@@ -135,8 +135,12 @@ typedef struct {
     int32_t b_lo, b_hi;
     int32_t nmax_lo, nmax_hi;
     int32_t mode;         /* pkv_mode */
-    int32_t num_splits;   /* SPLIT_S: requested S >= 1; BALANCED: blocks T >= 1 */
-    int32_t chunk_pages;  /* WORK_QUEUE: chunk size C >= 1 in pages */
+    int32_t num_splits;   /* SPLIT_S: requested S >= 1; BALANCED: blocks T >= 1;
+                             WORK_QUEUE with chunk_pages = 0: the item budget T >= 1 */
+    int32_t chunk_pages;  /* WORK_QUEUE: chunk size C >= 1 in pages, or 0: the smallest C
+                             whose queue has at most T = num_splits items (one wave of T
+                             blocks), or ceil(N_max / P) when one item per (row, KV head)
+                             already exceeds T */
     int32_t flags;        /* PKV_FLAG_* */
 } pkv_policy_rule;
 

@@ -298,7 +298,7 @@ class Rule:
     flags: int = 0
 
 
-def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tuple[int, int, int, int]:
+def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule], H_kv: int = 1) -> Tuple[int, int, int, int]:
     """Pick the execution path from (B, N_max) [PKV, Methodology 2 "Calibrated adaptive policy"].
 
     The first rule whose ranges hold (B, N_max) decides; no match, an empty
@@ -306,7 +306,9 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tup
     (mode, num_splits, chunk_pages, flags):
       NO_SPLIT    -> (0, 1, 0, flags)
       SPLIT_S     -> C = ceil(pages_max / S), S' = ceil(pages_max / C): (1, S', C, flags)
-      WORK_QUEUE  -> C from the rule,      S' = ceil(pages_max / C): (2, S', C, flags)
+      WORK_QUEUE  -> C from the rule,      S' = ceil(pages_max / C): (2, S', C, flags);
+                     a rule with chunk_pages = 0 asks for the smallest C whose
+                     queue has at most T = num_splits items (pages_max if none)
       BALANCED    -> T blocks from the rule's num_splits:              (3, T, 0, flags)
     where pages_max = ceil(N_max / P).
     """
@@ -324,8 +326,8 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tup
             raise ValueError("unknown mode in policy table")
         if r.mode in (SPLIT_S, BALANCED) and r.num_splits < 1:
             raise ValueError("SPLIT_S and BALANCED rules need num_splits >= 1")
-        if r.mode == WORK_QUEUE and r.chunk_pages < 1:
-            raise ValueError("WORK_QUEUE rule needs chunk_pages >= 1")
+        if r.mode == WORK_QUEUE and (r.chunk_pages < 0 or (r.chunk_pages == 0 and r.num_splits < 1)):
+            raise ValueError("WORK_QUEUE rule needs chunk_pages >= 1, or 0 with num_splits >= 1")
         if chosen is None and r.b_lo <= B < r.b_hi and r.nmax_lo <= n_max < r.nmax_hi:
             chosen = r
     if chosen is None or B == 0 or pages_max == 0:
@@ -336,9 +338,22 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule]) -> Tup
         return (BALANCED, chosen.num_splits, 0, chosen.flags)
     if chosen.mode == SPLIT_S:
         C = _ceil_div(pages_max, chosen.num_splits)
-    else:
+    elif chosen.chunk_pages > 0:
         C = chosen.chunk_pages
+    else:
+        # the first chunk size, counting up, whose queue fits T items
+        C = pages_max
+        for c in range(1, pages_max + 1):
+            if fill_items(lens, H_kv, P, c) <= chosen.num_splits:
+                C = c
+                break
     return (chosen.mode, _ceil_div(pages_max, C), C, chosen.flags)
+
+
+def fill_items(seq_lens: Sequence[int], H_kv: int, P: int, C: int) -> int:
+    """Items of the compact queue at chunk size C (one per non-empty chunk of
+    each (row, KV head), one empty item for a row with N_i = 0)."""
+    return H_kv * sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)
 
 
 def load_rules(path: str) -> List[Rule]:

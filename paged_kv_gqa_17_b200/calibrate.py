@@ -13,8 +13,9 @@ on a holdout seed].  This script does the same by measurement:
      16-token pages).
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
-     the work queue over seven chunk sizes, with and without the deep ring;
-     the balanced grid at one and two blocks per SM) as the steady-state device time of back-to-back
+     the work queue over seven chunk sizes, with and without the deep ring,
+     and with the chunk size that fills one wave of 296 or 444 blocks; the
+     balanced grid at one and two blocks per SM) as the steady-state device time of back-to-back
      steps over rotating pool copies.
   3. The fastest plan of each cell becomes a rule; neighbouring cells of one B
      with the same plan are merged.
@@ -53,6 +54,7 @@ def candidates():
         out.append((1, S, 0, 12))  # cluster merge, deep ring
     for C in (8, 16, 24, 32, 48, 64, 96):
         out += [(2, 1, C, 0), (2, 1, C, 4)]
+    out += [(2, 296, 0, 4), (2, 296, 0, 0), (2, 444, 0, 0)]  # C chosen to fill one wave of T blocks
     out += [(3, 296, 0, 0), (3, 148, 0, 4)]
     return out
 
@@ -98,7 +100,11 @@ def build_rules(best):
             if mode in (1, 3):
                 r["num_splits"] = S
             if mode == 2:
-                r["chunk_pages"] = C
+                if C > 0:
+                    r["chunk_pages"] = C
+                else:
+                    r["num_splits"] = S  # the item budget of the fill rule
+                    r["chunk_pages"] = 0
             if flags:
                 r["flags"] = flags
             rules.append(r)

@@ -57,10 +57,38 @@ int check_rules(const pkv_policy_rule *rules, int32_t n)
             return PKV_ERR_INVALID;
         if ((r.mode == PKV_SPLIT_S || r.mode == PKV_BALANCED) && r.num_splits < 1)
             return PKV_ERR_INVALID;
-        if (r.mode == PKV_WORK_QUEUE && r.chunk_pages < 1)
+        if (r.mode == PKV_WORK_QUEUE && (r.chunk_pages < 0 || (r.chunk_pages == 0 && r.num_splits < 1)))
             return PKV_ERR_INVALID;
     }
     return PKV_OK;
+}
+
+// Items of the compact queue at chunk size C: H_kv * sum_i max(1, ceil(pages_i / C)).
+int64_t queue_items(const int32_t *lens, int32_t B, int32_t H_kv, int32_t P, int64_t C)
+{
+    int64_t n = 0;
+    for (int32_t i = 0; i < B; ++i)
+        n += std::max<int64_t>(1, ceil_div(ceil_div(lens[i], P), C));
+    return n * H_kv;
+}
+
+// The smallest chunk size whose queue has at most T items (the queue fills
+// one wave of T blocks with as little work per block as possible); the
+// whole row (pages_max) when even one item per (row, KV head) exceeds T.
+// The item count only falls as C grows, so a bisection finds it.
+int64_t fill_chunk(const int32_t *lens, const pkv_shape &s, int64_t pages_max, int64_t T)
+{
+    if (queue_items(lens, s.B, s.H_kv, s.page_size, pages_max) > T)
+        return pages_max;
+    int64_t lo = 1, hi = pages_max;  // items(hi) <= T
+    while (lo < hi) {
+        const int64_t mid = lo + (hi - lo) / 2;
+        if (queue_items(lens, s.B, s.H_kv, s.page_size, mid) <= T)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    return lo;
 }
 
 }  // namespace
@@ -137,7 +165,8 @@ int pkv_select_policy(const int32_t *seq_lens_host, const pkv_shape *shape,
         return PKV_OK;
     }
     const int64_t C = chosen->mode == PKV_SPLIT_S ? ceil_div(pages_max, chosen->num_splits)
-                                                  : (int64_t)chosen->chunk_pages;
+                      : chosen->chunk_pages > 0 ? (int64_t)chosen->chunk_pages
+                                                : fill_chunk(seq_lens_host, *shape, pages_max, chosen->num_splits);
     *plan = {chosen->mode, (int32_t)ceil_div(pages_max, C), (int32_t)C, chosen->flags};
     return PKV_OK;
 }

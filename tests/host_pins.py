@@ -9,6 +9,8 @@ real oracle and against copies with a planted mistake.
   queue_bruteforce    enumerate-and-filter over a rectangular (i, h, c) grid
   policy_paper        the page's decisions at B = 1 / 4 / 8 (tests/golden/paper_policy.txt)
   policy_semantics    first match wins, ranges are half-open, S' and C closed forms
+  policy_fill         a queue rule with chunk_pages = 0 takes the smallest C whose
+                      queue (counted by building it) has at most T items
   launch_fanout       16 bucket launches vs 2 queue launches at B = 8
                       (tests/golden/launch_fanout_b8.txt)
   merge_state_closed  queue merge traffic = 2*G*(D+2)*4 * H_kv * (slots of
@@ -136,7 +138,8 @@ def policy_semantics(O):
     assert O.select_policy([], P, rules) == (O.NO_SPLIT, 1, 0, 0)
     assert O.select_policy([0, 0], P, rules) == (O.NO_SPLIT, 1, 0, 0)
     for bad in ([R(0, 9, 0, 9, 7)], [R(0, 9, 0, 9, O.SPLIT_S, num_splits=0)],
-                [R(0, 9, 0, 9, O.WORK_QUEUE, chunk_pages=0)], [R(0, 9, 0, 9, 3, num_splits=0)]):
+                [R(0, 9, 0, 9, O.WORK_QUEUE, chunk_pages=-1)],
+                [R(0, 9, 0, 9, O.WORK_QUEUE, num_splits=0, chunk_pages=0)], [R(0, 9, 0, 9, 3, num_splits=0)]):
         try:
             O.select_policy([5], P, bad)
         except ValueError:
@@ -264,7 +267,41 @@ def balanced_bruteforce(O):
         assert got_owner == want_owner, ("balanced_bruteforce owners", lens, T)
 
 
-HOST_PINS = (queue_closed_form, queue_cover, queue_bruteforce, policy_paper, policy_semantics,
+def policy_fill(O):
+    """The fill rule by its definition: the queue at the chosen C (built, not
+    counted by formula) has at most T items, and at C - 1 it has more; when
+    even whole rows exceed T, C is the longest row's page count."""
+    R = O.Rule
+    rng = random.Random(17)
+    P = 16
+    for _ in range(60):
+        B = rng.randint(1, 9)
+        lens = [rng.choice([0, rng.randint(1, 50), rng.randint(1, 900), rng.randint(1, 6000)]) for _ in range(B)]
+        H_kv = rng.choice([1, 2, 4, 8])
+        T = rng.choice([1, 7, 37, 148, 296])
+        pages_max = max(_cdiv(n, P) for n in lens)
+        mode, S, C, flags = O.select_policy(lens, P, [R(0, O.INT32_MAX, 0, O.INT32_MAX, O.WORK_QUEUE,
+                                                       num_splits=T, chunk_pages=0, flags=4)], H_kv)
+        if pages_max == 0:
+            assert mode == O.NO_SPLIT, ("policy_fill empty", lens)
+            continue
+        assert mode == O.WORK_QUEUE and flags == 4 and 1 <= C <= pages_max, ("policy_fill", lens, T, C)
+        assert S == _cdiv(pages_max, C), ("policy_fill S'", lens, T, C, S)
+        n_at = len(O.build_work_queue(lens, H_kv, P, C)[0])
+        if n_at > T:
+            assert C == pages_max, ("policy_fill: queue too long", lens, H_kv, T, C, n_at)
+            assert len(O.build_work_queue(lens, H_kv, P, pages_max)[0]) == B * H_kv
+        elif C > 1:
+            assert len(O.build_work_queue(lens, H_kv, P, C - 1)[0]) > T, ("policy_fill: not smallest", lens, T, C)
+    # worked case: B=8 mixed-like rows, 8 heads, one wave of 296 blocks
+    lens = [12129, 621, 1118, 1452, 2891, 1419, 518, 3174]
+    plan = O.select_policy(lens, P, [R(0, O.INT32_MAX, 0, O.INT32_MAX, O.WORK_QUEUE, num_splits=296)], 8)
+    # pages per row 759, 39, 70, 91, 181, 89, 33, 199.  C = 45: chunks 17+1+2+3+5+2+1+5 = 36 per head,
+    # 8 * 36 = 288 <= 296.  C = 44: 18+1+2+3+5+3+1+5 = 38, 8 * 38 = 304 > 296.  So C = 45, S' = 17.
+    assert plan == (O.WORK_QUEUE, 17, 45, 0), ("policy_fill worked case", plan)
+
+
+HOST_PINS = (queue_closed_form, queue_cover, queue_bruteforce, policy_paper, policy_semantics, policy_fill,
              launch_fanout, merge_state_closed, balanced_shares, balanced_cover, balanced_bruteforce)
 
 

@@ -76,11 +76,12 @@ def test_policy_matches_oracle_bit_exactly(L):
     tables = [bd.load_rules(os.path.join(ROOT, "paged_kv_gqa_17_b200", f))
               for f in ("policy_paper_rule.json", "policy_b200.json")]
     tables.append([bd.Rule(0, 3, 0, 5000, 1, 7, 0, 1), bd.Rule(3, 100, 100, 2**31 - 1, 2, 1, 5, 0)])
+    tables += [[bd.Rule(0, 2**31 - 1, 0, 2**31 - 1, 2, T, 0, 4)] for T in (1, 37, 296)]  # queue filling T blocks
     for lens, H_kv, G, D in _cases(1):
         shape = _shape(lens, H_kv, G, D)
         for rules in tables:
             got = bd.select_policy(lens, shape, rules).tuple()
-            want = O.select_policy(lens, 16, [O.Rule(*r.tuple()) for r in rules])
+            want = O.select_policy(lens, 16, [O.Rule(*r.tuple()) for r in rules], H_kv)
             assert got == want, (lens, got, want)
 
 
@@ -199,8 +200,8 @@ def test_host_pins_hold_for_the_c_planner(L):
             return [tuple(x) for x in items.tolist()], ptr[:pairs + 1], ptr[pairs + 1:]
 
         @staticmethod
-        def select_policy(lens, P, rules):
-            shape = bd.make_shape(len(lens), 8, 8, 64, P, 1, 1)
+        def select_policy(lens, P, rules, H_kv=1):
+            shape = bd.make_shape(len(lens), H_kv, H_kv, 64, P, 1, 1)
             try:
                 return bd.select_policy(lens, shape, [r.__dict__ if hasattr(r, "__dict__") else r for r in rules]
                                         ).tuple()

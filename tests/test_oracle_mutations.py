@@ -48,6 +48,10 @@ PY_MUTANTS = {
     "balanced share rounded up": ("starts = [(b * U) // T for b in range(T + 1)]",
                                   "starts = [min(U, -(-(b * U) // T)) for b in range(T + 1)]"),
     "balanced item not clipped to row": ("min((y - u) * P, n)", "(y - u) * P"),
+    "fill rule allows one item too many": ("if fill_items(lens, H_kv, P, c) <= chosen.num_splits:",
+                                           "if fill_items(lens, H_kv, P, c) <= chosen.num_splits + 1:"),
+    "fill rule ignores heads": ("    return H_kv * sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)",
+                                "    return sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)"),
 }
 
 
