@@ -1,24 +1,25 @@
 """Calibrate the built-in policy table on the GPU from measured timings.
 
-    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--steps 100]
+    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--steps 60] [--draws 3]
 
 The policy maps (batch size B, longest row N_max) to an execution plan
 [PersistentKV explainer, Technical summary > Methodology > 2 "Calibrated
 adaptive policy": thresholds calibrated by hand on one seed, results reported
 on a holdout seed].  This script does the same by measurement:
 
-  1. For every cell of a (B, N_max) grid it draws a batch with the calibration
-     seed 20260622: one row of the cell's representative length, the others
-     log-uniform between an eighth of it and it (H_q=32, H_kv=8, D=128,
-     16-token pages).
+  1. For every cell of a (B, N_max) grid it draws three batches with the
+     calibration seed 20260622: one row of the cell's representative length,
+     the others log-uniform between an eighth of it and it (H_q=32, H_kv=8,
+     D=128, 16-token pages).
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
      the work queue over seven chunk sizes, with and without the deep ring,
      and with the chunk size that fills one wave of 296 or 444 blocks; the
-     balanced grid at one and two blocks per SM) as the steady-state device time of back-to-back
-     steps over rotating pool copies.
-  3. The fastest plan of each cell becomes a rule; neighbouring cells of one B
-     with the same plan are merged.
+     balanced grid at one and two blocks per SM) as the steady-state device
+     time of back-to-back steps over rotating pool copies.
+  3. The plan with the smallest geometric-mean time over the cell's batches
+     becomes a rule; neighbouring cells of one B with the same plan are
+     merged.
   4. Every cell is re-measured with the holdout seed 20260623; the report
      lists the chosen plan's time against the best candidate (the regret).
 
@@ -59,29 +60,33 @@ def candidates():
     return out
 
 
-def cell_lengths(B: int, n_rep: int, seed: int):
+def cell_lengths(B: int, n_rep: int, seed: int, draw: int = 0):
     import torch
 
-    g = torch.Generator().manual_seed(seed * 1000 + B * 7 + n_rep)
+    g = torch.Generator().manual_seed(seed * 1000 + B * 7 + n_rep + 100003 * draw)
     lo = max(16, n_rep // 8)
     rest = torch.rand(max(0, B - 1), generator=g, dtype=torch.float64)
     lens = [n_rep] + [int(math.exp(math.log(lo) + float(u) * (math.log(n_rep) - math.log(lo)))) for u in rest]
     return lens
 
 
-def measure_cell(B, n_rep, seed, steps, cands, torch, bd, W, bench):
+def measure_cell(B, n_rep, seed, steps, cands, torch, bd, W, bench, draws=1):
+    """Geometric mean over `draws` batches of the cell of each candidate's
+    steady-state µs per step."""
     dev = torch.device("cuda")
-    w = W.make_custom(cell_lengths(B, n_rep, seed), 32, 8, 128, seed=seed, device=dev)
-    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
-    copies = bench.pool_copies(w, torch)
-    times = {}
-    for c in cands:
-        rule = bd.Rule(0, 2**31 - 1, 0, 2**31 - 1, *c)
-        dp = bd.plan_decode(w.seq_lens, shape, dev, rules=[rule])
-        times[c] = bench.time_steady(w, dp, steps, 3, torch, bd, copies) / steps * 1e3  # us per step
-    del copies, w
-    torch.cuda.empty_cache()
-    return times
+    logs = {c: 0.0 for c in cands}
+    for d in range(draws):
+        w = W.make_custom(cell_lengths(B, n_rep, seed, d), 32, 8, 128, seed=seed + d, device=dev)
+        shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+        copies = bench.pool_copies(w, torch)
+        for c in cands:
+            rule = bd.Rule(0, 2**31 - 1, 0, 2**31 - 1, *c)
+            dp = bd.plan_decode(w.seq_lens, shape, dev, rules=[rule])
+            us = bench.time_steady(w, dp, steps, 3, torch, bd, copies) / steps * 1e3
+            logs[c] += math.log(us) / draws
+        del copies, w
+        torch.cuda.empty_cache()
+    return {c: math.exp(v) for c, v in logs.items()}
 
 
 def build_rules(best):
@@ -116,7 +121,8 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--out", default=os.path.join(HERE, "policy_b200.json"))
     ap.add_argument("--report", default=os.path.join(ROOT, "profiles", "policy_calibration_b200.md"))
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--draws", type=int, default=3, help="batches per cell (geometric mean)")
     args = ap.parse_args(argv)
 
     import torch
@@ -130,7 +136,7 @@ def main(argv=None):
     best, calib = {}, {}
     for bi, B in enumerate(B_REP):
         for nj, n in enumerate(N_REP):
-            t = measure_cell(B, n, W.SEED_CALIBRATE, args.steps, cands, torch, bd, W, bench)
+            t = measure_cell(B, n, W.SEED_CALIBRATE, args.steps, cands, torch, bd, W, bench, args.draws)
             calib[(bi, nj)] = t
             best[(bi, nj)] = min(t, key=t.get)
             print(f"B={B:3d} N_max={n:6d} best {best[(bi, nj)]} {t[best[(bi, nj)]]:.2f} us", flush=True)
@@ -149,14 +155,15 @@ def main(argv=None):
     # holdout check
     lines = ["# Policy calibration on B200", "",
              "Command: `python -m paged_kv_gqa_17_b200.calibrate` (writes paged_kv_gqa_17_b200/policy_b200.json).", "",
-             "Steady-state µs per decode step (back-to-back steps over rotating pool copies), H_q=32, H_kv=8, "
-             "D=128. Calibration seed 20260622 picks the plan; holdout seed 20260623 re-measures it.", "",
+             "Steady-state µs per decode step (CUDA-graph replay of back-to-back steps over rotating pool copies), "
+             f"H_q=32, H_kv=8, D=128; each cell is the geometric mean over {args.draws} batches of its lengths. "
+             "Calibration seed 20260622 picks the plan; holdout seed 20260623 (other batches) re-measures it.", "",
              "| B | N_max | chosen plan (mode, S/T, C, flags) | calib µs | holdout µs | holdout best | best µs | regret |",
              "|---|---|---|---|---|---|---|---|"]
     for bi, B in enumerate(B_REP):
         for nj, n in enumerate(N_REP):
             c = best[(bi, nj)]
-            hold = measure_cell(B, n, W.SEED_REPORT, args.steps, cands, torch, bd, W, bench)
+            hold = measure_cell(B, n, W.SEED_REPORT, args.steps, cands, torch, bd, W, bench, args.draws)
             hb = min(hold, key=hold.get)
             lines.append(f"| {B} | {n} | {MODE_NAMES[c[0]]} {c[1:]} | {calib[(bi, nj)][c]:.2f} | {hold[c]:.2f} | "
                          f"{MODE_NAMES[hb[0]]} {hb[1:]} | {hold[hb]:.2f} | {100 * (hold[c] / hold[hb] - 1):.1f}% |")
