@@ -9,8 +9,8 @@ on a holdout seed].  This script does the same by measurement:
 
   1. For every cell of a (B, N_max) grid it draws three batches with the
      calibration seed 20260622: one row of the cell's representative length,
-     the others log-uniform between an eighth of it and it (H_q=32, H_kv=8,
-     D=128, 16-token pages).
+     the others log-uniform between 1/8, 1/64 and 1/512 of it (one batch
+     each) and it (H_q=32, H_kv=8, D=128, 16-token pages).
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
      the work queue over seven chunk sizes, with and without the deep ring,
@@ -64,7 +64,7 @@ def cell_lengths(B: int, n_rep: int, seed: int, draw: int = 0):
     import torch
 
     g = torch.Generator().manual_seed(seed * 1000 + B * 7 + n_rep + 100003 * draw)
-    lo = max(16, n_rep // 8)
+    lo = max(16, n_rep // (8, 64, 512)[draw % 3])  # mild, strong and extreme length skew
     rest = torch.rand(max(0, B - 1), generator=g, dtype=torch.float64)
     lens = [n_rep] + [int(math.exp(math.log(lo) + float(u) * (math.log(n_rep) - math.log(lo)))) for u in rest]
     return lens
