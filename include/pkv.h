@@ -219,6 +219,36 @@ PKV_API int pkv_build_balanced_queue(const int32_t *seq_lens_host, const pkv_sha
                                      int32_t n_blocks, pkv_work_item *items, int32_t capacity,
                                      int32_t *indptr, int32_t *n_items);
 
+/* Items pkv_build_balanced_queue can emit for any lengths of this shape:
+ * B*H_kv + n_blocks (an upper bound; the exact count is
+ * pkv_balanced_queue_size).  Sizes the buffers of the device-side builder. */
+PKV_API int pkv_balanced_queue_capacity(const pkv_shape *shape, int32_t n_blocks, int32_t *capacity);
+
+/* The balanced queue built on the device from device-resident lengths,
+ * bit-identical to pkv_build_balanced_queue for the same lengths, so that a
+ * decode step whose lengths change on the device (a replayed CUDA graph)
+ * needs no host planning.  There is no counterpart on the pages beyond the
+ * queue itself [PKV, Methodology 1 "Compact work queue"]; this is the
+ * device-side builder the queue invites.
+ *   seq_lens   device int32 [B] (read after the kernel queued before on
+ *              `stream` completes); a length outside [0, max_pages_per_seq * P]
+ *              is clamped and sets the seq_len bit in `workspace`'s error word
+ *   items      device, >= pkv_balanced_queue_capacity() entries; entries past
+ *              the real count are left untouched
+ *   indptr     device int32, B*H_kv + 1 + n_blocks + 1 entries: pair offsets,
+ *              then block offsets, as pkv_build_balanced_queue
+ *   workspace  the workspace of the decode call that will read the queue
+ *              (its error word)
+ * Then call pkv_paged_decode with a BALANCED plan of num_splits = n_blocks,
+ * the same items / indptr and n_items = the capacity (the workspace sized for
+ * that many items).  Asynchronous on `stream`, one kernel (one block of
+ * threads), capturable in a CUDA graph.  B must be <= 4096
+ * (PKV_ERR_UNSUPPORTED otherwise); capacity below the bound returns
+ * PKV_ERR_CAPACITY before anything is queued. */
+PKV_API int pkv_build_balanced_queue_device(const int32_t *seq_lens, const pkv_shape *shape,
+                                            int32_t n_blocks, pkv_work_item *items, int32_t capacity,
+                                            int32_t *indptr, void *workspace, void *stream);
+
 /* Closed-form workload counters of `plan` on this batch (host, pure). */
 PKV_API int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape,
                               const pkv_plan *plan, pkv_counters *counters);

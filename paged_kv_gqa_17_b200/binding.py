@@ -82,6 +82,8 @@ SIGNATURES = [
     ("pkv_build_work_queue", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p]),
     ("pkv_balanced_queue_size", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_build_balanced_queue", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p]),
+    ("pkv_balanced_queue_capacity", ctypes.c_int, [c_p, c_i32, c_p]),
+    ("pkv_build_balanced_queue_device", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p, c_p]),
     ("pkv_plan_counters", ctypes.c_int, [c_p, c_p, c_p, c_p]),
     ("pkv_workspace_bytes", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_workspace_init", ctypes.c_int, [c_p, c_sz, c_p]),
@@ -224,6 +226,23 @@ def build_balanced_queue(seq_lens_host, shape: Shape, n_blocks: int):
     return items[:n.value], indptr
 
 
+def balanced_queue_capacity(shape: Shape, n_blocks: int) -> int:
+    L = lib()
+    n = c_i32(0)
+    _check(L.pkv_balanced_queue_capacity(ctypes.byref(shape), n_blocks, ctypes.byref(n)), "pkv_balanced_queue_capacity")
+    return int(n.value)
+
+
+def build_balanced_queue_device(seq_lens: torch.Tensor, shape: Shape, n_blocks: int, items: torch.Tensor,
+                                indptr: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """pkv_build_balanced_queue_device: the balanced queue built on the GPU from
+    device lengths into `items` / `indptr` (see include/pkv.h)."""
+    L = lib()
+    _check(L.pkv_build_balanced_queue_device(seq_lens.data_ptr(), ctypes.byref(shape), n_blocks, items.data_ptr(),
+                                             int(items.shape[0]), indptr.data_ptr(), workspace.data_ptr(),
+                                             _stream_ptr(stream)), "pkv_build_balanced_queue_device")
+
+
 def plan_counters(seq_lens_host, shape: Shape, plan: Plan) -> dict:
     L = lib()
     lens, _ = _lens_array(seq_lens_host)
@@ -248,8 +267,10 @@ def _stream_ptr(stream=None) -> int:
 @dataclass
 class DecodePlan:
     """Everything a decode step needs besides the tensors: the plan, the queue
-    on the device (WORK_QUEUE) and a zeroed workspace.  Reusable for every
-    step with the same sequence lengths and shape."""
+    on the device (WORK_QUEUE, BALANCED) and a zeroed workspace.  Reusable for
+    every step with the same sequence lengths and shape; with device_queue
+    (BALANCED only) the queue is rebuilt on the GPU from the device lengths at
+    every step, so the plan serves any lengths up to the shape's maximum."""
 
     shape: Shape
     plan: Plan
@@ -258,12 +279,24 @@ class DecodePlan:
     n_items: int
     workspace: torch.Tensor
     counters: dict
+    device_queue: bool = False
 
 
-def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[Plan] = None) -> DecodePlan:
-    """Host planning for one batch: policy (unless `plan` is given), queue, workspace."""
+def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[Plan] = None,
+                device_queue: bool = False) -> DecodePlan:
+    """Host planning for one batch: policy (unless `plan` is given), queue, workspace.
+    device_queue=True (with a BALANCED plan) leaves the queue to the GPU: buffers
+    of pkv_balanced_queue_capacity items, filled by every paged_decode call."""
     if plan is None:
         plan = select_policy(seq_lens_host, shape, rules)
+    if device_queue:
+        if plan.mode != BALANCED:
+            raise PkvError(-1, "device_queue needs a BALANCED plan")
+        cap = balanced_queue_capacity(shape, plan.num_splits)
+        items = torch.zeros((cap, 4), dtype=torch.int32, device=device)
+        indptr = torch.zeros(shape.B * shape.H_kv + 1 + plan.num_splits + 1, dtype=torch.int32, device=device)
+        ws = torch.zeros(workspace_bytes(shape, plan, cap), dtype=torch.uint8, device=device)
+        return DecodePlan(shape, plan, items, indptr, cap, ws, plan_counters(seq_lens_host, shape, plan), True)
     items = indptr = None
     n_items = 0
     if plan.mode in (WORK_QUEUE, BALANCED):
@@ -297,6 +330,9 @@ def paged_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, bl
     shape = plan.shape
     if out is None:
         out = torch.empty_like(q)
+    if plan.device_queue:
+        build_balanced_queue_device(seq_lens, shape, plan.plan.num_splits, plan.items, plan.indptr, plan.workspace,
+                                    stream)
     rc = L.pkv_paged_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
                             seq_lens.data_ptr(), page_size, float(scale), out.data_ptr(), ctypes.byref(shape),
                             ctypes.byref(plan.plan), plan.items.data_ptr() if plan.items is not None else None,

@@ -1727,6 +1727,150 @@ __global__ void wait_timeout_selftest_kernel(uint32_t *err, uint64_t limit_ns)
 }
 
 // ---------------------------------------------------------------------------
+// Device-side builder of the balanced queue, so that a decode step whose
+// lengths change on the device (a CUDA graph replayed every step) needs no
+// host planning.  Same output as pkv_build_balanced_queue for the same
+// lengths: the (row, KV head) pairs laid end to end, U pages in all, block b
+// of T owning pages [floor(bU/T), floor((b+1)U/T)); every maximal run of one
+// pair's pages in one share is an item, a row with no tokens gets one empty
+// item per head owned by the last block whose share starts at or before the
+// pair's position; indptr holds the pair offsets, then the block offsets.
+// One block of threads: the row page counts and the per-pair item counts are
+// each prefix-summed over the block, and each thread emits its pair's items.
+
+constexpr int kBuildThreads = 1024;
+constexpr int kBuildMaxRows = 4096;
+
+__device__ __forceinline__ int64_t share_start(int64_t U, int64_t T, int64_t b) { return (b * U) / T; }
+
+// Last block whose share starts at or before page u: the largest b < T with
+// floor(bU/T) <= u, i.e. bU < (u+1)T, i.e. b = ceil((u+1)T / U) - 1.
+__device__ __forceinline__ int64_t share_owner(int64_t U, int64_t T, int64_t u)
+{
+    if (U == 0)
+        return T - 1;
+    const int64_t b = ((u + 1) * T + U - 1) / U - 1;
+    return b < T - 1 ? b : T - 1;
+}
+
+// Inclusive prefix sum of v over the block (all threads call it).
+__device__ int64_t block_inclusive_scan(int64_t v, int64_t *scan)
+{
+    const int tid = threadIdx.x;
+    scan[tid] = v;
+    __syncthreads();
+    for (int off = 1; off < kBuildThreads; off <<= 1) {
+        const int64_t add = tid >= off ? scan[tid - off] : 0;
+        __syncthreads();
+        scan[tid] += add;
+        __syncthreads();
+    }
+    const int64_t r = scan[tid];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kBuildThreads)
+    balanced_queue_kernel(const int32_t *lens, int32_t B, int32_t H_kv, int32_t P, int32_t max_pages, int32_t T,
+                          int4 *items, int32_t capacity, int32_t *indptr, uint32_t *err)
+{
+    __shared__ int64_t row_start[kBuildMaxRows + 1];  // pages of one head's rows before row i
+    __shared__ int64_t scan[kBuildThreads];
+    __shared__ int64_t total;
+    grid_dependency_wait();     // the lengths may come from the kernel before
+    grid_launch_dependents();  // the decode kernel may start its set-up
+    const int tid = threadIdx.x;
+    const int64_t cap_tokens = (int64_t)max_pages * P;
+    auto clamped_len = [&](int i) {
+        int64_t N = lens[i];
+        if (N < 0 || N > cap_tokens) {
+            atomicOr(err, kErrSeqLen);
+            N = N < 0 ? 0 : cap_tokens;
+        }
+        return N;
+    };
+    int64_t carry = 0;
+    for (int base = 0; base < B; base += kBuildThreads) {
+        const int i = base + tid;
+        const int64_t pg = i < B ? (clamped_len(i) + P - 1) / P : 0;
+        const int64_t incl = block_inclusive_scan(pg, scan);
+        if (i < B)
+            row_start[i] = carry + incl - pg;
+        if (tid == kBuildThreads - 1)
+            total = carry + incl;
+        __syncthreads();
+        carry = total;
+        __syncthreads();
+    }
+    if (tid == 0)
+        row_start[B] = carry;
+    __syncthreads();
+    const int64_t U = carry * H_kv;
+    const int64_t pairs = (int64_t)B * H_kv;
+    int32_t *block_ptr = indptr + pairs + 1;
+    // position and page count of pair q; the owner of its last item
+    auto pair_span = [&](int64_t q, int64_t &a, int64_t &n) {
+        const int iq = (int)(q / H_kv);
+        n = row_start[iq + 1] - row_start[iq];
+        a = row_start[iq] * H_kv + (q % H_kv) * n;
+    };
+    auto last_owner = [&](int64_t q) {
+        int64_t a, n;
+        pair_span(q, a, n);
+        return share_owner(U, T, n == 0 ? a : a + n - 1);
+    };
+    carry = 0;
+    for (int64_t base = 0; base < pairs; base += kBuildThreads) {
+        const int64_t p = base + tid;
+        int64_t a = 0, n = 0, cnt = 0;
+        if (p < pairs) {
+            pair_span(p, a, n);
+            // distinct owners of the pair's pages: every share holds a page when U >= T,
+            // exactly one page or none when U < T
+            const int64_t span = share_owner(U, T, a + n - 1) - share_owner(U, T, a) + 1;
+            cnt = n == 0 ? 1 : (span < n ? span : n);
+        }
+        const int64_t incl = block_inclusive_scan(cnt, scan);
+        const int64_t o = carry + incl - cnt;
+        if (p < pairs) {
+            indptr[p] = (int32_t)o;
+            const int i = (int)(p / H_kv), h = (int)(p % H_kv);
+            const int64_t N = clamped_len(i);
+            int64_t prev = p == 0 ? -1 : last_owner(p - 1);
+            int64_t x = a, idx = o;
+            for (int64_t k = 0; k < cnt; ++k, ++idx) {
+                const int64_t b = share_owner(U, T, x);
+                int4 it = make_int4(i, h, 0, 0);
+                if (n > 0) {
+                    const int64_t end = share_start(U, T, b + 1);
+                    const int64_t y = a + n < end ? a + n : end;
+                    it.z = (int)((x - a) * P);
+                    it.w = (int)((y - a) * P < N ? (y - a) * P : N);
+                    x = y;
+                }
+                if (idx < capacity)
+                    items[idx] = it;
+                else
+                    atomicOr(err, kErrItem);
+                for (int64_t c = prev + 1; c <= b; ++c)
+                    block_ptr[c] = (int32_t)idx;
+                prev = b;
+            }
+            if (p == pairs - 1) {
+                indptr[pairs] = (int32_t)(o + cnt);
+                for (int64_t c = prev + 1; c <= T; ++c)
+                    block_ptr[c] = (int32_t)(o + cnt);
+            }
+        }
+        if (tid == kBuildThreads - 1)
+            total = carry + incl;
+        __syncthreads();
+        carry = total;
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 
 namespace {
@@ -2195,6 +2339,40 @@ __attribute__((visibility("default"))) int pkv_trace_read(void *host, size_t byt
     return cudaMemcpyFromSymbol(host, g_pkv_trace_buf, bytes) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 #endif
+
+int pkv_build_balanced_queue_device(const int32_t *seq_lens, const pkv_shape *shape, int32_t n_blocks,
+                                    pkv_work_item *items, int32_t capacity, int32_t *indptr, void *workspace,
+                                    void *stream)
+{
+    int32_t need = 0;
+    int rc = pkv_balanced_queue_capacity(shape, n_blocks, &need);
+    if (rc != PKV_OK)
+        return rc;
+    const pkv_shape &s = *shape;
+    if (s.B == 0)
+        return PKV_OK;
+    if (s.B > kBuildMaxRows)
+        return PKV_ERR_UNSUPPORTED;
+    if (capacity < need)
+        return PKV_ERR_CAPACITY;
+    if (!seq_lens || !items || !indptr || !workspace)
+        return PKV_ERR_INVALID;
+    if (!aligned(items, 16) || !aligned(indptr, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 256))
+        return PKV_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kBuildThreads);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, balanced_queue_kernel, seq_lens, s.B, s.H_kv, s.page_size,
+                                             s.max_pages_per_seq, n_blocks, reinterpret_cast<int4 *>(items),
+                                             capacity, indptr, static_cast<uint32_t *>(workspace));
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
 
 int pkv_selftest_wait_timeout(void *workspace, size_t workspace_bytes, uint32_t limit_us, void *stream)
 {

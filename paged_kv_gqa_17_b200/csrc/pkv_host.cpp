@@ -284,6 +284,19 @@ int pkv_balanced_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape
     return PKV_OK;
 }
 
+int pkv_balanced_queue_capacity(const pkv_shape *shape, int32_t n_blocks, int32_t *capacity)
+{
+    if (!capacity || n_blocks < 1 || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    // each item is one pair's run inside one share: at most one per pair plus one
+    // per share boundary falling inside a pair's pages (T - 1 of them)
+    const int64_t c = (int64_t)shape->B * shape->H_kv + n_blocks;
+    if (c > INT32_MAX)
+        return PKV_ERR_CAPACITY;
+    *capacity = (int32_t)c;
+    return PKV_OK;
+}
+
 int pkv_build_balanced_queue(const int32_t *seq_lens_host, const pkv_shape *shape, int32_t n_blocks,
                              pkv_work_item *items, int32_t capacity, int32_t *indptr, int32_t *n_items)
 {

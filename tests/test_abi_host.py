@@ -222,3 +222,23 @@ def test_host_pins_hold_for_the_c_planner(L):
 
     failed = host_pins.run_all(Adapter)
     assert not failed, failed
+
+
+def test_device_queue_builder_host_checks(L):
+    """The device-side builder rejects what it cannot do before queueing
+    anything (no GPU needed for these paths)."""
+    shape = bd.make_shape(4, 8, 2, 128, 16, 8, 10)
+    cap = ctypes.c_int32(0)
+    assert L.pkv_balanced_queue_capacity(ctypes.byref(shape), 37, ctypes.byref(cap)) == 0
+    assert cap.value == 4 * 2 + 37
+    assert L.pkv_balanced_queue_capacity(ctypes.byref(shape), 0, ctypes.byref(cap)) == -1
+    # capacity below the bound
+    assert L.pkv_build_balanced_queue_device(None, ctypes.byref(shape), 37, None, 44, None, None, None) == -3
+    # missing buffers
+    assert L.pkv_build_balanced_queue_device(None, ctypes.byref(shape), 37, None, 45, None, None, None) == -1
+    # more rows than the one-block builder handles
+    big = bd.make_shape(5000, 8, 2, 128, 16, 8, 10)
+    assert L.pkv_build_balanced_queue_device(None, ctypes.byref(big), 37, None, 1 << 20, None, None, None) == -2
+    # an empty batch queues nothing
+    empty = bd.make_shape(0, 8, 2, 128, 16, 8, 10)
+    assert L.pkv_build_balanced_queue_device(None, ctypes.byref(empty), 37, None, 0, None, None, None) == 0

@@ -1,0 +1,117 @@
+"""The balanced queue built on the GPU (pkv_build_balanced_queue_device):
+bit-identical to the host builder, decodes that match the oracle, and a
+decode step captured once in a CUDA graph that stays correct while the
+lengths change on the device between replays."""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_gqa_17_b200 import binding as bd
+from paged_kv_gqa_17_b200 import workloads as W
+
+from .gpu_util import assert_close, oracle_full, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_gqa_17_b200 import build
+
+    build.build()
+    bd.lib()
+
+
+def _device_queue(lens, shape, T):
+    cap = bd.balanced_queue_capacity(shape, T)
+    items = torch.full((cap, 4), -7, dtype=torch.int32, device="cuda")
+    indptr = torch.full((shape.B * shape.H_kv + 1 + T + 1,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(bd.workspace_bytes(shape, bd.Plan(3, T, 0, 0), cap), dtype=torch.uint8, device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    bd.build_balanced_queue_device(lens_d, shape, T, items, indptr, ws)
+    torch.cuda.synchronize()
+    return items.cpu(), indptr.cpu(), ws
+
+
+def test_device_builder_matches_host_builder_bit_exactly():
+    rng = np.random.default_rng(21)
+    cases = [([0, 0, 0], 2, 5), ([1], 1, 296), ([17, 0, 5], 4, 296), ([16] * 5, 8, 7), ([32768], 8, 296),
+             ([12129, 621, 1118, 1452, 2891, 1419, 518, 3174], 8, 296), ([5000, 0, 1, 16, 17], 2, 1)]
+    for _ in range(40):
+        B = int(rng.integers(1, 70))
+        lens = [int(x) for x in rng.choice([0, 1, 15, 16, 17, 300, 5000, 40000], B)]
+        cases.append((lens, int(rng.choice([1, 2, 4, 8])), int(rng.choice([1, 3, 37, 148, 296, 1000]))))
+    for lens, H_kv, T in cases:
+        max_pages = max([-(-n // 16) for n in lens] + [1])
+        shape = bd.make_shape(len(lens), 4 * H_kv, H_kv, 128, 16, max_pages, 10)
+        h_items, h_indptr = bd.build_balanced_queue(lens, shape, T)
+        d_items, d_indptr, ws = _device_queue(lens, shape, T)
+        n = h_items.shape[0]
+        assert n <= d_items.shape[0]
+        assert torch.equal(d_items[:n], h_items), (lens, H_kv, T)
+        assert torch.equal(d_indptr, h_indptr), (lens, H_kv, T)
+        assert (d_items[n:] == -7).all()  # entries past the real count untouched
+        assert int(ws[:4].view(torch.int32)[0]) == 0
+
+
+@pytest.mark.parametrize("T", [1, 7, 37, 296])
+def test_decode_with_device_queue_matches_oracle(T):
+    w = to_device(W.make_custom([3000, 77, 1999, 16, 0, 1], 32, 8, 128, seed=140, poison=True))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", plan=bd.Plan(3, T, 0, 0), device_queue=True)
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
+    out = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp)
+    torch.cuda.synchronize()
+    assert bd.workspace_status(dp) == 0
+    got = out.float().cpu().double().numpy()
+    assert_close(got, oracle_full(w), f"device queue T={T}")
+    host = bd.plan_decode(w.seq_lens, shape, "cuda", plan=bd.Plan(3, T, 0, 0))
+    ref = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=host)
+    assert torch.equal(out, ref)  # same queue, same kernels: the same bits
+
+
+def test_graph_replay_follows_lengths_changed_on_the_device():
+    """One decode step captured in a CUDA graph (queue build + balanced
+    kernel); between replays only the device lengths change (rows grow,
+    shrink, empty), and every replay matches the oracle for its lengths."""
+    full = [2500, 900, 40, 1300]
+    w = to_device(W.make_custom(full, 16, 4, 128, seed=141, poison=False))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dp = bd.plan_decode(full, shape, "cuda", plan=bd.Plan(3, 37, 0, 0), device_queue=True)
+    lens = torch.tensor(full, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(w.q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    for step_lens in ([2500, 900, 40, 1300], [2501, 901, 41, 1301], [17, 0, 40, 2560], [0, 0, 0, 0], [1, 2, 3, 4],
+                      [2000, 2000, 2000, 2000]):
+        lens.copy_(torch.tensor(step_lens, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        assert bd.workspace_status(dp) == 0
+        w.seq_lens = list(step_lens)
+        assert_close(out.float().cpu().double().numpy(), oracle_full(w), f"replay {step_lens}")
+    del g
+
+
+def test_device_builder_flags_bad_lengths():
+    shape = bd.make_shape(3, 8, 2, 128, 16, 4, 10)
+    lens = torch.tensor([10, 4 * 16 + 1, -3], dtype=torch.int32, device="cuda")
+    cap = bd.balanced_queue_capacity(shape, 5)
+    items = torch.zeros((cap, 4), dtype=torch.int32, device="cuda")
+    indptr = torch.zeros(3 * 2 + 1 + 5 + 1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    bd.build_balanced_queue_device(lens, shape, 5, items, indptr, ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32)[0]) & 2
+    # the clamped lengths (10, 64, 0) give the host builder's queue
+    h_items, h_indptr = bd.build_balanced_queue([10, 64, 0], shape, 5)
+    assert torch.equal(items.cpu()[:h_items.shape[0]], h_items) and torch.equal(indptr.cpu(), h_indptr)
