@@ -91,7 +91,8 @@ def test_graph_replay_follows_lengths_changed_on_the_device():
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
-    for step_lens in ([2500, 900, 40, 1300], [2501, 901, 41, 1301], [17, 0, 40, 2560], [0, 0, 0, 0], [1, 2, 3, 4],
+    cap = shape.max_pages_per_seq * 16  # 157 pages: lengths up to 2512 fit the tables
+    for step_lens in ([2500, 900, 40, 1300], [2501, 901, 41, 1301], [17, 0, 40, cap], [0, 0, 0, 0], [1, 2, 3, 4],
                       [2000, 2000, 2000, 2000]):
         lens.copy_(torch.tensor(step_lens, dtype=torch.int32))
         g.replay()
