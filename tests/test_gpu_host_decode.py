@@ -75,18 +75,21 @@ def test_host_path_matches_oracle_and_device_path(name):
     assert np.array_equal(got, dev), name
 
 
-def test_host_path_default_policy_picks_balanced():
-    """B=8 with N_max in [16384, 65536): the built-in table picks the balanced
-    grid, whose queue the host path builds and uploads itself."""
+@pytest.mark.parametrize("rules", [[rule(3, 296)], [rule(2, 296, 0, 4)], None])
+def test_host_path_builds_the_queues_itself(rules):
+    """B=8, N_max = 20000: the balanced grid, the queue whose chunk fills one
+    wave (chunk_pages = 0) and the built-in table's plan, each built and
+    uploaded by the host path itself."""
     lens = [20000, 300, 9000, 17000, 64, 5000, 12345, 1]
     w = to_device(W.make_custom(lens, 32, 8, 128, seed=131, poison=True))
-    got, plan = host_decode(w)
-    assert plan.mode == bd.BALANCED, plan.tuple()
-    dev, dp = run(w)
+    got, plan = host_decode(w, rules=rules)
+    if rules is not None:
+        assert plan.mode == rules[0].mode, plan.tuple()
+    dev, dp = run(w, rules=rules)
     assert dp.plan.tuple() == plan.tuple()
     assert np.array_equal(got, dev)
     pairs = [(0, 0), (0, 31), (3, 17), (7, 5), (4, 9), (6, 30)]
-    assert_close(np.stack([got[r, h] for r, h in pairs]), oracle_sampled(w, pairs), "host/balanced")
+    assert_close(np.stack([got[r, h] for r, h in pairs]), oracle_sampled(w, pairs), f"host/{plan.tuple()}")
 
 
 @pytest.mark.parametrize("rules", [None, [rule(2, 1, 8)]])
