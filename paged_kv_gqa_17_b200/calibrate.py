@@ -10,7 +10,8 @@ on a holdout seed].  This script does the same by measurement:
   1. For every cell of a (B, N_max) grid it draws three batches with the
      calibration seed 20260622: one row of the cell's representative length,
      the others log-uniform between 1/8, 1/64 and 1/512 of it (one batch
-     each) and it (H_q=32, H_kv=8, D=128, 16-token pages).
+     each) and it (H_kv=8, D=128, 16-token pages; G = 4 for the first two
+     batches, G = 8 for the third).
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
      the work queue over seven chunk sizes, with and without the deep ring,
@@ -77,7 +78,8 @@ def measure_cell(B, n_rep, seed, steps, cands, torch, bd, W, bench, draws=1):
     dev = torch.device("cuda")
     logs = {c: 0.0 for c in cands}
     for d in range(draws):
-        w = W.make_custom(cell_lengths(B, n_rep, seed, d), 32, 8, 128, seed=seed + d, device=dev)
+        H_q = 64 if d % 3 == 2 else 32  # G = 4, and G = 8 for the third batch
+        w = W.make_custom(cell_lengths(B, n_rep, seed, d), H_q, 8, 128, seed=seed + d, device=dev)
         shape = bd.shape_of(w.q, w.k_pool, w.block_table)
         copies = bench.pool_copies(w, torch)
         for c in cands:
@@ -158,7 +160,7 @@ def main(argv=None):
         "name": "b200_calibrated",
         "about": "Built-in policy table of libpkv.so (pkv_default_policy), written by "
                  "paged_kv_gqa_17_b200/calibrate.py from steady-state timings on B200 with seed 20260622 "
-                 "(H_q=32, H_kv=8, D=128, 16-token pages). Rules are checked in order; the first whose "
+                 "(H_kv=8, G=4 and 8, D=128, 16-token pages). Rules are checked in order; the first whose "
                  "half-open ranges hold (B, N_max) decides.",
         "rules": rules,
     }
@@ -169,7 +171,7 @@ def main(argv=None):
     lines = ["# Policy calibration on B200", "",
              "Command: `python -m paged_kv_gqa_17_b200.calibrate` (writes paged_kv_gqa_17_b200/policy_b200.json).", "",
              "Steady-state µs per decode step (CUDA-graph replay of back-to-back steps over rotating pool copies), "
-             f"H_q=32, H_kv=8, D=128; each cell is the geometric mean over {args.draws} batches of its lengths. "
+             f"H_kv=8, D=128; each cell is the geometric mean over {args.draws} batches (G = 4, 4, 8). "
              "Calibration seed 20260622 picks the plan; holdout seed 20260623 (other batches) re-measures it.", "",
              "| B | N_max | chosen plan (mode, S/T, C, flags) | calib µs | holdout µs | holdout best | best µs | regret |",
              "|---|---|---|---|---|---|---|---|"]

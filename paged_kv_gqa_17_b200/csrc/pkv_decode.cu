@@ -867,22 +867,20 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
     return true;
 }
 
-// The last block's merge of a pair: up to kDirectMergeSlots states straight
-// into registers (one batch of L2 loads in flight per thread, or two), more
-// through the ring, whose bulk copies keep all of them in flight at once.
-// Both were timed on B200 with the step's own blocks as the merging blocks:
-// the direct path wins at 8-12 states (by about 1-2 us per step), the
-// staged one at 32.
-constexpr int kDirectMergeSlots = 16;
-
+// The last block's merge of a pair: through per-thread async copies into the
+// ring whenever the ring holds all n states ("landed"), else staged through
+// the ring in double-buffered bulk copies, else straight into registers.
+// Timed on B200 with the step's own blocks merging: landed beat staged at 17
+// states (mixed batch, 18.3 -> 17.5 us per step) and at 32 (long context,
+// 24.2 -> 23.2 us per step).
 template <int D, int NT, int NW, int NST>
 __device__ void merge_pair_last_block(const Params &p, uint8_t *smem, uint32_t mbar0, int row, int h, int slot0,
                                       int n, int tid, uint32_t (&uses)[2])
 {
     using C = Cfg<D, NT, NW, NST>;
-    if (n <= kDirectMergeSlots && merge_pair_landed<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid))
+    if (merge_pair_landed<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid))
         return;
-    if (n <= kDirectMergeSlots || !merge_pair_staged<D, NT, NW, NST>(p, smem, mbar0, row, h, slot0, n, tid, uses))
+    if (!merge_pair_staged<D, NT, NW, NST>(p, smem, mbar0, row, h, slot0, n, tid, uses))
         merge_pair_direct<D>(p, row, h, slot0, n, tid, C::kThreads);
 }
 
