@@ -371,12 +371,20 @@ def workspace_status(plan: DecodePlan, stream=None) -> int:
 
 class HostDecoder:
     """Caller-owned buffers for pkv_decode_host, grown on demand: one device
-    buffer (torch) and one page-locked host staging buffer."""
+    buffer (torch) and one page-locked host staging buffer.  Calls run on
+    `stream` (default: the device's current stream when the decoder is made)
+    unless a call passes its own; the per-call Python work is kept to the
+    argument pointers, since a serving loop calls this once per step."""
 
-    def __init__(self, device):
+    def __init__(self, device, stream=None):
         self.device = torch.device(device)
         self.dev = torch.empty(0, dtype=torch.uint8, device=self.device)
         self.host = torch.empty(0, dtype=torch.uint8).pin_memory()
+        self._stream = _stream_ptr(stream if stream is not None else torch.cuda.current_stream(self.device))
+        self._fn = lib().pkv_decode_host
+        self._plan = Plan()
+        self._plan_ref = ctypes.byref(self._plan)
+        self._bufs = (0, 0, 0, 0)
 
     def ensure(self, seq_lens_host, shape: Shape, rules=None):
         L = lib()
@@ -389,19 +397,19 @@ class HostDecoder:
             self.dev = torch.zeros(db.value, dtype=torch.uint8, device=self.device)
         if self.host.numel() < hb.value:
             self.host = torch.zeros(hb.value, dtype=torch.uint8).pin_memory()
+        self._bufs = (self.dev.data_ptr(), self.dev.numel(), self.host.data_ptr(), self.host.numel())
 
     def __call__(self, q_host: torch.Tensor, block_table_host: torch.Tensor, seq_lens_host: torch.Tensor,
                  out_host: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, scale: float, shape: Shape,
                  rules=None, stream=None) -> Plan:
-        L = lib()
-        arr, n = rules_array(rules)
-        plan = Plan()
-        rc = L.pkv_decode_host(q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(),
-                               out_host.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), float(scale),
-                               ctypes.byref(shape), arr, n, self.dev.data_ptr(), self.dev.numel(),
-                               self.host.data_ptr(), self.host.numel(), _stream_ptr(stream), ctypes.byref(plan))
-        _check(rc, "pkv_decode_host")
-        return plan
+        arr, n = rules_array(rules) if rules is not None else (None, 0)
+        dev, dev_n, host, host_n = self._bufs
+        rc = self._fn(q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(), out_host.data_ptr(),
+                      k_pool.data_ptr(), v_pool.data_ptr(), float(scale), ctypes.byref(shape), arr, n, dev, dev_n,
+                      host, host_n, self._stream if stream is None else _stream_ptr(stream), self._plan_ref)
+        if rc != 0:
+            raise PkvError(rc, "pkv_decode_host")
+        return Plan.from_buffer_copy(self._plan)
 
 
 def decode_host(*args, **kwargs):
