@@ -249,6 +249,26 @@ PKV_API int pkv_build_balanced_queue_device(const int32_t *seq_lens, const pkv_s
                                             int32_t n_blocks, pkv_work_item *items, int32_t capacity,
                                             int32_t *indptr, void *workspace, void *stream);
 
+/* Items the compact queue filling one wave of n_blocks blocks can hold for
+ * any lengths of this shape: max(n_blocks, B*H_kv). */
+PKV_API int pkv_fill_queue_capacity(const pkv_shape *shape, int32_t n_blocks, int32_t *capacity);
+
+/* The compact queue whose chunk fills one wave of T = n_blocks blocks, built
+ * on the device from device-resident lengths: the chunk C is the one
+ * pkv_select_policy picks for a WORK_QUEUE rule with chunk_pages = 0 and
+ * num_splits = T, and items / indptr (B*H_kv + 1 entries: pair offsets, the
+ * last one the item count) equal pkv_build_work_queue's at that C.  The
+ * device-side counterpart of the fill rule [PKV, Methodology 1 "Compact work
+ * queue"; the rule itself is this library's].  Arguments, errors, limits and
+ * capturability as pkv_build_balanced_queue_device; capacity >=
+ * pkv_fill_queue_capacity().  Then call pkv_paged_decode with a WORK_QUEUE
+ * plan (any chunk_pages >= 1: the items carry their token ranges), the same
+ * items / indptr and n_items = the capacity: the grid has that many blocks
+ * and those past the device-side count return at once. */
+PKV_API int pkv_build_fill_queue_device(const int32_t *seq_lens, const pkv_shape *shape, int32_t n_blocks,
+                                        pkv_work_item *items, int32_t capacity, int32_t *indptr,
+                                        void *workspace, void *stream);
+
 /* Closed-form workload counters of `plan` on this batch (host, pure). */
 PKV_API int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape,
                               const pkv_plan *plan, pkv_counters *counters);

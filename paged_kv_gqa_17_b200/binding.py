@@ -84,6 +84,8 @@ SIGNATURES = [
     ("pkv_build_balanced_queue", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p]),
     ("pkv_balanced_queue_capacity", ctypes.c_int, [c_p, c_i32, c_p]),
     ("pkv_build_balanced_queue_device", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p, c_p]),
+    ("pkv_fill_queue_capacity", ctypes.c_int, [c_p, c_i32, c_p]),
+    ("pkv_build_fill_queue_device", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p, c_p]),
     ("pkv_plan_counters", ctypes.c_int, [c_p, c_p, c_p, c_p]),
     ("pkv_workspace_bytes", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_workspace_init", ctypes.c_int, [c_p, c_sz, c_p]),
@@ -243,6 +245,23 @@ def build_balanced_queue_device(seq_lens: torch.Tensor, shape: Shape, n_blocks: 
                                              _stream_ptr(stream)), "pkv_build_balanced_queue_device")
 
 
+def fill_queue_capacity(shape: Shape, n_blocks: int) -> int:
+    L = lib()
+    n = c_i32(0)
+    _check(L.pkv_fill_queue_capacity(ctypes.byref(shape), n_blocks, ctypes.byref(n)), "pkv_fill_queue_capacity")
+    return int(n.value)
+
+
+def build_fill_queue_device(seq_lens: torch.Tensor, shape: Shape, n_blocks: int, items: torch.Tensor,
+                            indptr: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """pkv_build_fill_queue_device: the queue whose chunk fills one wave of
+    n_blocks blocks, built on the GPU from device lengths (see include/pkv.h)."""
+    L = lib()
+    _check(L.pkv_build_fill_queue_device(seq_lens.data_ptr(), ctypes.byref(shape), n_blocks, items.data_ptr(),
+                                         int(items.shape[0]), indptr.data_ptr(), workspace.data_ptr(),
+                                         _stream_ptr(stream)), "pkv_build_fill_queue_device")
+
+
 def plan_counters(seq_lens_host, shape: Shape, plan: Plan) -> dict:
     L = lib()
     lens, _ = _lens_array(seq_lens_host)
@@ -280,23 +299,35 @@ class DecodePlan:
     workspace: torch.Tensor
     counters: dict
     device_queue: bool = False
+    fill_blocks: int = 0  # device queue of a WORK_QUEUE plan: the wave it fills
 
 
 def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[Plan] = None,
-                device_queue: bool = False) -> DecodePlan:
+                device_queue: bool = False, fill_blocks: int = 296) -> DecodePlan:
     """Host planning for one batch: policy (unless `plan` is given), queue, workspace.
-    device_queue=True (with a BALANCED plan) leaves the queue to the GPU: buffers
-    of pkv_balanced_queue_capacity items, filled by every paged_decode call."""
+
+    device_queue=True leaves the queue to the GPU, rebuilt from the device
+    lengths by every paged_decode call (so one plan, or one captured CUDA
+    graph, serves any lengths up to the shape's maximum): a BALANCED plan
+    gets the balanced queue of its T blocks, a WORK_QUEUE plan the queue
+    whose chunk fills one wave of `fill_blocks` blocks."""
     if plan is None:
         plan = select_policy(seq_lens_host, shape, rules)
     if device_queue:
-        if plan.mode != BALANCED:
-            raise PkvError(-1, "device_queue needs a BALANCED plan")
-        cap = balanced_queue_capacity(shape, plan.num_splits)
+        pairs = shape.B * shape.H_kv
+        if plan.mode == BALANCED:
+            cap = balanced_queue_capacity(shape, plan.num_splits)
+            n_ptr = pairs + 1 + plan.num_splits + 1
+        elif plan.mode == WORK_QUEUE:
+            cap = fill_queue_capacity(shape, fill_blocks)
+            n_ptr = pairs + 1
+        else:
+            raise PkvError(-1, "device_queue needs a BALANCED or WORK_QUEUE plan")
         items = torch.zeros((cap, 4), dtype=torch.int32, device=device)
-        indptr = torch.zeros(shape.B * shape.H_kv + 1 + plan.num_splits + 1, dtype=torch.int32, device=device)
+        indptr = torch.zeros(n_ptr, dtype=torch.int32, device=device)
         ws = torch.zeros(workspace_bytes(shape, plan, cap), dtype=torch.uint8, device=device)
-        return DecodePlan(shape, plan, items, indptr, cap, ws, plan_counters(seq_lens_host, shape, plan), True)
+        return DecodePlan(shape, plan, items, indptr, cap, ws, plan_counters(seq_lens_host, shape, plan), True,
+                          fill_blocks if plan.mode == WORK_QUEUE else 0)
     items = indptr = None
     n_items = 0
     if plan.mode in (WORK_QUEUE, BALANCED):
@@ -330,9 +361,11 @@ def paged_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, bl
     shape = plan.shape
     if out is None:
         out = torch.empty_like(q)
-    if plan.device_queue:
+    if plan.device_queue and plan.plan.mode == BALANCED:
         build_balanced_queue_device(seq_lens, shape, plan.plan.num_splits, plan.items, plan.indptr, plan.workspace,
                                     stream)
+    elif plan.device_queue:
+        build_fill_queue_device(seq_lens, shape, plan.fill_blocks, plan.items, plan.indptr, plan.workspace, stream)
     rc = L.pkv_paged_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
                             seq_lens.data_ptr(), page_size, float(scale), out.data_ptr(), ctypes.byref(shape),
                             ctypes.byref(plan.plan), plan.items.data_ptr() if plan.items is not None else None,

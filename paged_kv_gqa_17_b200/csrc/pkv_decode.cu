@@ -995,6 +995,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     int e_first = 0;
     int row_len = -1;  // the row's length where known (for the early dependency gate)
     if (p.mode == PKV_WORK_QUEUE) {
+        // a queue built on the device may hold fewer items than the grid has blocks
+        if ((int)blockIdx.x >= __ldg(p.indptr + p.B * p.H_kv))
+            return;
         const int4 it = __ldg(p.items + blockIdx.x);
         row = it.x;
         h = it.y;
@@ -1868,6 +1871,124 @@ __global__ void __launch_bounds__(kBuildThreads)
     }
 }
 
+// The compact queue whose chunk fills one wave of T blocks, built on the
+// device: the same items and pair offsets as pkv_select_policy's fill rule
+// followed by pkv_build_work_queue.  C is the smallest chunk (in pages) with
+// H_kv * sum_i max(1, ceil(pages_i / C)) <= T, found by bisection over block
+// sums (the count only falls as C grows), or the longest row's page count
+// when whole rows already exceed T.
+__global__ void __launch_bounds__(kBuildThreads)
+    fill_queue_kernel(const int32_t *lens, int32_t B, int32_t H_kv, int32_t P, int32_t max_pages, int32_t T,
+                      int4 *items, int32_t capacity, int32_t *indptr, uint32_t *err)
+{
+    __shared__ int32_t pages[kBuildMaxRows];
+    // items of one head's rows before row i (the whole queue is bounded by the
+    // int32 capacity, so 32 bits hold it)
+    __shared__ int32_t row_start[kBuildMaxRows + 1];
+    __shared__ int64_t scan[kBuildThreads];
+    __shared__ int64_t total;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int tid = threadIdx.x;
+    const int64_t cap_tokens = (int64_t)max_pages * P;
+    auto clamped_len = [&](int i) {
+        int64_t N = lens[i];
+        if (N < 0 || N > cap_tokens) {
+            atomicOr(err, kErrSeqLen);
+            N = N < 0 ? 0 : cap_tokens;
+        }
+        return N;
+    };
+    int64_t pmax = 0;
+    for (int i = tid; i < B; i += kBuildThreads) {
+        pages[i] = (int32_t)((clamped_len(i) + P - 1) / P);
+        pmax = pmax > pages[i] ? pmax : pages[i];
+    }
+    // block max of the page counts (as a sum of per-thread maxima would not be)
+    scan[tid] = pmax;
+    __syncthreads();
+    for (int off = kBuildThreads / 2; off > 0; off >>= 1) {
+        if (tid < off)
+            scan[tid] = scan[tid] > scan[tid + off] ? scan[tid] : scan[tid + off];
+        __syncthreads();
+    }
+    const int64_t pages_max = scan[0] > 0 ? scan[0] : 1;
+    __syncthreads();
+    // items of one head at chunk size C, summed over the block
+    auto head_items = [&](int64_t C) {
+        int64_t n = 0;
+        for (int i = tid; i < B; i += kBuildThreads) {
+            const int64_t c = (pages[i] + C - 1) / C;
+            n += c > 1 ? c : 1;
+        }
+        scan[tid] = n;
+        __syncthreads();
+        for (int off = kBuildThreads / 2; off > 0; off >>= 1) {
+            if (tid < off)
+                scan[tid] += scan[tid + off];
+            __syncthreads();
+        }
+        const int64_t r = scan[0];
+        __syncthreads();
+        return r;
+    };
+    int64_t C = pages_max;
+    if (head_items(pages_max) * H_kv <= T) {
+        int64_t lo = 1, hi = pages_max;
+        while (lo < hi) {
+            const int64_t mid = lo + (hi - lo) / 2;
+            if (head_items(mid) * H_kv <= T)
+                hi = mid;
+            else
+                lo = mid + 1;
+        }
+        C = lo;
+    }
+    // row offsets of the items (one head), then every pair's items
+    int64_t carry = 0;
+    for (int base = 0; base < B; base += kBuildThreads) {
+        const int i = base + tid;
+        int64_t cnt = 0;
+        if (i < B) {
+            cnt = (pages[i] + C - 1) / C;
+            cnt = cnt > 1 ? cnt : 1;
+        }
+        const int64_t incl = block_inclusive_scan(cnt, scan);
+        if (i < B)
+            row_start[i] = (int32_t)(carry + incl - cnt);
+        if (tid == kBuildThreads - 1)
+            total = carry + incl;
+        __syncthreads();
+        carry = total;
+        __syncthreads();
+    }
+    if (tid == 0)
+        row_start[B] = (int32_t)carry;
+    __syncthreads();
+    const int64_t pairs = (int64_t)B * H_kv;
+    const int64_t span = C * P;
+    for (int64_t p = tid; p < pairs; p += kBuildThreads) {
+        const int i = (int)(p / H_kv), h = (int)(p % H_kv);
+        const int64_t cnt = (int64_t)row_start[i + 1] - row_start[i];
+        const int64_t o = (int64_t)row_start[i] * H_kv + h * cnt;
+        indptr[p] = (int32_t)o;
+        const int64_t N = pages[i] == 0 ? 0 : clamped_len(i);
+        for (int64_t c = 0; c < cnt; ++c) {
+            int4 it = make_int4(i, h, 0, 0);
+            if (N > 0) {
+                it.z = (int)(c * span);
+                it.w = (int)((c + 1) * span < N ? (c + 1) * span : N);
+            }
+            if (o + c < capacity)
+                items[o + c] = it;
+            else
+                atomicOr(err, kErrItem);
+        }
+    }
+    if (tid == 0)
+        indptr[pairs] = (int32_t)(carry * H_kv);
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 
@@ -2367,6 +2488,40 @@ int pkv_build_balanced_queue_device(const int32_t *seq_lens, const pkv_shape *sh
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, balanced_queue_kernel, seq_lens, s.B, s.H_kv, s.page_size,
+                                             s.max_pages_per_seq, n_blocks, reinterpret_cast<int4 *>(items),
+                                             capacity, indptr, static_cast<uint32_t *>(workspace));
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_build_fill_queue_device(const int32_t *seq_lens, const pkv_shape *shape, int32_t n_blocks,
+                                pkv_work_item *items, int32_t capacity, int32_t *indptr, void *workspace,
+                                void *stream)
+{
+    int32_t need = 0;
+    int rc = pkv_fill_queue_capacity(shape, n_blocks, &need);
+    if (rc != PKV_OK)
+        return rc;
+    const pkv_shape &s = *shape;
+    if (s.B == 0)
+        return PKV_OK;
+    if (s.B > kBuildMaxRows)
+        return PKV_ERR_UNSUPPORTED;
+    if (capacity < need)
+        return PKV_ERR_CAPACITY;
+    if (!seq_lens || !items || !indptr || !workspace)
+        return PKV_ERR_INVALID;
+    if (!aligned(items, 16) || !aligned(indptr, 4) || !aligned(seq_lens, 4) || !aligned(workspace, 256))
+        return PKV_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kBuildThreads);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fill_queue_kernel, seq_lens, s.B, s.H_kv, s.page_size,
                                              s.max_pages_per_seq, n_blocks, reinterpret_cast<int4 *>(items),
                                              capacity, indptr, static_cast<uint32_t *>(workspace));
     return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;

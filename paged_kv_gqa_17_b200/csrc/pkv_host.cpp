@@ -284,6 +284,18 @@ int pkv_balanced_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape
     return PKV_OK;
 }
 
+int pkv_fill_queue_capacity(const pkv_shape *shape, int32_t n_blocks, int32_t *capacity)
+{
+    if (!capacity || n_blocks < 1 || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    // at most T items, or one per (row, KV head) when whole rows exceed T
+    const int64_t c = std::max<int64_t>(n_blocks, (int64_t)shape->B * shape->H_kv);
+    if (c > INT32_MAX)
+        return PKV_ERR_CAPACITY;
+    *capacity = (int32_t)c;
+    return PKV_OK;
+}
+
 int pkv_balanced_queue_capacity(const pkv_shape *shape, int32_t n_blocks, int32_t *capacity)
 {
     if (!capacity || n_blocks < 1 || check_shape(shape) != PKV_OK)

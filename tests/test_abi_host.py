@@ -242,3 +242,10 @@ def test_device_queue_builder_host_checks(L):
     # an empty batch queues nothing
     empty = bd.make_shape(0, 8, 2, 128, 16, 8, 10)
     assert L.pkv_build_balanced_queue_device(None, ctypes.byref(empty), 37, None, 0, None, None, None) == 0
+    # the fill-one-wave builder: capacity max(T, B*H_kv), the same checks
+    assert L.pkv_fill_queue_capacity(ctypes.byref(shape), 5, ctypes.byref(cap)) == 0 and cap.value == 8
+    assert L.pkv_fill_queue_capacity(ctypes.byref(shape), 296, ctypes.byref(cap)) == 0 and cap.value == 296
+    assert L.pkv_build_fill_queue_device(None, ctypes.byref(shape), 296, None, 295, None, None, None) == -3
+    assert L.pkv_build_fill_queue_device(None, ctypes.byref(shape), 296, None, 296, None, None, None) == -1
+    assert L.pkv_build_fill_queue_device(None, ctypes.byref(big), 296, None, 1 << 20, None, None, None) == -2
+    assert L.pkv_build_fill_queue_device(None, ctypes.byref(empty), 296, None, 0, None, None, None) == 0

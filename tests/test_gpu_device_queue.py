@@ -1,7 +1,7 @@
-"""The balanced queue built on the GPU (pkv_build_balanced_queue_device):
-bit-identical to the host builder, decodes that match the oracle, and a
-decode step captured once in a CUDA graph that stays correct while the
-lengths change on the device between replays."""
+"""The queues built on the GPU (pkv_build_balanced_queue_device,
+pkv_build_fill_queue_device): bit-identical to the host builders, decodes
+that match the oracle, and decode steps captured once in a CUDA graph that
+stay correct while the lengths change on the device between replays."""
 import numpy as np
 import pytest
 import torch
@@ -12,6 +12,12 @@ from paged_kv_gqa_17_b200 import workloads as W
 from .gpu_util import assert_close, oracle_full, to_device
 
 pytestmark = pytest.mark.gpu
+
+ANY = (0, 2**31 - 1, 0, 2**31 - 1)
+
+
+def rule(mode, S=1, C=0, flags=0):
+    return bd.Rule(*ANY, mode, S, C, flags)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -116,3 +122,83 @@ def test_device_builder_flags_bad_lengths():
     # the clamped lengths (10, 64, 0) give the host builder's queue
     h_items, h_indptr = bd.build_balanced_queue([10, 64, 0], shape, 5)
     assert torch.equal(items.cpu()[:h_items.shape[0]], h_items) and torch.equal(indptr.cpu(), h_indptr)
+
+
+def _fill_queue(lens, shape, T):
+    cap = bd.fill_queue_capacity(shape, T)
+    items = torch.full((cap, 4), -7, dtype=torch.int32, device="cuda")
+    indptr = torch.full((shape.B * shape.H_kv + 1,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    bd.build_fill_queue_device(lens_d, shape, T, items, indptr, ws)
+    torch.cuda.synchronize()
+    return items.cpu(), indptr.cpu(), ws
+
+
+def test_fill_builder_matches_policy_and_host_queue_bit_exactly():
+    """The device's chunk is the host policy's fill chunk, and its queue is
+    pkv_build_work_queue's at that chunk."""
+    rng = np.random.default_rng(22)
+    cases = [([1], 1, 296), ([17, 0, 5], 4, 296), ([32768], 8, 296), ([16] * 5, 8, 7), ([5000, 0, 1, 16, 17], 2, 1),
+             ([12129, 621, 1118, 1452, 2891, 1419, 518, 3174], 8, 296), ([40000] * 64, 8, 296)]
+    for _ in range(40):
+        B = int(rng.integers(1, 70))
+        lens = [int(x) for x in rng.choice([0, 1, 15, 16, 17, 300, 5000, 40000], B)]
+        if max(lens) == 0:
+            lens[0] = 1
+        cases.append((lens, int(rng.choice([1, 2, 4, 8])), int(rng.choice([1, 3, 37, 148, 296, 444]))))
+    for lens, H_kv, T in cases:
+        max_pages = max(-(-n // 16) for n in lens)
+        shape = bd.make_shape(len(lens), 4 * H_kv, H_kv, 128, 16, max_pages, 10)
+        plan = bd.select_policy(lens, shape, [rule(2, T, 0, 0)])
+        h_items, h_indptr = bd.build_work_queue(lens, shape, plan.chunk_pages)
+        d_items, d_indptr, ws = _fill_queue(lens, shape, T)
+        n = h_items.shape[0]
+        assert torch.equal(d_items[:n], h_items), (lens, H_kv, T, plan.tuple())
+        assert torch.equal(d_indptr, h_indptr), (lens, H_kv, T)
+        assert (d_items[n:] == -7).all()
+        assert int(ws[:4].view(torch.int32)[0]) == 0
+
+
+@pytest.mark.parametrize("T,flags", [(37, 0), (296, 4), (5, 1)])
+def test_decode_with_device_fill_queue_matches_oracle(T, flags):
+    w = to_device(W.make_custom([3000, 77, 1999, 16, 0, 1], 32, 8, 128, seed=142, poison=True))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    plan = bd.select_policy(w.seq_lens, shape, [rule(2, T, 0, flags)])
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", plan=plan, device_queue=True, fill_blocks=T)
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
+    out = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp)
+    torch.cuda.synchronize()
+    assert bd.workspace_status(dp) == 0
+    assert_close(out.float().cpu().double().numpy(), oracle_full(w), f"device fill queue T={T}")
+    host = bd.plan_decode(w.seq_lens, shape, "cuda", plan=plan)
+    ref = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=host)
+    assert torch.equal(out, ref)  # same queue, same kernels: the same bits
+
+
+def test_graph_replay_of_the_fill_queue_follows_device_lengths():
+    full = [2500, 900, 40, 1300]
+    w = to_device(W.make_custom(full, 16, 4, 128, seed=143, poison=False))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    plan = bd.select_policy(full, shape, [rule(2, 148, 0, 4)])
+    dp = bd.plan_decode(full, shape, "cuda", plan=plan, device_queue=True, fill_blocks=148)
+    lens = torch.tensor(full, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(w.q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    cap = shape.max_pages_per_seq * 16
+    for step_lens in ([2500, 900, 40, 1300], [17, 0, 40, cap], [0, 0, 0, 0], [1, 2, 3, 4], [cap] * 4):
+        lens.copy_(torch.tensor(step_lens, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        assert bd.workspace_status(dp) == 0
+        w.seq_lens = list(step_lens)
+        assert_close(out.float().cpu().double().numpy(), oracle_full(w), f"fill replay {step_lens}")
+    del g

@@ -45,6 +45,9 @@ MODES = {
     "split3_cl": rule(1, 3, 0, 8),
     "split1_cl": rule(1, 1, 0, 8),
     "split12_cl_nopdl": rule(1, 12, 0, 10),
+    "wqfill37": rule(2, 37, 0, 0),          # queue whose chunk fills 37 blocks
+    "wqfill296_deep": rule(2, 296, 0, 4),   # ... one wave of 296, deep ring
+    "wqfill5_sep": rule(2, 5, 0, 1),        # tiny budget: whole rows, separate merge
 }
 
 
@@ -81,7 +84,8 @@ CASES = {
 @pytest.mark.parametrize("case", sorted(CASES))
 @pytest.mark.parametrize("mode", ["nosplit", "split7", "split32", "split32_sep", "wq3", "wq3_sep", "split32_deep",
                                   "wq3_deep_sep", "split7_nopdl", "bal1", "bal7", "bal296", "bal148_deep",
-                                  "bal64_sep", "split16_cl", "split8_cl_deep", "split3_cl", "split12_cl_nopdl"])
+                                  "bal64_sep", "split16_cl", "split8_cl_deep", "split3_cl", "split12_cl_nopdl",
+                                  "wqfill37", "wqfill296_deep", "wqfill5_sep"])
 def test_ragged_shapes(case, mode):
     lens, H_q, H_kv, D = CASES[case]
     w = to_device(W.make_custom(lens, H_q, H_kv, D, seed=101, poison=True, q_scale=3.0))
