@@ -995,10 +995,12 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     int e_first = 0;
     int row_len = -1;  // the row's length where known (for the early dependency gate)
     if (p.mode == PKV_WORK_QUEUE) {
-        // a queue built on the device may hold fewer items than the grid has blocks
-        if ((int)blockIdx.x >= __ldg(p.indptr + p.B * p.H_kv))
-            return;
+        // a queue built on the device may hold fewer items than the grid has
+        // blocks (the buffer holds one per block); both loads go out at once
+        const int n_real = __ldg(p.indptr + p.B * p.H_kv);
         const int4 it = __ldg(p.items + blockIdx.x);
+        if ((int)blockIdx.x >= n_real)
+            return;
         row = it.x;
         h = it.y;
         tb = it.z;
