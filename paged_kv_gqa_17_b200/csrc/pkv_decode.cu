@@ -438,7 +438,7 @@ struct Cfg {
     static constexpr int kCombineBytes = NW * kGP * (kOStride + 2) * 4;
     static constexpr int kRingBytes = 2 * NST * kStageBytes;
     static constexpr int kBarOff = ((kRingBytes > kCombineBytes ? kRingBytes : kCombineBytes) + 63) / 64 * 64;
-    static constexpr int kMiscOff = kBarOff + 2 * NST * 8;  // int flag, then two merge mbarriers at +8, +16
+    static constexpr int kMiscOff = kBarOff + 2 * NST * 8;  // int flag, merge mbarriers at +8, +16, a guessed item at +32
     static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + slack to align the base to 1024
     static constexpr int kMaxMergeTasks = (kGP * (D / 4) + kThreads - 1) / kThreads;
     // cluster merge: this block's final state [m: 16][l: 16][acc: kGP][D] in the idle ring
@@ -894,8 +894,15 @@ __device__ void merge_pair_last_block(const Params &p, uint8_t *smem, uint32_t m
 // uses is read again after the wait, and L2 is coherent with the writes of
 // the kernel before.  In a back-to-back decode loop this streams the first
 // pages while the previous step finishes its merges.
+// In the work-queue grid the producer also hands the speculatively read
+// item to the block (*spec, set when it is a well-formed item): after the
+// wait the block then issues the loads that depend on the item (the pair's
+// slot range, the first block-table entries) at the addresses the guess
+// gives, together with the item itself, and keeps them only if the item
+// read after the wait equals the guess.  Every value used is read after the
+// wait; the guess only saves one round trip to L2 when it is right.
 template <int D>
-__device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lane, int64_t row_cap)
+__device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lane, int64_t row_cap, int4 *spec)
 {
 #if PKV_L2_PREFETCH_PAGES > 0
     int row, h;
@@ -904,6 +911,8 @@ __device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lan
         const int4 it = ld_l2_only(p.items + blockIdx.x);
         if (!(it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w && it.w <= row_cap))
             return;
+        if (lane == 0)
+            *spec = it;
         row = it.x;
         h = it.y;
         pg0 = it.z / kPage;
@@ -981,9 +990,15 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     // promises that kernel writes neither the lengths, the table, the queue
     // nor any KV page but a row's last, so those are read first and the wait
     // comes before q, the last page and any global write.
+    // guessed work item (row = -1: none), see l2_prefetch_first_pages
+    int4 *spec_item = reinterpret_cast<int4 *>(smem + C::kMiscOff + 32);
+    if (tid == 0)
+        *spec_item = make_int4(-1, 0, 0, 0);
     if (!p.pdl_early) {
+        __syncthreads();
         if (warp == NW && (int)blockIdx.x < p.prefetch_blocks)
-            l2_prefetch_first_pages<D>(p, lane, row_cap);
+            l2_prefetch_first_pages<D>(p, lane, row_cap, spec_item);
+        __syncthreads();
         grid_dependency_wait();
     }
 
@@ -993,14 +1008,27 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     // no-split and split-S grids is before the row length arrives.
     int row, h, tb, te, slot0 = 0, nslots = 1, my_slot = 0;
     int e_first = 0;
+    bool hit = false;  // the guessed work item was the real one
     int row_len = -1;  // the row's length where known (for the early dependency gate)
     if (p.mode == PKV_WORK_QUEUE) {
         // a queue built on the device may hold fewer items than the grid has
-        // blocks (the buffer holds one per block); both loads go out at once
+        // blocks (the buffer holds one per block); the item, the item count
+        // and the loads at the guessed item's addresses go out at once
+        const int4 guess = p.pdl_early ? make_int4(-1, 0, 0, 0) : *spec_item;  // written before the last barrier
         const int n_real = __ldg(p.indptr + p.B * p.H_kv);
         const int4 it = __ldg(p.items + blockIdx.x);
+        int g_slot0 = 0, g_slot1 = 0, g_entry = 0;
+        if (guess.x >= 0) {
+            const int gpair = guess.x * p.H_kv + guess.y;
+            g_slot0 = __ldg(p.indptr + gpair);
+            g_slot1 = __ldg(p.indptr + gpair + 1);
+            const int idx = guess.z / kPage + lane;
+            if (warp == NW && idx < p.max_pages)
+                g_entry = __ldg(p.block_table + (int64_t)guess.x * p.max_pages + idx);
+        }
         if ((int)blockIdx.x >= n_real)
             return;
+        hit = guess.x >= 0 && guess.x == it.x && guess.y == it.y && guess.z == it.z && guess.w == it.w;
         row = it.x;
         h = it.y;
         tb = it.z;
@@ -1009,8 +1037,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
                   (tb % kPage) == 0;
         if (ok) {
             const int pair = row * p.H_kv + h;
-            slot0 = __ldg(p.indptr + pair);
-            nslots = __ldg(p.indptr + pair + 1) - slot0;
+            slot0 = hit ? g_slot0 : __ldg(p.indptr + pair);
+            nslots = (hit ? g_slot1 : __ldg(p.indptr + pair + 1)) - slot0;
+            e_first = g_entry;
             my_slot = blockIdx.x;
             ok = nslots >= 1 && slot0 >= 0 && my_slot >= slot0 && my_slot < slot0 + nslots &&
                  slot0 + nslots <= p.n_items;
@@ -1022,7 +1051,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         }
         if (warp == NW) {
             const int idx = tb / kPage + lane;
-            if (idx < p.max_pages)
+            if (!hit && idx < p.max_pages)
                 e_first = __ldg(p.block_table + (int64_t)row * p.max_pages + idx);
             if (p.pdl_early)
                 row_len = __ldg(p.seq_lens + row);
