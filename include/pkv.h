@@ -19,8 +19,11 @@
  * Conventions for every function:
  *  - The return value is a pkv_status; nothing else reports errors.
  *  - Device memory is allocated by the caller (e.g. PyTorch) and owned by the
- *    caller; the library allocates no device memory and keeps no pointer
- *    after a call returns.  Host functions are pure and thread-safe.
+ *    caller; the library allocates no device memory at run time (the scratch
+ *    of pkv_paged_decode_noalloc is a fixed array in the library image) and
+ *    touches no caller buffer after a call returns (a small host-side cache
+ *    of encoded TMA descriptors is keyed by pool address and shape).  Host
+ *    functions are pure and thread-safe.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Device work is queued on it asynchronously unless stated.
  *  - Sizes are element counts unless the name ends in _bytes.

@@ -3,9 +3,11 @@
 Single-token decode attention read straight through a paged KV cache's block
 table, where G = H_q / H_kv query heads share each KV head: a split-S kernel
 whose chunks produce partial softmax states, an exact merge, a compact work
-queue and a calibrated policy that picks no-split, split-S or work-queue per
-batch.  Every step runs in the C-ABI library `libpkv.so` (CUDA for sm_100a plus
-host C++); this package only marshals arguments to it.
+queue (with a chunk that can fill one wave of the GPU, and a balanced cut for
+a persistent grid, both also buildable on the device) and a calibrated policy
+that picks the plan per batch.  Every step runs in the C-ABI library
+`libpkv.so` (CUDA for sm_100a plus host C++); this package only marshals
+arguments to it.
 
 The CUDA library is loaded on first use of anything but `workloads`; if it is
 missing or cannot find a GPU, the call raises instead of falling back.
