@@ -15,7 +15,7 @@ on a holdout seed].  This script does the same by measurement:
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
      the work queue over seven chunk sizes, with and without the deep ring,
-     and with the chunk size that fills one wave of 296 or 444 blocks; the
+     and with the chunk size that fills one wave of 222 to 444 blocks; the
      balanced grid at one and two blocks per SM) as the steady-state device
      time of back-to-back steps over rotating pool copies.
   3. The plan with the smallest geometric-mean time over the cell's batches
@@ -57,7 +57,9 @@ def candidates():
         out.append((1, S, 0, 12))  # cluster merge, deep ring
     for C in (8, 16, 24, 32, 48, 64, 96):
         out += [(2, 1, C, 0), (2, 1, C, 4)]
-    out += [(2, 296, 0, 4), (2, 296, 0, 0), (2, 444, 0, 0)]  # C chosen to fill one wave of T blocks
+    # C chosen to fill one wave of T blocks: about 1.5, 1.8 and 2 blocks per SM with
+    # the deep ring (two fit per SM), 2 and 3 per SM with the 8-page ring
+    out += [(2, 222, 0, 4), (2, 264, 0, 4), (2, 296, 0, 4), (2, 296, 0, 0), (2, 444, 0, 0)]
     out += [(3, 296, 0, 0), (3, 148, 0, 4)]
     return out
 
