@@ -1770,7 +1770,8 @@ __global__ void wait_timeout_selftest_kernel(uint32_t *err, uint64_t limit_ns)
 // One block of threads: the row page counts and the per-pair item counts are
 // each prefix-summed over the block, and each thread emits its pair's items.
 
-constexpr int kBuildThreads = 1024;
+constexpr int kBuildThreads = 256;
+constexpr int kBuildWarps = kBuildThreads / 32;
 constexpr int kBuildMaxRows = 4096;
 
 __device__ __forceinline__ int64_t share_start(int64_t U, int64_t T, int64_t b) { return (b * U) / T; }
@@ -1785,19 +1786,56 @@ __device__ __forceinline__ int64_t share_owner(int64_t U, int64_t T, int64_t u)
     return b < T - 1 ? b : T - 1;
 }
 
-// Inclusive prefix sum of v over the block (all threads call it).
+// Block-wide primitives of the queue builders (all threads call them):
+// shuffles inside each warp, one shared-memory pass over the warps' values,
+// two barriers in all.  `scan` holds kBuildWarps values.
 __device__ int64_t block_inclusive_scan(int64_t v, int64_t *scan)
 {
-    const int tid = threadIdx.x;
-    scan[tid] = v;
-    __syncthreads();
-    for (int off = 1; off < kBuildThreads; off <<= 1) {
-        const int64_t add = tid >= off ? scan[tid - off] : 0;
-        __syncthreads();
-        scan[tid] += add;
-        __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int64_t add = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off)
+            v += add;
     }
-    const int64_t r = scan[tid];
+    if (lane == 31)
+        scan[warp] = v;
+    __syncthreads();
+    int64_t before = 0;
+    for (int w = 0; w < warp; ++w)
+        before += scan[w];
+    __syncthreads();  // scan[] is free again
+    return v + before;
+}
+
+__device__ int64_t block_sum(int64_t v, int64_t *scan)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0)
+        scan[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int64_t r = 0;
+    for (int w = 0; w < kBuildWarps; ++w)
+        r += scan[w];
+    __syncthreads();
+    return r;
+}
+
+__device__ int64_t block_max(int64_t v, int64_t *scan)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const int64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = o > v ? o : v;
+    }
+    if ((threadIdx.x & 31) == 0)
+        scan[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int64_t r = scan[0];
+    for (int w = 1; w < kBuildWarps; ++w)
+        r = scan[w] > r ? scan[w] : r;
     __syncthreads();
     return r;
 }
@@ -1807,7 +1845,7 @@ __global__ void __launch_bounds__(kBuildThreads)
                           int4 *items, int32_t capacity, int32_t *indptr, uint32_t *err)
 {
     __shared__ int64_t row_start[kBuildMaxRows + 1];  // pages of one head's rows before row i
-    __shared__ int64_t scan[kBuildThreads];
+    __shared__ int64_t scan[kBuildWarps];
     __shared__ int64_t total;
     grid_dependency_wait();     // the lengths may come from the kernel before
     grid_launch_dependents();  // the decode kernel may start its set-up
@@ -1916,7 +1954,7 @@ __global__ void __launch_bounds__(kBuildThreads)
     // items of one head's rows before row i (the whole queue is bounded by the
     // int32 capacity, so 32 bits hold it)
     __shared__ int32_t row_start[kBuildMaxRows + 1];
-    __shared__ int64_t scan[kBuildThreads];
+    __shared__ int64_t scan[kBuildWarps];
     __shared__ int64_t total;
     grid_dependency_wait();
     grid_launch_dependents();
@@ -1935,16 +1973,9 @@ __global__ void __launch_bounds__(kBuildThreads)
         pages[i] = (int32_t)((clamped_len(i) + P - 1) / P);
         pmax = pmax > pages[i] ? pmax : pages[i];
     }
-    // block max of the page counts (as a sum of per-thread maxima would not be)
-    scan[tid] = pmax;
-    __syncthreads();
-    for (int off = kBuildThreads / 2; off > 0; off >>= 1) {
-        if (tid < off)
-            scan[tid] = scan[tid] > scan[tid + off] ? scan[tid] : scan[tid + off];
-        __syncthreads();
-    }
-    const int64_t pages_max = scan[0] > 0 ? scan[0] : 1;
-    __syncthreads();
+    __syncthreads();  // pages[] complete
+    int64_t pages_max = block_max(pmax, scan);
+    pages_max = pages_max > 0 ? pages_max : 1;
     // items of one head at chunk size C, summed over the block
     auto head_items = [&](int64_t C) {
         int64_t n = 0;
@@ -1952,16 +1983,7 @@ __global__ void __launch_bounds__(kBuildThreads)
             const int64_t c = (pages[i] + C - 1) / C;
             n += c > 1 ? c : 1;
         }
-        scan[tid] = n;
-        __syncthreads();
-        for (int off = kBuildThreads / 2; off > 0; off >>= 1) {
-            if (tid < off)
-                scan[tid] += scan[tid + off];
-            __syncthreads();
-        }
-        const int64_t r = scan[0];
-        __syncthreads();
-        return r;
+        return block_sum(n, scan);
     };
     int64_t C = pages_max;
     if (head_items(pages_max) * H_kv <= T) {
