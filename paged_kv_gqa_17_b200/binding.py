@@ -310,19 +310,20 @@ def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[
     lengths by every paged_decode call (so one plan, or one captured CUDA
     graph, serves any lengths up to the shape's maximum): a BALANCED plan
     gets the balanced queue of its T blocks, a WORK_QUEUE plan the queue
-    whose chunk fills one wave of `fill_blocks` blocks."""
+    whose chunk fills one wave of `fill_blocks` blocks.  NO_SPLIT and
+    SPLIT_S plans have no queue and read the lengths on the device anyway;
+    they serve lengths up to those they were planned for (SPLIT_S: S' chunks
+    of C pages)."""
     if plan is None:
         plan = select_policy(seq_lens_host, shape, rules)
-    if device_queue:
+    if device_queue and plan.mode in (WORK_QUEUE, BALANCED):
         pairs = shape.B * shape.H_kv
         if plan.mode == BALANCED:
             cap = balanced_queue_capacity(shape, plan.num_splits)
             n_ptr = pairs + 1 + plan.num_splits + 1
-        elif plan.mode == WORK_QUEUE:
+        else:
             cap = fill_queue_capacity(shape, fill_blocks)
             n_ptr = pairs + 1
-        else:
-            raise PkvError(-1, "device_queue needs a BALANCED or WORK_QUEUE plan")
         items = torch.zeros((cap, 4), dtype=torch.int32, device=device)
         indptr = torch.zeros(n_ptr, dtype=torch.int32, device=device)
         ws = torch.zeros(workspace_bytes(shape, plan, cap), dtype=torch.uint8, device=device)
