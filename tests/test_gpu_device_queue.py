@@ -202,3 +202,33 @@ def test_graph_replay_of_the_fill_queue_follows_device_lengths():
         w.seq_lens = list(step_lens)
         assert_close(out.float().cpu().double().numpy(), oracle_full(w), f"fill replay {step_lens}")
     del g
+
+
+def test_device_queue_request_passes_queue_free_plans_through():
+    """device_queue=True with a split-S plan needs no queue: the plan reads the
+    lengths on the device, so a captured step serves any lengths up to those
+    it was planned for."""
+    full = [2000, 700, 1500]
+    w = to_device(W.make_custom(full, 16, 4, 128, seed=144, poison=False))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dp = bd.plan_decode(full, shape, "cuda", rules=[rule(1, 8, 0, 4)], device_queue=True)
+    assert dp.plan.mode == bd.SPLIT_S and not dp.device_queue and dp.items is None
+    lens = torch.tensor(full, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(w.q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp, out=out)
+    for step_lens in ([2000, 700, 1500], [1999, 0, 2000], [5, 6, 7]):
+        lens.copy_(torch.tensor(step_lens, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        assert bd.workspace_status(dp) == 0
+        w.seq_lens = list(step_lens)
+        assert_close(out.float().cpu().double().numpy(), oracle_full(w), f"split-S replay {step_lens}")
+    del g
