@@ -48,3 +48,18 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["steps"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["unit"] == d["unit"]
+
+
+def test_recorded_traffic_follows_the_kernel_source_hash(monkeypatch):
+    """The roofline's traffic figure is reported only for the kernel sources
+    it was captured on."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    assert rows, "profiles/traffic.txt lists no capture"
+    name, digest, nbytes = rows[0]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: digest)
+    assert bench.recorded_traffic(name) == int(nbytes)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.recorded_traffic(name) is None
+    assert bench.recorded_traffic("no-such-workload") is None
+
