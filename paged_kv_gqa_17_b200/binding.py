@@ -147,14 +147,71 @@ def make_shape(B: int, H_q: int, H_kv: int, head_dim: int, page_size: int, max_p
     return Shape(B, H_q, H_kv, D, P, max_pages, num_pool_pages, 0, *strides)
 
 
-def shape_of(q: torch.Tensor, k_pool: torch.Tensor, block_table: torch.Tensor, layout: str = "HND") -> Shape:
-    """Shape of a decode step from q [B][H_q][D], a pool and block_table [B][max_pages]."""
+def shape_of(q: torch.Tensor, k_pool: torch.Tensor, block_table: torch.Tensor, layout: str = "HND",
+             v_pool: Optional[torch.Tensor] = None) -> Shape:
+    """Shape of a decode step from q [B][H_q][D], a pool and block_table [B][max_pages].
+
+    The pool strides are the tensor's own (in elements), so a pool that is a
+    view into a larger cache needs no copy: K and V halves of one combined
+    cache ([pages][2][H_kv][P][D] gives k = kv[:, 0], v = kv[:, 1]), or pages
+    padded past their last row.  The head_dim axis must be contiguous; with
+    `v_pool`, its shape and strides must equal k_pool's (one set of strides
+    serves both pools).  Axes of extent 1 take the packed stride, which is
+    never used to address an element."""
+    if k_pool.dim() != 4:
+        raise ValueError(f"k_pool must be 4-D, got shape {tuple(k_pool.shape)}")
+    if v_pool is not None and (tuple(v_pool.shape) != tuple(k_pool.shape) or v_pool.stride() != k_pool.stride()):
+        raise ValueError("k_pool and v_pool must have the same shape and strides")
     B, H_q, D = (int(x) for x in q.shape)
     if layout == "HND":
-        pages, H_kv, P, _ = (int(x) for x in k_pool.shape)
+        (pages, H_kv, P, _), (sp, sh, st, sd) = k_pool.shape, k_pool.stride()
+    elif layout == "NHD":
+        (pages, P, H_kv, _), (sp, st, sh, sd) = k_pool.shape, k_pool.stride()
     else:
-        pages, P, H_kv, _ = (int(x) for x in k_pool.shape)
-    return make_shape(B, H_q, H_kv, D, P, int(block_table.shape[1]), pages, layout)
+        raise ValueError(layout)
+    if sd != 1 and D > 1:
+        raise ValueError("the pool's head_dim axis must be contiguous (stride 1)")
+    s = make_shape(B, H_q, int(H_kv), D, int(P), int(block_table.shape[1]), int(pages), layout)
+    if pages > 1:
+        s.kv_stride_page = sp
+    if H_kv > 1:
+        s.kv_stride_head = sh
+    if P > 1:
+        s.kv_stride_token = st
+    return s
+
+
+def _check_decode_tensors(q, k_pool, v_pool, block_table, seq_lens, out, shape: Shape):
+    """Reject tensors whose type, layout or device differs from what the
+    pointers passed to the library are taken to address."""
+    for name, t, dt in (("q", q, torch.bfloat16), ("out", out, torch.bfloat16), ("k_pool", k_pool, torch.bfloat16),
+                        ("v_pool", v_pool, torch.bfloat16), ("block_table", block_table, torch.int32),
+                        ("seq_lens", seq_lens, torch.int32)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+    for name, t in (("q", q), ("out", out), ("block_table", block_table), ("seq_lens", seq_lens)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    want = (shape.B, shape.H_q, shape.head_dim)
+    if tuple(q.shape) != want or tuple(out.shape) != want:
+        raise ValueError(f"q and out must be {list(want)}, got {list(q.shape)} and {list(out.shape)}")
+    if tuple(block_table.shape) != (shape.B, shape.max_pages_per_seq):
+        raise ValueError(f"block_table must be [{shape.B}][{shape.max_pages_per_seq}], got {list(block_table.shape)}")
+    if seq_lens.numel() < shape.B:
+        raise ValueError(f"seq_lens holds {seq_lens.numel()} lengths for {shape.B} rows")
+    if k_pool.dim() != 4 or tuple(v_pool.shape) != tuple(k_pool.shape) or v_pool.stride() != k_pool.stride():
+        raise ValueError("k_pool and v_pool must be 4-D with the same shape and strides")
+    if k_pool.shape[0] < shape.num_pool_pages or (k_pool.shape[0] > 1 and k_pool.stride(0) != shape.kv_stride_page):
+        raise ValueError("the pools' pages differ from the plan's shape (page count or page stride)")
+    if k_pool.stride(-1) != 1 and shape.head_dim > 1:
+        raise ValueError("the pools' head_dim axis must be contiguous (stride 1)")
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError(f"q must be on a CUDA device, not {dev}")
+    for name, t in (("out", out), ("k_pool", k_pool), ("v_pool", v_pool), ("block_table", block_table),
+                    ("seq_lens", seq_lens)):
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, q on {dev}")
 
 
 def rules_array(rules: Optional[Sequence]) -> tuple:
@@ -350,18 +407,21 @@ def paged_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, bl
     """out = softmax(scale * q K^T) V per (row, query head), read through the block table.
 
     q bf16 [B][H_q][D]; pools bf16 (layout "HND" [pages][H_kv][P][D] or "NHD"
-    [pages][P][H_kv][D]); block_table int32 [B][max_pages]; seq_lens int32 [B],
-    all on one CUDA device.  Without `plan`, the policy and queue are built from
-    `seq_lens_host` (or a host copy of seq_lens).
+    [pages][P][H_kv][D], any strides with a contiguous head_dim axis, see
+    shape_of); block_table int32 [B][max_pages]; seq_lens int32 [B], all on one
+    CUDA device.  Without `plan`, the policy and queue are built from
+    `seq_lens_host` (or a host copy of seq_lens).  Tensors of another dtype,
+    device or layout raise TypeError / ValueError before anything is launched.
     """
     L = lib()
     if plan is None:
-        shape = shape_of(q, k_pool, block_table, layout)
+        shape = shape_of(q, k_pool, block_table, layout, v_pool)
         host = seq_lens_host if seq_lens_host is not None else seq_lens.detach().cpu()
         plan = plan_decode(host, shape, q.device, rules)
     shape = plan.shape
     if out is None:
         out = torch.empty_like(q)
+    _check_decode_tensors(q, k_pool, v_pool, block_table, seq_lens, out, shape)
     if plan.device_queue and plan.plan.mode == BALANCED:
         build_balanced_queue_device(seq_lens, shape, plan.plan.num_splits, plan.items, plan.indptr, plan.workspace,
                                     stream)
@@ -385,6 +445,7 @@ def paged_decode_noalloc(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Te
     L = lib()
     if out is None:
         out = torch.empty_like(q)
+    _check_decode_tensors(q, k_pool, v_pool, block_table, seq_lens, out, plan.shape)
     rc = L.pkv_paged_decode_noalloc(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
                                     seq_lens.data_ptr(), page_size, float(scale), out.data_ptr(),
                                     ctypes.byref(plan.shape), ctypes.byref(plan.plan),
