@@ -93,7 +93,11 @@ typedef enum {
  * k_pool / v_pool lives at  page*kv_stride_page + kv_head*kv_stride_head +
  * slot*kv_stride_token + d  (elements).  The default "HND" pool
  * [num_pool_pages][H_kv][page_size][head_dim] has strides
- * (H_kv*P*D, P*D, D); an "NHD" pool [pages][P][H_kv][D] has (P*H_kv*D, D, H_kv*D). */
+ * (H_kv*P*D, P*D, D); an "NHD" pool [pages][P][H_kv][D] has (P*H_kv*D, D, H_kv*D).
+ * K and V share these strides, and either pool may be a view into a larger
+ * cache: the halves of one combined [pages][2][H_kv][P][D] cache (page stride
+ * 2*H_kv*P*D, V at K + H_kv*P*D elements), rows padded past D, pages holding
+ * more heads.  Nothing outside the addressed elements is read. */
 typedef struct {
     int32_t B;                  /* rows (sequences) in the batch, >= 0 */
     int32_t H_q;                /* query heads, a multiple of H_kv */
