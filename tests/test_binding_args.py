@@ -122,3 +122,37 @@ def test_paged_decode_rejects_a_mismatched_out(L):
         _decode(a, plan, out=torch.zeros(2, 8, 32, dtype=BF16))
     with pytest.raises(TypeError):
         _decode(a, plan, out=torch.zeros(2, 8, 64, dtype=torch.float32))
+
+
+def test_combined_check_passes_exactly_the_calls_the_itemised_checks_pass(L, monkeypatch):
+    """The one-expression test that passes well-formed calls and the itemised
+    checks that name a problem agree: with every tensor taken to be on device
+    0, the valid call passes the combined test, and each malformed one fails it
+    and gets a specific error from the itemised checks."""
+    monkeypatch.setattr(torch.Tensor, "get_device", lambda self: 0)
+    a = _args()
+    plan = _plan(a)
+    out = torch.zeros(2, 8, 64, dtype=BF16)
+    assert bd._check_decode_tensors(a["q"], a["k_pool"], a["v_pool"], a["block_table"], a["seq_lens"], out,
+                                    plan.shape) is None
+    bad_cases = [
+        dict(q=torch.zeros(2, 8, 64, dtype=torch.float16)),
+        dict(seq_lens=torch.zeros(2, dtype=torch.int64)),
+        dict(q=torch.zeros(8, 2, 64, dtype=BF16).transpose(0, 1)),
+        dict(block_table=torch.zeros(2, 5, dtype=torch.int32)),
+        dict(seq_lens=torch.zeros(1, dtype=torch.int32)),
+        dict(v_pool=torch.zeros(10, 2, 16, 72, dtype=BF16)[..., :64]),
+        dict(k_pool=torch.zeros(9, 2, 16, 64, dtype=BF16), v_pool=torch.zeros(9, 2, 16, 64, dtype=BF16)),
+        dict(k_pool=torch.zeros(10, 3, 16, 64, dtype=BF16)[:, :2], v_pool=torch.zeros(10, 3, 16, 64, dtype=BF16)[:, :2]),
+        dict(k_pool=torch.zeros(10, 2, 64, 16, dtype=BF16).transpose(2, 3),
+             v_pool=torch.zeros(10, 2, 64, 16, dtype=BF16).transpose(2, 3)),
+        dict(k_pool=torch.zeros(10, 2, 16, 64, dtype=BF16)[0], v_pool=torch.zeros(10, 2, 16, 64, dtype=BF16)[0]),
+    ]
+    for bad in bad_cases:
+        b = dict(a, **bad)
+        args = (b["q"], b["k_pool"], b["v_pool"], b["block_table"], b["seq_lens"], out, plan.shape)
+        with pytest.raises((TypeError, ValueError)) as e:
+            bd._diagnose_decode_tensors(*args)
+        assert "CUDA device" not in str(e.value), (bad, e.value)   # named before the device check
+        with pytest.raises((TypeError, ValueError)):
+            bd._check_decode_tensors(*args)
