@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import json
 import os
+import weakref
 from dataclasses import dataclass
 from typing import List, Optional, Sequence
 
@@ -236,6 +237,38 @@ def _diagnose_decode_tensors(q, k_pool, v_pool, block_table, seq_lens, out, shap
                     ("seq_lens", seq_lens)):
         if t.device != dev:
             raise ValueError(f"{name} is on {t.device}, q on {dev}")
+
+
+def _check_host_call(q_host, block_table_host, seq_lens_host, out_host, k_pool, v_pool, shape: Shape,
+                     device_index: int):
+    """The tensors of a pkv_decode_host call: host q / out (bf16 [B][H_q][D]),
+    host table (int32 [B][max_pages]) and lengths (int32, >= B), contiguous;
+    pools on the decoder's CUDA device with the shape's page count and strides."""
+    n_q = shape.B * shape.H_q * shape.head_dim
+    for name, t, dt, n in (("q_host", q_host, torch.bfloat16, n_q), ("out_host", out_host, torch.bfloat16, n_q),
+                           ("block_table_host", block_table_host, torch.int32, shape.B * shape.max_pages_per_seq),
+                           ("seq_lens_host", seq_lens_host, torch.int32, None)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+        if t.device.type != "cpu":
+            raise ValueError(f"{name} must be a host tensor, not on {t.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if n is not None and t.numel() != n:
+            raise ValueError(f"{name} holds {t.numel()} elements, the shape needs {n}")
+    if seq_lens_host.numel() < shape.B:
+        raise ValueError(f"seq_lens_host holds {seq_lens_host.numel()} lengths for {shape.B} rows")
+    for name, t in (("k_pool", k_pool), ("v_pool", v_pool)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be torch.bfloat16, got {t.dtype}")
+        if t.get_device() != device_index:
+            raise ValueError(f"{name} must be on the decoder's device cuda:{device_index}")
+    if k_pool.dim() != 4 or tuple(v_pool.shape) != tuple(k_pool.shape) or v_pool.stride() != k_pool.stride():
+        raise ValueError("k_pool and v_pool must be 4-D with the same shape and strides")
+    if k_pool.shape[0] < shape.num_pool_pages or (k_pool.shape[0] > 1 and k_pool.stride(0) != shape.kv_stride_page):
+        raise ValueError("the pools' pages differ from the shape (page count or page stride)")
+    if k_pool.stride(-1) != 1 and shape.head_dim > 1:
+        raise ValueError("the pools' head_dim axis must be contiguous (stride 1)")
 
 
 def rules_array(rules: Optional[Sequence]) -> tuple:
@@ -492,8 +525,10 @@ class HostDecoder:
     """Caller-owned buffers for pkv_decode_host, grown on demand: one device
     buffer (torch) and one page-locked host staging buffer.  Calls run on
     `stream` (default: the device's current stream when the decoder is made)
-    unless a call passes its own; the per-call Python work is kept to the
-    argument pointers, since a serving loop calls this once per step."""
+    unless a call passes its own.  The tensors of a call are checked (dtype,
+    size, contiguity, pool strides and device) when a tensor object or shape
+    is first seen; a serving loop that reuses its buffers pays only identity
+    comparisons per step.  Checked tensors must not be resized in place."""
 
     def __init__(self, device, stream=None):
         self.device = torch.device(device)
@@ -504,6 +539,7 @@ class HostDecoder:
         self._plan = Plan()
         self._plan_ref = ctypes.byref(self._plan)
         self._bufs = (0, 0, 0, 0)
+        self._checked = ()  # weak references to the tensors (and the shape) of the last checked call
 
     def ensure(self, seq_lens_host, shape: Shape, rules=None):
         L = lib()
@@ -521,6 +557,14 @@ class HostDecoder:
     def __call__(self, q_host: torch.Tensor, block_table_host: torch.Tensor, seq_lens_host: torch.Tensor,
                  out_host: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, scale: float, shape: Shape,
                  rules=None, stream=None) -> Plan:
+        seen = self._checked
+        if not (seen and seen[6] is shape and seen[0]() is q_host and seen[1]() is block_table_host
+                and seen[2]() is seq_lens_host and seen[3]() is out_host and seen[4]() is k_pool
+                and seen[5]() is v_pool):
+            _check_host_call(q_host, block_table_host, seq_lens_host, out_host, k_pool, v_pool, shape,
+                             self.dev.get_device())
+            self._checked = tuple(weakref.ref(t) for t in (q_host, block_table_host, seq_lens_host, out_host,
+                                                            k_pool, v_pool)) + (shape,)
         arr, n = rules_array(rules) if rules is not None else (None, 0)
         dev, dev_n, host, host_n = self._bufs
         rc = self._fn(q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(), out_host.data_ptr(),

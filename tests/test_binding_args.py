@@ -1,6 +1,8 @@
 """The binding's argument marshalling on the CPU: pool strides read from the
 tensors (views into combined or padded caches), and tensors of the wrong
 type, layout or device rejected before anything reaches the library."""
+import ctypes
+
 import pytest
 import torch
 
@@ -156,3 +158,69 @@ def test_combined_check_passes_exactly_the_calls_the_itemised_checks_pass(L, mon
         assert "CUDA device" not in str(e.value), (bad, e.value)   # named before the device check
         with pytest.raises((TypeError, ValueError)):
             bd._check_decode_tensors(*args)
+
+
+def _host_args(B=2, H_q=8, H_kv=2, D=64, pages=10, max_pages=4):
+    a = _args(B, H_q, H_kv, D, pages, max_pages)
+    shape = bd.shape_of(a["q"], a["k_pool"], a["block_table"])
+    return dict(q_host=a["q"], block_table_host=a["block_table"], seq_lens_host=a["seq_lens"],
+                out_host=torch.zeros_like(a["q"]), k_pool=a["k_pool"], v_pool=a["v_pool"]), shape
+
+
+@pytest.mark.parametrize("bad, exc", [
+    (dict(q_host=torch.zeros(2, 8, 64, dtype=torch.float16)), TypeError),
+    (dict(q_host=torch.zeros(2, 8, 32, dtype=BF16)), ValueError),                 # too small: would overrun
+    (dict(out_host=torch.zeros(1, 8, 64, dtype=BF16)), ValueError),
+    (dict(out_host=torch.zeros(8, 2, 64, dtype=BF16).transpose(0, 1)), ValueError),
+    (dict(block_table_host=torch.zeros(2, 3, dtype=torch.int32)), ValueError),
+    (dict(block_table_host=torch.zeros(2, 4, dtype=torch.int64)), TypeError),
+    (dict(seq_lens_host=torch.zeros(1, dtype=torch.int32)), ValueError),
+    (dict(k_pool=torch.zeros(9, 2, 16, 64, dtype=BF16), v_pool=torch.zeros(9, 2, 16, 64, dtype=BF16)), ValueError),
+    (dict(v_pool=torch.zeros(10, 2, 16, 64, dtype=torch.float32)), TypeError),
+])
+def test_host_call_checks_name_each_problem(monkeypatch, bad, exc):
+    monkeypatch.setattr(torch.Tensor, "get_device", lambda self: 0)   # pools "on" cuda:0
+    a, shape = _host_args()
+    bd._check_host_call(**a, shape=shape, device_index=0)             # the well-formed call passes
+    a.update(bad)
+    with pytest.raises(exc):
+        bd._check_host_call(**a, shape=shape, device_index=0)
+
+
+def test_host_call_rejects_pools_off_the_decoders_device():
+    a, shape = _host_args()                                           # CPU pools: get_device() == -1
+    with pytest.raises(ValueError):
+        bd._check_host_call(**a, shape=shape, device_index=0)
+
+
+def test_host_decoder_checks_each_new_tensor_object_once(monkeypatch):
+    """A HostDecoder checks a call's tensors when it first sees them; repeated
+    calls with the same objects skip straight to the library, and a new object
+    (or shape) is checked again before the library is reached."""
+    monkeypatch.setattr(torch.Tensor, "get_device", lambda self: 0)
+    checks, calls = [], []
+    real = bd._check_host_call
+    monkeypatch.setattr(bd, "_check_host_call", lambda *x, **k: (checks.append(1), real(*x, **k)))
+    dec = object.__new__(bd.HostDecoder)                              # no CUDA here: set the fields by hand
+    dec.dev = torch.zeros(1, dtype=torch.uint8)
+    dec._stream, dec._bufs, dec._checked = 0, (0, 0, 0, 0), ()
+    dec._plan = bd.Plan()
+    dec._plan_ref = ctypes.byref(dec._plan)
+    dec._fn = lambda *x: (calls.append(1), 0)[1]
+    a, shape = _host_args()
+    args = [a[k] for k in ("q_host", "block_table_host", "seq_lens_host", "out_host", "k_pool", "v_pool")]
+
+    def call(q=None, shp=None):
+        dec(q if q is not None else args[0], *args[1:4], args[4], args[5], 0.125, shp or shape)
+
+    call()
+    call()
+    call()
+    assert len(checks) == 1 and len(calls) == 3
+    call(q=args[0].clone())                                           # a new q object
+    assert len(checks) == 2
+    call(shp=bd.shape_of(a["q_host"], a["k_pool"], a["block_table_host"]))   # a new shape object
+    assert len(checks) == 3 and len(calls) == 5
+    with pytest.raises(ValueError):
+        call(q=torch.zeros(2, 8, 32, dtype=BF16))                     # too small: stopped before the library
+    assert len(calls) == 5
