@@ -19,7 +19,7 @@ from hypothesis import strategies as st
 from oracle import oracle as O
 from paged_kv_gqa_17_b200 import workloads as W
 
-SETTINGS = settings(max_examples=30, deadline=None,
+SETTINGS = settings(max_examples=30, deadline=None, derandomize=True,
                     suppress_health_check=[HealthCheck.too_slow, HealthCheck.function_scoped_fixture])
 
 lens_st = st.lists(st.one_of(st.integers(0, 40), st.integers(1, 300)), min_size=1, max_size=4)
