@@ -188,7 +188,7 @@ _DECODE_DTYPES = (torch.bfloat16, torch.bfloat16, torch.bfloat16, torch.bfloat16
 def _check_decode_tensors(q, k_pool, v_pool, block_table, seq_lens, out, shape: Shape):
     """Reject tensors whose type, layout or device differs from what the
     pointers passed to the library are taken to address.  One combined test
-    (about a microsecond) passes every well-formed call; only a failing call
+    (a few microseconds) passes every well-formed call; only a failing call
     runs the itemised checks that name the problem."""
     dev = q.get_device()
     kst = k_pool.stride()
