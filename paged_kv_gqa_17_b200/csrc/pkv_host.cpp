@@ -179,10 +179,7 @@ int pkv_work_queue_size(const int32_t *seq_lens_host, const pkv_shape *shape, in
     int rc = check_lens(seq_lens_host, shape->B);
     if (rc != PKV_OK)
         return rc;
-    int64_t n = 0;
-    for (int32_t i = 0; i < shape->B; ++i)
-        n += std::max<int64_t>(1, ceil_div(ceil_div(seq_lens_host[i], shape->page_size), chunk_pages));
-    n *= shape->H_kv;
+    const int64_t n = queue_items(seq_lens_host, shape->B, shape->H_kv, shape->page_size, chunk_pages);
     if (n > INT32_MAX)
         return PKV_ERR_CAPACITY;
     *n_items = (int32_t)n;
