@@ -15,6 +15,10 @@ real oracle and against copies with a planted mistake.
                       (tests/golden/launch_fanout_b8.txt)
   merge_state_closed  queue merge traffic = 2*G*(D+2)*4 * H_kv * (slots of
                       multi-chunk pairs); rectangular = the same over B*H_kv*S slots
+  counters_recount    every counter of every mode, recounted from what the step
+                      really moves: the bytes of the queue as built, the pages
+                      the row's tokens touch (token by token), the blocks a
+                      grid launches; plus two worked examples by hand
 """
 from __future__ import annotations
 
@@ -301,8 +305,82 @@ def policy_fill(O):
     assert plan == (O.WORK_QUEUE, 17, 45, 0), ("policy_fill worked case", plan)
 
 
+def counters_recount(O):
+    """Counters recounted by another route than the oracle's closed forms.
+
+    queue_bytes: 16 bytes per item of the queue as built plus 4 per entry of
+    its offset arrays (pair offsets; for BALANCED also the block offsets);
+    kv_bytes_streamed: the distinct pages that the rows' tokens fall on,
+    enumerated token by token, times a whole page of K and V per KV head;
+    work_items / empty_items: the blocks of the grid and those with no token;
+    merge_state_bytes: a state written and read back for every slot of a pair
+    with more than one slot.  A state is G * (D + 2) fp32 values."""
+    R = O.Rule
+    for lens, H_kv, P, C in itertools.chain(CASES, _random_cases(21, 25)):
+        G, D = 2, 64
+        H_q = G * H_kv
+        state = G * (D + 2) * 4
+        B = len(lens)
+        pages_touched = sum(len({t // P for t in range(n)}) for n in lens)
+        streamed = pages_touched * P * H_kv * 2 * D * 2
+        S = max(1, _cdiv(_cdiv(max(lens, default=0), P), C))
+        T = (C * 7) % 41 + 1
+        plans = [(O.NO_SPLIT, 1, 0, 0), (O.NO_SPLIT, 1, 0, O.FLAG_SEPARATE_MERGE), (O.SPLIT_S, S, C, 0),
+                 (O.WORK_QUEUE, S, C, 0), (O.WORK_QUEUE, S, C, O.FLAG_SEPARATE_MERGE), (O.BALANCED, T, 0, 0)]
+        for plan in plans:
+            mode, S_, C_, flags = plan
+            c = O.counters(lens, H_q, H_kv, D, P, plan)
+            what = ("counters_recount", lens, H_kv, P, plan)
+            assert c.kv_bytes_streamed == streamed, what
+            assert c.kv_bytes == sum(lens) * H_kv * 2 * D * 2, what
+            assert c.q_bytes == c.out_bytes == B * H_q * D * 2, what
+            if mode == O.NO_SPLIT:
+                assert (c.work_items, c.merge_state_bytes, c.queue_bytes, c.launches) == (B * H_kv, 0, 0, 1), what
+                assert c.empty_items == sum(1 for i in range(B) for h in range(H_kv) if lens[i] == 0), what
+                continue
+            if mode == O.SPLIT_S:
+                grid = [(i, h, s) for i in range(B) for h in range(H_kv) for s in range(S_)]
+                assert c.work_items == len(grid) and c.queue_bytes == 0, what
+                assert c.empty_items == sum(1 for (i, h, s) in grid if s * C_ * P >= lens[i]), what
+                assert c.merge_state_bytes == (2 * state * len(grid) if S_ > 1 else 0), what
+                continue
+            if mode == O.WORK_QUEUE:
+                items, indptr = O.build_work_queue(lens, H_kv, P, C_)
+                offsets = len(indptr)
+            else:
+                items, indptr, bptr = O.build_balanced_queue(lens, H_kv, P, S_)
+                offsets = len(indptr) + len(bptr)
+            assert c.queue_bytes == 16 * len(items) + 4 * offsets, what
+            assert c.work_items == (len(items) if mode == O.WORK_QUEUE else S_), what
+            assert c.empty_items == sum(1 for it in items if it[2] == it[3]), what
+            multi = sum(indptr[k + 1] - indptr[k] for k in range(B * H_kv) if indptr[k + 1] - indptr[k] > 1)
+            assert c.merge_state_bytes == 2 * state * multi, what
+            assert c.launches == 1 + (1 if flags & O.FLAG_SEPARATE_MERGE else 0), what
+    # Worked example, by hand: lens [40, 0], H_q = 4, H_kv = 2, D = 64, P = 16, T = 3.
+    # Pages per pair: 3 and 0, so U = 6 and the shares are [0,2) [2,4) [4,6).
+    # Pair (0,0) = pages 0..2 -> items (0,0,0,32) in block 0 and (0,0,32,40) in block 1;
+    # pair (0,1) = pages 3..5 -> (0,1,0,16) in block 1 and (0,1,16,40) in block 2;
+    # row 1 is empty -> (1,0,0,0), (1,1,0,0) in block 2.  Six items, 5 pair offsets,
+    # 4 block offsets: 16*6 + 4*5 + 4*4 = 132 queue bytes.  Two pairs of two slots with
+    # states of 2*(64+2)*4 = 528 bytes: 2 * 4 * 528 = 4224 merge bytes.  K+V of 40 tokens:
+    # 40 * 2 * 2 * 64 * 2 = 20480; of 3 whole pages: 48 * 512 = 24576.
+    c = O.counters([40, 0], 4, 2, 64, 16, (O.BALANCED, 3, 0, 0))
+    assert (c.launches, c.work_items, c.empty_items, c.merge_state_bytes, c.kv_bytes, c.kv_bytes_streamed,
+            c.queue_bytes) == (1, 3, 2, 4224, 20480, 24576, 132), ("counters worked balanced", c)
+    # The same batch without a split: 4 blocks, 2 of them for the empty row, nothing to merge.
+    c = O.counters([40, 0], 4, 2, 64, 16, (O.NO_SPLIT, 1, 0, 0))
+    assert (c.launches, c.work_items, c.empty_items, c.merge_state_bytes, c.queue_bytes) == (1, 4, 2, 0, 0), \
+        ("counters worked no-split", c)
+    # The work queue at C = 2 pages: pair (0,h) has items [0,32) and [32,40), row 1 one empty
+    # item per head -> 6 items and 5 offsets: 16*6 + 4*5 = 116 bytes; merge 2 * 4 * 528.
+    c = O.counters([40, 0], 4, 2, 64, 16, (O.WORK_QUEUE, 2, 2, 0))
+    assert (c.work_items, c.empty_items, c.merge_state_bytes, c.queue_bytes) == (6, 2, 4224, 116), \
+        ("counters worked queue", c)
+
+
 HOST_PINS = (queue_closed_form, queue_cover, queue_bruteforce, policy_paper, policy_semantics, policy_fill,
-             launch_fanout, merge_state_closed, balanced_shares, balanced_cover, balanced_bruteforce)
+             launch_fanout, merge_state_closed, counters_recount, balanced_shares, balanced_cover,
+             balanced_bruteforce)
 
 
 def run_all(O):

@@ -50,6 +50,16 @@ PY_MUTANTS = {
     "balanced item not clipped to row": ("min((y - u) * P, n)", "(y - u) * P"),
     "fill rule allows one item too many": ("if fill_items(lens, H_kv, P, c) <= chosen.num_splits:",
                                            "if fill_items(lens, H_kv, P, c) <= chosen.num_splits + 1:"),
+    "queue bytes miss the last pair offset": ("qbytes = 16 * work + 4 * (B * H_kv + 1)\n",
+                                              "qbytes = 16 * work + 4 * B * H_kv\n"),
+    "balanced queue bytes miss the block offsets": (" + 4 * (B * H_kv + 1) + 4 * (S + 1)", " + 4 * (B * H_kv + 1)"),
+    "streamed bytes count valid tokens only": ("kv_streamed = sum(pages) * P * H_kv", "kv_streamed = sum(lens) * H_kv"),
+    "balanced merge counts single-slot pairs": ("        merge = 2 * sum(k for k in per_pair if k > 1) * state",
+                                                "        merge = 2 * sum(per_pair) * state"),
+    "balanced work counts items": ("        work = S\n", "        work = len(items)\n"),
+    "no-split empty rows not per head": ("work = B * H_kv\n        empty = H_kv * sum(",
+                                         "work = B * H_kv\n        empty = sum("),
+    "no-split work counts rows": ("        work = B * H_kv\n", "        work = B\n"),
     "fill rule ignores heads": ("    return H_kv * sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)",
                                 "    return sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)"),
 }
