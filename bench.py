@@ -46,7 +46,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from paged_kv_gqa_17_b200.timing import Flush, pool_copies, time_isolated, time_steady  # noqa: E402
+from paged_kv_gqa_17_b200.timing import Flush, n_pool_copies, pool_copies, time_isolated, time_steady  # noqa: E402
 
 METRIC = "paged GQA decode: KV GB/s (% of B200 HBM peak) and µs/step at batch 1/4/8"
 FALLBACK_HBM_GBS = 6650.0
@@ -248,6 +248,15 @@ def _describe(w, plan):
     }
 
 
+def arm_config(w, plan, world: int, graph: bool):
+    """The `config` object of the JSON line; both arms print the same one."""
+    n_copies = n_pool_copies(w)
+    return dict(_describe(w, plan), parallelism=f"replicas x{world} (one workload per GPU)",
+                timed_steps="one CUDA graph of the K steps, replayed" if graph else "K steps queued from Python",
+                l2=f"inputs larger than L2: back-to-back steps rotate over {n_copies} copies of the KV pool "
+                   f"({n_copies * w.kv_bytes() / 2**20:.0f} MiB of step data); latency_us is flushed per step")
+
+
 def time_e2e(w, K, W, torch, bd, flush):
     """Per-step wall times (ms) of synchronized pkv_decode_host calls from pinned host buffers."""
     q_h = w.q.cpu().pin_memory()
@@ -268,10 +277,29 @@ def time_e2e(w, K, W, torch, bd, flush):
         t0 = time.perf_counter()
         plan = dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape)
         times.append((time.perf_counter() - t0) * 1e3)
+    # where the time goes: the same calls once more through pkv_decode_host_timed
+    # (host clock inside the library, CUDA events around the copies and kernels)
+    parts = []
+    for i in range(min(K, 50)):
+        flush(i)
+        torch.cuda.synchronize()
+        tm = bd.HostTiming()
+        t0 = time.perf_counter()
+        dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, timing=tm)
+        d = tm.as_dict()
+        d["wall_us"] = (time.perf_counter() - t0) * 1e6
+        parts.append(d)
+    breakdown = {k: round(statistics.median(p[k] for p in parts), 2) for k in parts[0]}
+    breakdown["binding_us"] = round(breakdown["wall_us"] - sum(breakdown[k] for k in (
+        "host_plan_us", "host_enqueue_us", "host_wait_us", "host_unpack_us")), 2)
+    breakdown["note"] = ("medians over timed calls: host_* from the library's host clock (plan = policy + queue + "
+                         "staging image; enqueue = copies and launches queued; wait = cudaStreamSynchronize; unpack "
+                         "= out read from staging), dev_* from CUDA events, binding_us = Python and ctypes around "
+                         "the call")
     counters = bd.plan_counters(w.seq_lens, shape, plan)
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + lens_h.numel() * 4 + counters["queue_bytes"]
     d2h = out_h.numel() * 2 + 4
-    return times, h2d, d2h, out_h
+    return times, h2d, d2h, out_h, breakdown
 
 
 def measure_workload(name, seed, device, K, W, torch, bd, W_mod, flush):
@@ -337,7 +365,6 @@ def run_ours(args):
         steady_ms = time_steady(w, dp, args.steps, args.warmup, torch, bd, copies, graph=not args.no_graph)
     torch.cuda.synchronize()
     barrier(dist, device)
-    n_copies = len(copies)
     del copies
     total_ms = max_over_ranks(steady_ms, dist, device)
     total_bytes = sum_over_ranks(float(w.algorithmic_bytes() * args.steps), dist, device)
@@ -351,7 +378,8 @@ def run_ours(args):
     early_ms = time_steady(w, dp_early, args.steps, args.warmup, torch, bd, copies,
                            graph=not args.no_graph) / args.steps
     del copies, dp_early
-    e2e_ms, h2d, d2h, _ = time_e2e(w, args.e2e_steps or args.steps, min(args.warmup, 3), torch, bd, flush)
+    e2e_ms, h2d, d2h, _, e2e_parts = time_e2e(w, args.e2e_steps or args.steps, min(args.warmup, 3), torch, bd,
+                                              flush)
     e2e_total = max_over_ranks(sum(e2e_ms), dist, device)
     e2e_bytes = sum_over_ranks(float(w.algorithmic_bytes() * len(e2e_ms)), dist, device)
 
@@ -383,11 +411,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded bf16 N(0,1) q/K/V, random page placement)",
-        "config": dict(_describe(w, dp.plan), parallelism=f"replicas x{world} (one workload per GPU)",
-                       timed_steps="one CUDA graph of the K steps, replayed" if not args.no_graph
-                       else "K steps queued from Python",
-                       l2=f"inputs larger than L2: back-to-back steps rotate over {n_copies} copies of the KV pool "
-                          f"({n_copies * w.kv_bytes() / 2**20:.0f} MiB of step data); latency_us is flushed per step"),
+        "config": arm_config(w, dp.plan, world, not args.no_graph),
         "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4),
         "roofline": {
             "bound": "hbm",
@@ -408,6 +432,7 @@ def run_ours(args):
             "d2h_bytes_per_step": d2h,
             "note": "synchronized pkv_decode_host per step: host plan + queue, H2D of q/table/lengths/queue "
                     "from pinned memory, kernels, D2H of out; KV cache resident",
+            "breakdown": e2e_parts,
         },
         "gpu_launches": int(counters["launches"] * args.steps),
         "counters": counters,
@@ -460,6 +485,11 @@ def run_reference(args):
     seed = args.seed if args.seed is not None else W_mod.SEED_REPORT
     w = W_mod.make(args.workload, seed=seed)
     pr = O.problem(w.q, w.k_pool, w.v_pool, w.block_table, w.seq_lens, w.scale)
+    # the plan our arm runs, from the oracle's own policy lookup over the built-in
+    # table (bit-identical to the library's), so that both lines carry one config
+    rules = O.load_rules(os.path.join(ROOT, "paged_kv_gqa_17_b200", "policy_b200.json"))
+    plan = type("Plan", (), dict(zip(("mode", "num_splits", "chunk_pages", "flags"),
+                                     O.select_policy(w.seq_lens, w.P, rules, w.H_kv))))
     cores = os.cpu_count() or 1
     for _ in range(args.warmup):
         O.paged_decode(pr, n_threads=cores)
@@ -474,12 +504,12 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": _describe(w, type("P", (), {"mode": 0, "num_splits": 1, "chunk_pages": 0, "flags": 0})()),
+        "config": arm_config(w, plan, world, not args.no_graph),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": f"full decode steps of the {w.name} workload, fp64 C oracle, {cores} threads"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    line["config"]["plan"] = "fp64 two-pass softmax per (row, head), no split"
+    line["reference_method"] = "fp64 two-pass softmax per (row, head), no split (the CPU oracle)"
     print(json.dumps(line), flush=True)
 
 

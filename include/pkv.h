@@ -353,22 +353,31 @@ PKV_API int pkv_paged_decode(const void *q, const void *k_pool, const void *v_po
  * cudaMalloc, no cudaFree, no allocating library routine.
  *  - A plan whose workspace (pkv_workspace_bytes) exceeds the array returns
  *    PKV_ERR_CAPACITY before anything is queued.
- *  - The first call on a device looks up the array's device address with
- *    cudaGetSymbolAddress (with that device current) and caches it; make
- *    that first call before any stream capture.
- *  - Each call queues a memset that zeroes the error word and the counters,
- *    then the kernels; the array keeps the last call's contents otherwise.
+ *  - The first call in a CUDA context looks up the array's device address
+ *    with cudaGetSymbolAddress (the device current) and caches it for that
+ *    context; make that first call before any stream capture.  After
+ *    cudaDeviceReset the cached address may be stale: reload the library.
+ *  - A call that passes every argument check queues a memset that zeroes the
+ *    error word and the counters, then the kernels; a rejected call queues
+ *    nothing.  The array keeps the last call's contents otherwise.
  *  - All calls share the one array: calls that may overlap on the GPU (two
  *    streams, two threads) race and corrupt each other's results.  Order
  *    them on one stream.
- *  - Errors the kernels detect on device data cannot be read back through
- *    this entry point; use pkv_paged_decode with a workspace to diagnose.
+ *  - Errors the kernels detect on device data are read back with
+ *    pkv_noalloc_status.
  * Other arguments, layouts and return codes as pkv_paged_decode. */
 PKV_API int pkv_paged_decode_noalloc(const void *q, const void *k_pool, const void *v_pool,
                                      const int32_t *block_table, const int32_t *seq_lens,
                                      int32_t page_size, float scale, void *out, const pkv_shape *shape,
                                      const pkv_plan *plan, const pkv_work_item *items,
                                      const int32_t *indptr, int32_t n_items, void *stream);
+
+/* pkv_workspace_status for the scratch of pkv_paged_decode_noalloc:
+ * synchronize `stream`, then read the error word the last no-alloc call left
+ * (PKV_OK, PKV_ERR_TIMEOUT or PKV_ERR_DEVICE_INPUT; the raw bit mask in
+ * *device_error when not NULL).  Allocates nothing.  The paper has no
+ * counterpart. */
+PKV_API int pkv_noalloc_status(void *stream, int32_t *device_error);
 
 /* Sizes of the caller buffers pkv_decode_host needs for this batch and
  * policy table (rules NULL = built-in): *device_bytes of device memory and
@@ -399,6 +408,30 @@ PKV_API int pkv_decode_host(const void *q_host, const int32_t *block_table_host,
                             const pkv_policy_rule *rules, int32_t n_rules, void *device_buffer,
                             size_t device_buffer_bytes, void *host_staging,
                             size_t host_staging_bytes, void *stream, pkv_plan *plan_out);
+
+/* Where the time of one pkv_decode_host call goes (pkv_decode_host_timed).
+ * Host parts from a monotonic host clock, device parts from CUDA events
+ * recorded on the call's stream around the copies and the kernels. */
+typedef struct {
+    double host_plan_us;     /* policy, queue and the upload image written into host_staging */
+    double host_enqueue_us;  /* the copies and the kernel launches queued on the stream */
+    double host_wait_us;     /* cudaStreamSynchronize, from the last enqueue until it returned */
+    double host_unpack_us;   /* out and the error word read back from host_staging */
+    double dev_h2d_us;       /* device time of the host->device copies */
+    double dev_kernel_us;    /* device time of the decode kernels */
+    double dev_d2h_us;       /* device time of the device->host copies */
+} pkv_host_timing;
+
+/* pkv_decode_host that also reports where its time went into *timing (when
+ * not NULL; the events it records add a little device time of their own).
+ * Arguments and return codes as pkv_decode_host [PKV, Methodology 3
+ * "Evaluation protocol": synchronized wall time including host planning]. */
+PKV_API int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host,
+                                  const int32_t *seq_lens_host, void *out_host, const void *k_pool,
+                                  const void *v_pool, float scale, const pkv_shape *shape,
+                                  const pkv_policy_rule *rules, int32_t n_rules, void *device_buffer,
+                                  size_t device_buffer_bytes, void *host_staging, size_t host_staging_bytes,
+                                  void *stream, pkv_plan *plan_out, pkv_host_timing *timing);
 
 #ifdef __cplusplus
 }

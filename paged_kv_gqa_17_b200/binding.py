@@ -71,6 +71,15 @@ class Counters(ctypes.Structure):
         return {f: int(getattr(self, f)) for f, _ in self._fields_}
 
 
+class HostTiming(ctypes.Structure):
+    """Where one pkv_decode_host call's time went (pkv_host_timing), in microseconds."""
+    _fields_ = [(n, ctypes.c_double) for n in ("host_plan_us", "host_enqueue_us", "host_wait_us", "host_unpack_us",
+                                               "dev_h2d_us", "dev_kernel_us", "dev_d2h_us")]
+
+    def as_dict(self):
+        return {f: float(getattr(self, f)) for f, _ in self._fields_}
+
+
 _lib = None
 
 # (name, restype, argtypes) of every function include/pkv.h declares
@@ -96,9 +105,12 @@ SIGNATURES = [
      [c_p, c_p, c_p, c_p, c_p, c_i32, ctypes.c_float, c_p, c_p, c_p, c_p, c_p, c_i32, c_p, c_sz, c_p]),
     ("pkv_paged_decode_noalloc", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_i32, ctypes.c_float, c_p, c_p, c_p, c_p, c_p, c_i32, c_p]),
+    ("pkv_noalloc_status", ctypes.c_int, [c_p, c_p]),
     ("pkv_decode_host_bytes", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_p, c_p]),
     ("pkv_decode_host", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p]),
+    ("pkv_decode_host_timed", ctypes.c_int,
+     [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p, c_p]),
 ]
 
 
@@ -513,6 +525,17 @@ def paged_decode_noalloc(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Te
     return out
 
 
+def noalloc_status(stream=None) -> int:
+    """Synchronize and return the raw device error mask the last
+    pkv_paged_decode_noalloc call left in the library's scratch (0 = clean)."""
+    L = lib()
+    err = c_i32(0)
+    rc = L.pkv_noalloc_status(_stream_ptr(stream), ctypes.byref(err))
+    if rc not in (0, -5, -6):
+        _check(rc, "pkv_noalloc_status")
+    return int(err.value)
+
+
 def workspace_status(plan: DecodePlan, stream=None) -> int:
     """Synchronize and return the raw device error mask of a plan's workspace (0 = clean)."""
     L = lib()
@@ -536,6 +559,7 @@ class HostDecoder:
         self.host = torch.empty(0, dtype=torch.uint8).pin_memory()
         self._stream = _stream_ptr(stream if stream is not None else torch.cuda.current_stream(self.device))
         self._fn = lib().pkv_decode_host
+        self._fn_timed = lib().pkv_decode_host_timed
         self._plan = Plan()
         self._plan_ref = ctypes.byref(self._plan)
         self._bufs = (0, 0, 0, 0)
@@ -556,7 +580,9 @@ class HostDecoder:
 
     def __call__(self, q_host: torch.Tensor, block_table_host: torch.Tensor, seq_lens_host: torch.Tensor,
                  out_host: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, scale: float, shape: Shape,
-                 rules=None, stream=None) -> Plan:
+                 rules=None, stream=None, timing: Optional[HostTiming] = None) -> Plan:
+        """One synchronized step; with `timing` (a HostTiming), pkv_decode_host_timed
+        also fills in where the call's time went."""
         seen = self._checked
         if not (seen and seen[6] is shape and seen[0]() is q_host and seen[1]() is block_table_host
                 and seen[2]() is seq_lens_host and seen[3]() is out_host and seen[4]() is k_pool
@@ -567,9 +593,10 @@ class HostDecoder:
                                                             k_pool, v_pool)) + (shape,)
         arr, n = rules_array(rules) if rules is not None else (None, 0)
         dev, dev_n, host, host_n = self._bufs
-        rc = self._fn(q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(), out_host.data_ptr(),
-                      k_pool.data_ptr(), v_pool.data_ptr(), float(scale), ctypes.byref(shape), arr, n, dev, dev_n,
-                      host, host_n, self._stream if stream is None else _stream_ptr(stream), self._plan_ref)
+        args = (q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(), out_host.data_ptr(),
+                k_pool.data_ptr(), v_pool.data_ptr(), float(scale), ctypes.byref(shape), arr, n, dev, dev_n,
+                host, host_n, self._stream if stream is None else _stream_ptr(stream), self._plan_ref)
+        rc = self._fn(*args) if timing is None else self._fn_timed(*args, ctypes.byref(timing))
         if rc != 0:
             raise PkvError(rc, "pkv_decode_host")
         return Plan.from_buffer_copy(self._plan)

@@ -1,6 +1,7 @@
 """Calibrate the built-in policy table on the GPU from measured timings.
 
-    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--steps 60] [--draws 3]
+    python -m paged_kv_gqa_17_b200.calibrate [--out paged_kv_gqa_17_b200/policy_b200.json] [--report REPORT.md]
+        [--steps 60] [--draws 3]
 
 The policy maps (batch size B, longest row N_max) to an execution plan
 [PersistentKV explainer, Technical summary > Methodology > 2 "Calibrated
@@ -26,7 +27,7 @@ on a holdout seed].  This script does the same by measurement:
      lists the chosen plan's time against the best candidate (the regret).
 
 It writes the table as JSON (the library's build turns it into its built-in
-table) and a markdown report.
+table) and prints a markdown report (also written to --report when given).
 """
 from __future__ import annotations
 
@@ -137,7 +138,7 @@ def build_rules(best):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--out", default=os.path.join(HERE, "policy_b200.json"))
-    ap.add_argument("--report", default=os.path.join(ROOT, "profiles", "policy_calibration_b200.md"))
+    ap.add_argument("--report", default=None, help="also write the markdown report to this file")
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--draws", type=int, default=3, help="batches per cell (geometric mean)")
     args = ap.parse_args(argv)
@@ -171,7 +172,8 @@ def main(argv=None):
         f.write("\n")
     # holdout check
     lines = ["# Policy calibration on B200", "",
-             "Command: `python -m paged_kv_gqa_17_b200.calibrate` (writes paged_kv_gqa_17_b200/policy_b200.json).", "",
+             "Command: `python -m paged_kv_gqa_17_b200.calibrate" + (f" --report {args.report}" if args.report else "")
+             + "` (writes paged_kv_gqa_17_b200/policy_b200.json).", "",
              "Steady-state µs per decode step (CUDA-graph replay of back-to-back steps over rotating pool copies), "
              f"H_kv=8, D=128; each cell is the geometric mean over {args.draws} batches (G = 4, 4, 8). "
              "Calibration seed 20260622 picks the plan; holdout seed 20260623 (other batches) re-measures it.", "",
@@ -185,10 +187,12 @@ def main(argv=None):
             lines.append(f"| {B} | {n} | {MODE_NAMES[c[0]]} {c[1:]} | {calib[(bi, nj)][c]:.2f} | {hold[c]:.2f} | "
                          f"{MODE_NAMES[hb[0]]} {hb[1:]} | {hold[hb]:.2f} | {100 * (hold[c] / hold[hb] - 1):.1f}% |")
             print(lines[-1], flush=True)
-    os.makedirs(os.path.dirname(args.report), exist_ok=True)
-    with open(args.report, "w") as f:
-        f.write("\n".join(lines) + "\n")
-    print(f"wrote {args.out} and {args.report}")
+    if args.report:
+        os.makedirs(os.path.dirname(os.path.abspath(args.report)), exist_ok=True)
+        with open(args.report, "w") as f:
+            f.write("\n".join(lines) + "\n")
+    print("\n".join(lines))
+    print(f"wrote {args.out}" + (f" and {args.report}" if args.report else ""))
 
 
 if __name__ == "__main__":

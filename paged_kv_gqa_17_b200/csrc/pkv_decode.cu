@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <chrono>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -2364,11 +2365,15 @@ struct WsPtrs {
 // Internal entry shared by pkv_paged_decode, pkv_paged_decode_noalloc and
 // pkv_decode_host.  With `sections` NULL the workspace sections are carved
 // out of `workspace` (checked against workspace_bytes); otherwise they are
-// taken from `sections` and workspace/workspace_bytes are ignored.
+// taken from `sections` and workspace/workspace_bytes are ignored.  With
+// zero_bytes > 0 the first zero_bytes of the workspace (error word and
+// completion counters) are cleared on the stream once every argument check
+// has passed, right before the launch, so a rejected call queues nothing.
 int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, const int32_t *block_table,
                       const int32_t *seq_lens, int32_t page_size, float scale, void *out, const pkv_shape *shape,
                       const pkv_plan *plan, const pkv_work_item *items, const int32_t *indptr, int32_t n_items,
-                      void *workspace, size_t workspace_bytes, cudaStream_t st, const WsPtrs *sections = nullptr)
+                      void *workspace, size_t workspace_bytes, cudaStream_t st, const WsPtrs *sections = nullptr,
+                      size_t zero_bytes = 0)
 {
     if (check_shape(shape) != PKV_OK || !plan || page_size != shape->page_size)
         return PKV_ERR_INVALID;
@@ -2461,6 +2466,8 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     const bool deep = (pl.flags & PKV_FLAG_DEEP_RING) != 0;
     // cluster merge: the S blocks of each (row, KV head) form one cluster
     const unsigned cluster = (pl.flags & PKV_FLAG_CLUSTER_MERGE) ? (unsigned)pl.num_splits : 0u;
+    if (zero_bytes > 0 && cudaMemsetAsync(wp.error, 0, zero_bytes, st) != cudaSuccess)
+        return PKV_ERR_CUDA;
     cudaError_t le;
     if (pl.mode == PKV_BALANCED)
         le = deep ? launch_balanced_nst<PKV_NST_BAL_DEEP>(s.head_dim, NT, prm, grid, st, pdl)
@@ -2622,24 +2629,54 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device.  In host code
-// the symbol is only a host-side handle; the address has to be looked up once
-// per device (with that device current) and is cached here.
+// Device address of g_noalloc_scratch in the current CUDA context.  In host
+// code the symbol is only a host-side handle: the address is looked up with
+// cudaGetSymbolAddress (the device in question current) the first time a
+// context calls, and cached per context, so a caller that makes a context of
+// its own current on the same device gets that context's copy.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
+
 void *noalloc_scratch_address()
 {
     static std::mutex mu;
-    static void *addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    static CUcontext ctxs[64] = {};
+    static void *addrs[64] = {};
+    static int used = 0;
+    CtxGetCurrentFn current = ctx_get_current();
+    if (!current)
+        return nullptr;
+    CUcontext ctx = nullptr;
+    if (current(&ctx) != CUDA_SUCCESS)
         return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess)
-            return nullptr;
-        addr[dev] = ptr;
-    }
-    return addr[dev];
+    for (int i = 0; ctx && i < used; ++i)
+        if (ctxs[i] == ctx)
+            return addrs[i];
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+        return nullptr;
+    // the lookup makes the device's primary context current if none was
+    if (!ctx && (current(&ctx) != CUDA_SUCCESS || !ctx))
+        return ptr;
+    const int slot = used < 64 ? used++ : 63;
+    ctxs[slot] = ctx;
+    addrs[slot] = ptr;
+    return ptr;
 }
 
 // pkv_decode_host moves a step's inputs in one host->device copy and its
@@ -2667,6 +2704,25 @@ struct HostLayout {
     size_t up_bytes, down_bytes, dev_total;
     size_t h_down_off, host_total;
 };
+
+// Four timing events per device for pkv_decode_host_timed, made on first use.
+cudaEvent_t *timing_events()
+{
+    static std::mutex mu;
+    static cudaEvent_t events[64][4] = {};
+    static bool made[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!made[dev]) {
+        for (int i = 0; i < 4; ++i)
+            if (cudaEventCreate(&events[dev][i]) != cudaSuccess)
+                return nullptr;
+        made[dev] = true;
+    }
+    return events[dev];
+}
 
 int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_rule *rules, int32_t n_rules,
                 HostLayout *L)
@@ -2738,13 +2794,20 @@ int pkv_paged_decode_noalloc(const void *q, const void *k_pool, const void *v_po
     void *scratch = noalloc_scratch_address();
     if (!scratch)
         return PKV_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     // The array keeps whatever the previous call left in it: the error word
-    // and the completion counters must start at zero, the partial states not.
-    if (cudaMemsetAsync(scratch, 0, ws.m_off, st) != cudaSuccess)
-        return PKV_ERR_CUDA;
+    // and the completion counters must start at zero (cleared on the stream
+    // after the argument checks, just before the launch), the partial states not.
     return paged_decode_impl(q, k_pool, v_pool, block_table, seq_lens, page_size, scale, out, shape, plan, items,
-                             indptr, n_items, scratch, kNoAllocScratchBytes, st);
+                             indptr, n_items, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream),
+                             nullptr, ws.m_off);
+}
+
+int pkv_noalloc_status(void *stream, int32_t *device_error)
+{
+    void *scratch = noalloc_scratch_address();
+    if (!scratch)
+        return PKV_ERR_CUDA;
+    return pkv_workspace_status(scratch, stream, device_error);
 }
 
 int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape *shape, const pkv_policy_rule *rules,
@@ -2766,6 +2829,25 @@ int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const i
                     const pkv_policy_rule *rules, int32_t n_rules, void *device_buffer, size_t device_buffer_bytes,
                     void *host_staging, size_t host_staging_bytes, void *stream, pkv_plan *plan_out)
 {
+    return pkv_decode_host_timed(q_host, block_table_host, seq_lens_host, out_host, k_pool, v_pool, scale, shape,
+                                 rules, n_rules, device_buffer, device_buffer_bytes, host_staging,
+                                 host_staging_bytes, stream, plan_out, nullptr);
+}
+
+int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, const int32_t *seq_lens_host,
+                          void *out_host, const void *k_pool, const void *v_pool, float scale,
+                          const pkv_shape *shape, const pkv_policy_rule *rules, int32_t n_rules,
+                          void *device_buffer, size_t device_buffer_bytes, void *host_staging,
+                          size_t host_staging_bytes, void *stream, pkv_plan *plan_out, pkv_host_timing *timing)
+{
+    using clock = std::chrono::steady_clock;
+    const clock::time_point t0 = clock::now();
+    cudaEvent_t *ev = nullptr;
+    if (timing) {
+        std::memset(timing, 0, sizeof *timing);
+        if (!(ev = timing_events()))
+            return PKV_ERR_CUDA;
+    }
     HostLayout L;
     int rc = host_layout(seq_lens_host, shape, rules, n_rules, &L);
     if (rc != PKV_OK)
@@ -2800,12 +2882,16 @@ int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const i
         rc = pkv_build_balanced_queue(seq_lens_host, shape, L.plan.num_splits, h_items, L.n_items, h_indptr, &n);
     if (rc != PKV_OK)
         return rc;
-    bool ok = cudaMemcpyAsync(dev, hst, L.up_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    const clock::time_point t1 = clock::now();
+    bool ok = !ev || cudaEventRecord(ev[0], st) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dev, hst, L.up_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
     if (ok && !L.q_inline)
         ok = cudaMemcpyAsync(dev + L.q_off, q_host, L.q_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
     if (ok && !L.bt_inline)
         ok = cudaMemcpyAsync(dev + L.bt_off, block_table_host, L.bt_bytes, cudaMemcpyHostToDevice, st) ==
              cudaSuccess;
+    if (ok && ev)
+        ok = cudaEventRecord(ev[1], st) == cudaSuccess;
     if (!ok)
         return PKV_ERR_CUDA;
     const WsPtrs wp{reinterpret_cast<uint32_t *>(dev + L.err_off), reinterpret_cast<uint32_t *>(dev + L.counters_off),
@@ -2817,16 +2903,36 @@ int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const i
                            reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, nullptr, 0, st, &wp);
     if (rc != PKV_OK)
         return rc;
+    ok = !ev || cudaEventRecord(ev[2], st) == cudaSuccess;
     uint8_t *h_down = hst + L.h_down_off;
-    ok = cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
     if (ok && !L.out_inline)
         ok = cudaMemcpyAsync(out_host, dev + L.out_off, L.q_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    if (ok && ev)
+        ok = cudaEventRecord(ev[3], st) == cudaSuccess;
+    const clock::time_point t2 = clock::now();
     if (!ok || cudaStreamSynchronize(st) != cudaSuccess)
         return PKV_ERR_CUDA;
+    const clock::time_point t3 = clock::now();
     if (L.out_inline)
         std::memcpy(out_host, h_down + (L.out_off - L.err_off), L.q_bytes);
     uint32_t err;
     std::memcpy(&err, h_down, 4);
+    if (timing) {
+        const clock::time_point t4 = clock::now();
+        auto us = [](clock::duration d) { return std::chrono::duration<double, std::micro>(d).count(); };
+        timing->host_plan_us = us(t1 - t0);
+        timing->host_enqueue_us = us(t2 - t1);
+        timing->host_wait_us = us(t3 - t2);
+        timing->host_unpack_us = us(t4 - t3);
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, ev[0], ev[1]) == cudaSuccess)
+            timing->dev_h2d_us = ms * 1e3;
+        if (cudaEventElapsedTime(&ms, ev[1], ev[2]) == cudaSuccess)
+            timing->dev_kernel_us = ms * 1e3;
+        if (cudaEventElapsedTime(&ms, ev[2], ev[3]) == cudaSuccess)
+            timing->dev_d2h_us = ms * 1e3;
+    }
     return status_from_error_word(err);
 }
 

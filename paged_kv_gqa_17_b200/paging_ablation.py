@@ -1,7 +1,7 @@
 """Paging-overhead ablation on B200: how much the block-table indirection and
 the pool layout cost.
 
-    python -m paged_kv_gqa_17_b200.paging_ablation [--out profiles/paging_ablation_b200.md]
+    python -m paged_kv_gqa_17_b200.paging_ablation [--out REPORT.md]
 
 "Chapter 8 - Next-generation KV cache management" (actionbridge.io), section
 8.1, states that a paged kernel runs within a few percent of a kernel over a
@@ -52,7 +52,7 @@ def identity_copy(w, torch):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--out", default=os.path.join(ROOT, "profiles", "paging_ablation_b200.md"))
+    ap.add_argument("--out", default=None, help="also write the markdown report to this file")
     ap.add_argument("--steps", type=int, default=300)
     args = ap.parse_args(argv)
 
@@ -64,7 +64,7 @@ def main(argv=None):
 
     dev = torch.device("cuda")
     lines = ["# Paging-overhead ablation (B200)", "",
-             "Command: `python -m paged_kv_gqa_17_b200.paging_ablation`. Same values, same plan (built-in policy); "
+             "Command: `python -m paged_kv_gqa_17_b200.paging_ablation" + (f" --out {args.out}" if args.out else "") + "`. Same values, same plan (built-in policy); "
              "steady-state µs per step (CUDA-graph replay of back-to-back steps over rotating pool copies).", "",
              "| workload | plan | permuted HND | identity HND | permuted NHD | identity / permuted |",
              "|---|---|---|---|---|---|"]
@@ -85,9 +85,10 @@ def main(argv=None):
         lines.append(f"| {name} | {plan.tuple()} | {res['permuted HND']:.2f} | {res['identity HND']:.2f} | "
                      f"{res['permuted NHD']:.2f} | {res['identity HND'] / res['permuted HND']:.3f} |")
         torch.cuda.empty_cache()
-    os.makedirs(os.path.dirname(args.out), exist_ok=True)
-    with open(args.out, "w") as f:
-        f.write("\n".join(lines) + "\n")
+    if args.out:
+        os.makedirs(os.path.dirname(os.path.abspath(args.out)), exist_ok=True)
+        with open(args.out, "w") as f:
+            f.write("\n".join(lines) + "\n")
     print("\n".join(lines))
 
 

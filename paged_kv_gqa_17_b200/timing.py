@@ -28,11 +28,16 @@ class Flush:
         self.b.sum()
 
 
-def pool_copies(w, torch, l2_bytes=126 << 20):
-    """Copies of the KV pool so that >= 3 L2 sizes of step data separate two
-    reads of the same copy (at most 8 copies; 1 when one step already exceeds that)."""
+def n_pool_copies(w, l2_bytes=126 << 20) -> int:
+    """How many copies of the KV pool put >= 3 L2 sizes of step data between
+    two reads of the same copy (at most 8; 1 when one step already exceeds that)."""
     per_step = w.kv_bytes()
-    n = 1 if per_step >= 3 * l2_bytes else min(8, -(-3 * l2_bytes // per_step) + 1)
+    return 1 if per_step >= 3 * l2_bytes else min(8, -(-3 * l2_bytes // per_step) + 1)
+
+
+def pool_copies(w, torch, l2_bytes=126 << 20):
+    """The pool and n_pool_copies(w) - 1 clones of it."""
+    n = n_pool_copies(w, l2_bytes)
     return [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone()) for _ in range(n - 1)]
 
 

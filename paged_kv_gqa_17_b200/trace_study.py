@@ -1,6 +1,6 @@
 """Scheduler study on B=8 traces: launch fan-out, merge-state traffic, time.
 
-    python -m paged_kv_gqa_17_b200.trace_study [--out profiles/trace_study_b200.md]
+    python -m paged_kv_gqa_17_b200.trace_study [--out REPORT.md]
 
 The PersistentKV explainer (Technical summary > Results, scheduling overhead)
 reports on a bimodal B=8 trace that the compact work queue cut launch fan-out
@@ -34,7 +34,7 @@ CHUNK = 16  # pages per chunk for the rectangular-vs-queue comparison
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--out", default=os.path.join(ROOT, "profiles", "trace_study_b200.md"))
+    ap.add_argument("--out", default=None, help="also write the markdown report to this file")
     ap.add_argument("--steps", type=int, default=200)
     args = ap.parse_args(argv)
 
@@ -46,7 +46,7 @@ def main(argv=None):
 
     dev = torch.device("cuda")
     lines = ["# Scheduler study on B=8 traces (B200)", "",
-             "Command: `python -m paged_kv_gqa_17_b200.trace_study`. Traces from workloads.py (seed 20260623; "
+             "Command: `python -m paged_kv_gqa_17_b200.trace_study" + (f" --out {args.out}" if args.out else "") + "`. Traces from workloads.py (seed 20260623; "
              "generated parameters, the pages publish none). H_q=32, H_kv=8, D=128, 16-token pages. Times are "
              "steady-state µs per step (back-to-back steps over rotating pool copies).", "",
              f"Counters (closed form, library `pkv_plan_counters`), chunk C = {CHUNK} pages:", "",
@@ -90,9 +90,10 @@ def main(argv=None):
         cells = [f"{us:.2f} ({gbs:.0f})" for _, us, gbs in row[1:]]
         cells[-1] = f"{row[-1][0][7:]}: {cells[-1]}"
         lines.append(f"| {row[0]} | " + " | ".join(cells) + " |")
-    os.makedirs(os.path.dirname(args.out), exist_ok=True)
-    with open(args.out, "w") as f:
-        f.write("\n".join(lines) + "\n")
+    if args.out:
+        os.makedirs(os.path.dirname(os.path.abspath(args.out)), exist_ok=True)
+        with open(args.out, "w") as f:
+            f.write("\n".join(lines) + "\n")
     print("\n".join(lines))
 
 

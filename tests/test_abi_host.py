@@ -177,7 +177,7 @@ def test_host_pins_hold_for_the_c_planner(L):
     """The oracle's host pins, run against an adapter over the C planner."""
 
     class Adapter:
-        NO_SPLIT, SPLIT_S, WORK_QUEUE, FLAG_SEPARATE_MERGE, INT32_MAX = 0, 1, 2, 1, 2**31 - 1
+        NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED, FLAG_SEPARATE_MERGE, INT32_MAX = 0, 1, 2, 3, 1, 2**31 - 1
         Rule = O.Rule
         load_rules = staticmethod(O.load_rules)
 

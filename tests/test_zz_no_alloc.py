@@ -30,6 +30,9 @@ RULES = [
     bd.Rule(*ANY, 2, 1, 5, 1),    # work queue, separate merge kernel
     bd.Rule(*ANY, 0, 1, 0, 0),    # no split
     bd.Rule(*ANY, 1, 9, 0, 0),    # split-S again, other slot layout
+    bd.Rule(*ANY, 3, 24, 0, 0),   # balanced grid: several items per block, deferred merges
+    bd.Rule(*ANY, 1, 8, 0, 8),    # split-S as clusters merging over distributed shared memory
+    bd.Rule(*ANY, 3, 37, 0, 4),   # balanced grid, deep ring
 ]
 
 
@@ -75,6 +78,7 @@ def test_noalloc_matches_workspace_entry_point(L, lens, H_q, H_kv, D):
         first = _noalloc(L, w, dp, lens_dev)
         second = _noalloc(L, w, dp, lens_dev)  # the scratch now holds the first call's states
         torch.cuda.synchronize()
+        assert bd.noalloc_status() == 0, f"device error after the no-alloc calls, plan {dp.plan}"
         _close(first, ref, f"first call, plan {dp.plan}")
         _close(second, ref, f"second call, plan {dp.plan}")
 
@@ -88,3 +92,24 @@ def test_noalloc_rejects_plans_larger_than_its_scratch(L):
     rc = L.pkv_paged_decode_noalloc(None, None, None, None, None, 16, ctypes.c_float(1.0), None,
                                     ctypes.byref(shape), ctypes.byref(plan), None, None, 5000, None)
     assert rc == -3
+
+
+def test_noalloc_rejected_call_queues_nothing(L):
+    """A call the argument checks reject leaves the scratch as it was: the
+    error word a flagged call left stays readable."""
+    w = to_device(W.make_custom([100, 200], 8, 2, 64, seed=302))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", rules=[bd.Rule(*ANY, 0, 1, 0, 0)])
+    lens_bad = torch.tensor([100, shape.max_pages_per_seq * 16 + 5], dtype=torch.int32, device="cuda")
+    _noalloc(L, w, dp, lens_bad)  # the kernel clamps the length and flags it
+    assert bd.noalloc_status() & 2
+    bad_plan = bd.Plan(1, 0, 0, 0)  # SPLIT_S with no splits: rejected before anything is queued
+    rc = L.pkv_paged_decode_noalloc(
+        w.q.data_ptr(), w.k_pool.data_ptr(), w.v_pool.data_ptr(), w.block_table.data_ptr(), lens_bad.data_ptr(),
+        w.P, ctypes.c_float(w.scale), w.q.data_ptr(), ctypes.byref(dp.shape), ctypes.byref(bad_plan), None, None, 0,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == -1
+    assert bd.noalloc_status() & 2, "a rejected call cleared the scratch"
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
+    _noalloc(L, w, dp, lens)
+    assert bd.noalloc_status() == 0
