@@ -88,6 +88,13 @@ typedef enum {
                                      run as one thread-block cluster and merge their states through
                                      distributed shared memory (no partial states in the workspace,
                                      no merge launch); other modes return PKV_ERR_UNSUPPORTED */
+#define PKV_FLAG_DEVICE_FILL 32   /* WORK_QUEUE only, plan {2, T, 0, flags}: no queue is passed; every
+                                     block derives its own item of the compact queue whose chunk fills
+                                     one wave of T blocks (the fill rule of pkv_select_policy) from the
+                                     device seq_lens, so one plan, or one captured CUDA graph, serves any
+                                     lengths without host planning or a builder kernel.  items / indptr
+                                     may be NULL; n_items (the grid) must be >= max(T, B * H_kv); B <=
+                                     1024; not with PKV_FLAG_SEPARATE_MERGE (PKV_ERR_UNSUPPORTED) */
 
 /* Problem shape and pool layout.  Pool element (page, kv_head, slot, d) of
  * k_pool / v_pool lives at  page*kv_stride_page + kv_head*kv_stride_head +
@@ -116,6 +123,7 @@ typedef struct {
  *   NO_SPLIT:    {0, 1, 0, flags}
  *   SPLIT_S:     {1, S', C, flags}  C = ceil(pages_max / S), S' = ceil(pages_max / C)
  *   WORK_QUEUE:  {2, S', C, flags}  C from the rule,        S' = ceil(pages_max / C)
+ *                {2, T, 0, flags}   with PKV_FLAG_DEVICE_FILL: the fill budget T, C found on the device
  *   BALANCED:    {3, T, 0, flags}   T blocks from the rule's num_splits
  * where pages_max = ceil(N_max / P).  S' is the most chunks any row needs. */
 typedef struct {
@@ -275,6 +283,43 @@ PKV_API int pkv_fill_queue_capacity(const pkv_shape *shape, int32_t n_blocks, in
 PKV_API int pkv_build_fill_queue_device(const int32_t *seq_lens, const pkv_shape *shape, int32_t n_blocks,
                                         pkv_work_item *items, int32_t capacity, int32_t *indptr,
                                         void *workspace, void *stream);
+
+/* Sizes of the prefix-sharing queue (pkv_build_prefix_queue): *n_items
+ * items and *n_units units. */
+PKV_API int pkv_prefix_queue_size(const int32_t *seq_lens_host, const int32_t *block_table_host,
+                                  const pkv_shape *shape, int32_t chunk_pages, int32_t max_members,
+                                  int32_t *n_items, int32_t *n_units);
+
+/* The compact work queue that stages shared prefix pages once for several
+ * rows ["Chapter 8 - Next-generation KV cache management" (actionbridge.io),
+ * 8.1: reference-counted block sharing, best-of-8 over one prompt; 8.3:
+ * prefix caches, whose sharers hold the same physical blocks; PKV,
+ * Methodology 1 "Compact work queue", "Row-local bounds"].
+ *  - Sharing groups: rows with at least one full page and the same first
+ *    physical page in block_table_host (host int32 [B][max_pages_per_seq]);
+ *    the lowest row leads.  A group's shared length L is the number of
+ *    leading entries every member has in common with the leader, counting
+ *    only pages that are full in every member.  Groups of one row or with
+ *    L = 0 are dropped.
+ *  - Items, in lexicographic (row, kv_head) order with pair offsets as in
+ *    pkv_build_work_queue: a grouped row's [0, L*P) is cut into chunks of C
+ *    = chunk_pages pages from 0, then [L*P, N_i) into chunks of C pages from
+ *    L*P; other rows as pkv_build_work_queue.
+ *  - Units (the blocks of the decode grid): for each group, KV head and
+ *    shared chunk, the members' items in row order, in runs of at most
+ *    max_members; every other item is a unit of its own; units ordered by
+ *    their first member.  A unit's members read the same pages, staged once.
+ * indptr (host int32, indptr_capacity >= B*H_kv + 1 + n_units + 1 + n_items
+ * entries) receives the pair offsets, then the unit offsets (n_units + 1),
+ * then the members' item indices unit by unit.  Decode with a WORK_QUEUE plan
+ * carrying PKV_FLAG_SHARED_PREFIX, n_items = the item count (the workspace
+ * sized for that many items); max_members * G must be <= 16.  Capacity
+ * errors as pkv_build_work_queue; PKV_ERR_INVALID for a length past the
+ * table.  Pure host function. */
+PKV_API int pkv_build_prefix_queue(const int32_t *seq_lens_host, const int32_t *block_table_host,
+                                   const pkv_shape *shape, int32_t chunk_pages, int32_t max_members,
+                                   pkv_work_item *items, int32_t capacity, int32_t *indptr,
+                                   int32_t indptr_capacity, int32_t *n_items, int32_t *n_units);
 
 /* Closed-form workload counters of `plan` on this batch (host, pure). */
 PKV_API int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape,

@@ -29,6 +29,9 @@ SPLIT_S = 1
 WORK_QUEUE = 2
 BALANCED = 3  # the compact work queue, cut into equal shares for a fixed number of blocks
 FLAG_SEPARATE_MERGE = 1
+# a work-queue plan whose chunk is found per step from the lengths on the device:
+# the plan carries the fill budget T instead of the chunk, (WORK_QUEUE, T, 0, flags)
+FLAG_DEVICE_FILL = 32
 INT32_MAX = 2**31 - 1
 
 _lib = None
@@ -284,6 +287,114 @@ def build_balanced_queue(seq_lens: Sequence[int], H_kv: int, P: int, n_blocks: i
     return items, indptr, block_ptr
 
 
+def shared_prefixes(seq_lens: Sequence[int], block_table, P: int):
+    """Groups of rows whose block tables start with the same physical pages
+    ["Chapter 8 - Next-generation KV cache management", 8.1: reference-counted
+    block sharing, best-of-8 over one prompt; 8.3: the first thousands of
+    tokens repeat across requests and the block table makes them shared
+    physical blocks].
+
+    Rows with at least one full page and the same first physical page form a
+    group (its lowest row leads); the group's shared length L (pages) is the
+    number of leading table entries every member has in common with the
+    leader, counting only pages that are full in every member, so no member's
+    last, partial page falls inside the shared range.  Returns a list of
+    (rows in ascending order, L) for every group of two or more rows with
+    L >= 1."""
+    lens = [int(n) for n in seq_lens]
+    by_first = {}
+    for i, n in enumerate(lens):
+        if n >= P:
+            by_first.setdefault(int(block_table[i][0]), []).append(i)
+    groups = []
+    for first in sorted(by_first, key=lambda f: by_first[f][0]):
+        rows = by_first[first]
+        if len(rows) < 2:
+            continue
+        lead = rows[0]
+        L = lens[lead] // P
+        for r in rows[1:]:
+            full = lens[r] // P
+            k = 0
+            while k < min(full, L) and int(block_table[r][k]) == int(block_table[lead][k]):
+                k += 1
+            L = min(L, k)
+        if L >= 1:
+            groups.append((rows, L))
+    return groups
+
+
+def build_prefix_queue(seq_lens: Sequence[int], block_table, H_kv: int, P: int, chunk_pages: int,
+                       max_members: int):
+    """Compact work queue that stages shared prefix pages once for several rows.
+
+    Items per (row i, KV head h), in lexicographic order as in
+    build_work_queue: a row in a sharing group (shared_prefixes) with shared
+    length L pages has its shared range [0, L*P) cut into chunks of C pages
+    from 0, then the rest [L*P, N_i) cut into chunks of C pages from L*P;
+    every other row is cut as in build_work_queue.  Row-local, page-aligned
+    bounds as on the pages [PKV, Methodology 1 "Compact work queue",
+    "Row-local bounds"].
+
+    Units (what one block runs): for every group, KV head and shared chunk,
+    the members' items of that chunk, in row order, in runs of at most
+    `max_members`; every other item is a unit of its own.  The members of a
+    unit cover the same tokens of the same KV head on the same physical
+    pages, so one staging of each page serves all of them; each member still
+    gets its own item, i.e. its own partial state, and its pair merges as in
+    the plain queue.  Units are ordered by their first member's item.
+
+    Returns (items, indptr over pairs, unit_ptr of length n_units + 1,
+    unit_items: the members' item indices, unit by unit)."""
+    if chunk_pages < 1 or H_kv < 1 or P < 1 or max_members < 1:
+        raise ValueError("chunk_pages, H_kv, P and max_members must be positive")
+    lens = [int(n) for n in seq_lens]
+    if any(n < 0 for n in lens):
+        raise ValueError("negative sequence length")
+    span = chunk_pages * P
+    shared = {}
+    for g, (rows, L) in enumerate(shared_prefixes(lens, block_table, P)):
+        for r in rows:
+            shared[r] = (g, L)
+    items, indptr = [], [0]
+    chunk_item = {}  # (group, h, shared chunk c, row) -> item index
+    for i, n in enumerate(lens):
+        for h in range(H_kv):
+            if n == 0:
+                items.append((i, h, 0, 0))
+            elif i in shared:
+                g, L = shared[i]
+                c = 0
+                while c * span < L * P:
+                    chunk_item[(g, h, c, i)] = len(items)
+                    items.append((i, h, c * span, min((c + 1) * span, L * P)))
+                    c += 1
+                t = L * P
+                while t < n:
+                    items.append((i, h, t, min(t + span, n)))
+                    t += span
+            else:
+                c = 0
+                while c * span < n:
+                    items.append((i, h, c * span, min((c + 1) * span, n)))
+                    c += 1
+            indptr.append(len(items))
+    grouped = set(chunk_item.values())
+    units = []
+    keys = sorted({k[:3] for k in chunk_item})
+    for key in keys:
+        members = [chunk_item[key + (r,)] for r in sorted(r for (g, h, c, r) in chunk_item if (g, h, c) == key)]
+        for k in range(0, len(members), max_members):
+            units.append(members[k:k + max_members])
+    units += [[x] for x in range(len(items)) if x not in grouped]
+    units.sort(key=lambda u: u[0])
+    unit_ptr, unit_items = [0], []
+    for u in units:
+        unit_items += u
+        unit_ptr.append(len(unit_items))
+    return items, indptr, unit_ptr, unit_items
+
+
 @dataclass(frozen=True)
 class Rule:
     """One row of a policy table: half-open ranges on B and N_max -> a plan."""
@@ -310,6 +421,8 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule], H_kv: 
                      a rule with chunk_pages = 0 asks for the smallest C whose
                      queue has at most T = num_splits items (pages_max if none)
       BALANCED    -> T blocks from the rule's num_splits:              (3, T, 0, flags)
+      a WORK_QUEUE rule with FLAG_DEVICE_FILL leaves the chunk to the device:
+                     its fill budget T as given                         (2, T, 0, flags)
     where pages_max = ceil(N_max / P).
     """
     if P < 1:
@@ -328,6 +441,8 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule], H_kv: 
             raise ValueError("SPLIT_S and BALANCED rules need num_splits >= 1")
         if r.mode == WORK_QUEUE and (r.chunk_pages < 0 or (r.chunk_pages == 0 and r.num_splits < 1)):
             raise ValueError("WORK_QUEUE rule needs chunk_pages >= 1, or 0 with num_splits >= 1")
+        if r.flags & FLAG_DEVICE_FILL and (r.mode != WORK_QUEUE or r.chunk_pages != 0):
+            raise ValueError("a device-fill rule is a WORK_QUEUE rule with chunk_pages = 0")
         if chosen is None and r.b_lo <= B < r.b_hi and r.nmax_lo <= n_max < r.nmax_hi:
             chosen = r
     if chosen is None or B == 0 or pages_max == 0:
@@ -336,6 +451,8 @@ def select_policy(seq_lens: Sequence[int], P: int, rules: Sequence[Rule], H_kv: 
         return (NO_SPLIT, 1, 0, chosen.flags)
     if chosen.mode == BALANCED:
         return (BALANCED, chosen.num_splits, 0, chosen.flags)
+    if chosen.flags & FLAG_DEVICE_FILL:
+        return (WORK_QUEUE, chosen.num_splits, 0, chosen.flags)
     if chosen.mode == SPLIT_S:
         C = _ceil_div(pages_max, chosen.num_splits)
     elif chosen.chunk_pages > 0:
@@ -401,7 +518,8 @@ def counters(seq_lens: Sequence[int], H_q: int, H_kv: int, D: int, P: int, plan)
       2 * slots * G * (D + 2) * 4 over every (row, head) pair with more than one slot;
     kv_bytes: K and V of the valid tokens; kv_bytes_streamed: whole pages;
     queue_bytes: items (16 B each) plus indptr (4 B per pair, +4; for BALANCED
-      also 4 B per block, +4) sent to the device;
+      also 4 B per block, +4) sent to the device; none for a device-fill plan,
+      whose blocks derive their items (counted at the chunk they find);
     bucket_launches: exact-length bucketing, one split and one merge launch per
       distinct non-zero length [PKV, Results: "16.00 -> 2.00 launches per step"].
     """
@@ -424,11 +542,21 @@ def counters(seq_lens: Sequence[int], H_q: int, H_kv: int, D: int, P: int, plan)
         qbytes = 0
         launches = 1 + (1 if flags & FLAG_SEPARATE_MERGE else 0)
     elif mode == WORK_QUEUE:
+        device_fill = bool(flags & FLAG_DEVICE_FILL)
+        if device_fill:
+            # the chunk the device finds for these lengths: the fill rule with budget T = S
+            pages_max = max(pages, default=0)
+            C = pages_max
+            for c in range(1, pages_max + 1):
+                if fill_items(lens, H_kv, P, c) <= S:
+                    C = c
+                    break
+            C = max(C, 1)
         per_pair = [max(1, _ceil_div(p, C)) for p in pages]
         work = H_kv * sum(per_pair)
         empty = H_kv * sum(1 for n in lens if n == 0)
         merge = 2 * H_kv * sum(k for k in per_pair if k > 1) * state
-        qbytes = 16 * work + 4 * (B * H_kv + 1)
+        qbytes = 0 if device_fill else 16 * work + 4 * (B * H_kv + 1)
         launches = 1 + (1 if flags & FLAG_SEPARATE_MERGE else 0)
     elif mode == BALANCED:
         items, indptr, _ = build_balanced_queue(lens, H_kv, P, S)

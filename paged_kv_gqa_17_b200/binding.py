@@ -21,6 +21,8 @@ LIB_PATH = os.path.join(HERE, "libpkv.so")
 
 NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED = 0, 1, 2, 3
 FLAG_SEPARATE_MERGE, FLAG_NO_PDL, FLAG_DEEP_RING, FLAG_CLUSTER_MERGE, FLAG_PDL_EARLY = 1, 2, 4, 8, 16
+FLAG_DEVICE_FILL = 32
+FILL_MAX_ROWS = 1024  # rows a device-fill plan can plan for on the device
 INT32_MAX = 2**31 - 1
 _MODE_NAMES = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE, "BALANCED": BALANCED}
 
@@ -96,6 +98,8 @@ SIGNATURES = [
     ("pkv_build_balanced_queue_device", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p, c_p]),
     ("pkv_fill_queue_capacity", ctypes.c_int, [c_p, c_i32, c_p]),
     ("pkv_build_fill_queue_device", ctypes.c_int, [c_p, c_p, c_i32, c_p, c_i32, c_p, c_p, c_p]),
+    ("pkv_prefix_queue_size", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_i32, c_p, c_p]),
+    ("pkv_build_prefix_queue", ctypes.c_int, [c_p, c_p, c_p, c_i32, c_i32, c_p, c_i32, c_p, c_i32, c_p, c_p]),
     ("pkv_plan_counters", ctypes.c_int, [c_p, c_p, c_p, c_p]),
     ("pkv_workspace_bytes", ctypes.c_int, [c_p, c_p, c_i32, c_p]),
     ("pkv_workspace_init", ctypes.c_int, [c_p, c_sz, c_p]),
@@ -354,6 +358,25 @@ def build_balanced_queue(seq_lens_host, shape: Shape, n_blocks: int):
     return items[:n.value], indptr
 
 
+def build_prefix_queue(seq_lens_host, block_table_host, shape: Shape, chunk_pages: int, max_members: int):
+    """-> (items int32 [n][4], indptr int32: pair offsets [B*H_kv + 1], unit offsets
+    [n_units + 1], the units' member item indices [n]; n_units).  The queue that
+    stages shared prefix pages once for several rows (pkv_build_prefix_queue)."""
+    L = lib()
+    lens, _ = _lens_array(seq_lens_host)
+    bt = torch.as_tensor(block_table_host, dtype=torch.int32).cpu().contiguous()
+    n, u = c_i32(0), c_i32(0)
+    _check(L.pkv_prefix_queue_size(lens, bt.data_ptr(), ctypes.byref(shape), chunk_pages, max_members,
+                                   ctypes.byref(n), ctypes.byref(u)), "pkv_prefix_queue_size")
+    items = torch.zeros((max(1, n.value), 4), dtype=torch.int32)
+    n_ptr = shape.B * shape.H_kv + 1 + u.value + 1 + n.value
+    indptr = torch.zeros(n_ptr, dtype=torch.int32)
+    _check(L.pkv_build_prefix_queue(lens, bt.data_ptr(), ctypes.byref(shape), chunk_pages, max_members,
+                                    items.data_ptr(), n.value, indptr.data_ptr(), n_ptr, ctypes.byref(n),
+                                    ctypes.byref(u)), "pkv_build_prefix_queue")
+    return items[:n.value], indptr, int(u.value)
+
+
 def balanced_queue_capacity(shape: Shape, n_blocks: int) -> int:
     L = lib()
     n = c_i32(0)
@@ -414,8 +437,9 @@ class DecodePlan:
     """Everything a decode step needs besides the tensors: the plan, the queue
     on the device (WORK_QUEUE, BALANCED) and a zeroed workspace.  Reusable for
     every step with the same sequence lengths and shape; with device_queue
-    (BALANCED only) the queue is rebuilt on the GPU from the device lengths at
-    every step, so the plan serves any lengths up to the shape's maximum."""
+    the queue comes from the device lengths at every step (built by a kernel
+    of its own, or derived by each decode block under PKV_FLAG_DEVICE_FILL),
+    so the plan serves any lengths up to the shape's maximum."""
 
     shape: Shape
     plan: Plan
@@ -429,19 +453,36 @@ class DecodePlan:
 
 
 def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[Plan] = None,
-                device_queue: bool = False, fill_blocks: int = 296) -> DecodePlan:
+                device_queue: bool = False, fill_blocks: int = 296,
+                device_fill: Optional[bool] = None) -> DecodePlan:
     """Host planning for one batch: policy (unless `plan` is given), queue, workspace.
 
     device_queue=True leaves the queue to the GPU, rebuilt from the device
     lengths by every paged_decode call (so one plan, or one captured CUDA
     graph, serves any lengths up to the shape's maximum): a BALANCED plan
     gets the balanced queue of its T blocks, a WORK_QUEUE plan the queue
-    whose chunk fills one wave of `fill_blocks` blocks.  NO_SPLIT and
-    SPLIT_S plans have no queue and read the lengths on the device anyway;
-    they serve lengths up to those they were planned for (SPLIT_S: S' chunks
-    of C pages)."""
+    whose chunk fills one wave of `fill_blocks` blocks.  For the latter the
+    decode blocks derive their own items (PKV_FLAG_DEVICE_FILL, one launch)
+    where the plan allows it (B <= 1024, merge fused); device_fill=False
+    asks for the builder kernel instead.  NO_SPLIT and SPLIT_S plans have no
+    queue and read the lengths on the device anyway; they serve lengths up
+    to those they were planned for (SPLIT_S: S' chunks of C pages)."""
     if plan is None:
         plan = select_policy(seq_lens_host, shape, rules)
+    if plan.mode == WORK_QUEUE and plan.flags & FLAG_DEVICE_FILL:
+        device_queue, device_fill, fill_blocks = True, True, plan.num_splits
+    if device_queue and plan.mode == WORK_QUEUE:
+        fill_ok = shape.B <= FILL_MAX_ROWS and not plan.flags & FLAG_SEPARATE_MERGE
+        if device_fill is None:
+            device_fill = fill_ok
+        if device_fill:
+            if not fill_ok:
+                raise ValueError("a device-fill plan needs B <= 1024 and the fused merge")
+            dplan = Plan(WORK_QUEUE, fill_blocks, 0, plan.flags | FLAG_DEVICE_FILL)
+            cap = max(fill_blocks, shape.B * shape.H_kv)
+            ws = torch.zeros(workspace_bytes(shape, dplan, cap), dtype=torch.uint8, device=device)
+            return DecodePlan(shape, dplan, None, None, cap, ws, plan_counters(seq_lens_host, shape, dplan), True,
+                              fill_blocks)
     if device_queue and plan.mode in (WORK_QUEUE, BALANCED):
         pairs = shape.B * shape.H_kv
         if plan.mode == BALANCED:
@@ -494,6 +535,8 @@ def paged_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, bl
     if plan.device_queue and plan.plan.mode == BALANCED:
         build_balanced_queue_device(seq_lens, shape, plan.plan.num_splits, plan.items, plan.indptr, plan.workspace,
                                     stream)
+    elif plan.device_queue and plan.plan.flags & FLAG_DEVICE_FILL:
+        pass  # every decode block derives its own item from the device lengths
     elif plan.device_queue:
         build_fill_queue_device(seq_lens, shape, plan.fill_blocks, plan.items, plan.indptr, plan.workspace, stream)
     rc = L.pkv_paged_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),

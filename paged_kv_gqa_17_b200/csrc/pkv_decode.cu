@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <climits>
@@ -91,6 +92,8 @@ struct __align__(64) Params {
     int32_t pdl_early;  // may read lengths, table and KV pages (but a row's last) before the dependency wait
     int32_t n_items;
     int32_t prefetch_blocks;  // blocks below this index warm L2 before the wait (the grid's first wave)
+    int32_t device_fill;      // WORK_QUEUE: every block derives its own item from the device lengths
+    int32_t fill_blocks;      // ... of the queue whose chunk fills one wave of this many blocks
 #ifdef PKV_TRACE
     int32_t trace_epoch;
 #endif
@@ -943,6 +946,206 @@ __device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lan
 #endif
 }
 
+// L2 prefetch of pages [pg0, pg_end) of (row, KV head h), at most
+// PKV_L2_PREFETCH_PAGES of them, one page per lane of the calling warp; the
+// block-table entries are read speculatively through L2 (see above).
+template <int D>
+__device__ __forceinline__ void l2_prefetch_range(const Params &p, int lane, int row, int h, int64_t pg0,
+                                                  int64_t pg_end)
+{
+#if PKV_L2_PREFETCH_PAGES > 0
+    const int64_t j = pg0 + lane;
+    if (lane < PKV_L2_PREFETCH_PAGES && j < pg_end && j < p.max_pages) {
+        const int e = ld_l2_only(p.block_table + (int64_t)row * p.max_pages + j);
+        if (e >= 0 && e < p.num_pool_pages) {
+            tma_prefetch_page_l2<D>(&p.tm_k, h, e);
+            tma_prefetch_page_l2<D>(&p.tm_v, h, e);
+        }
+    }
+#endif
+}
+
+// Rows a block can plan for itself (PKV_FLAG_DEVICE_FILL): the derivation
+// keeps three int32 per row in the idle shared-memory ring.
+constexpr int kFillMaxRows = 1024;
+
+struct FillItem {
+    int row, h, tb, te, slot0, nslots, len;
+    bool valid;
+};
+
+__device__ __forceinline__ int warp_sum_i32(int v)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+__device__ __forceinline__ int warp_max_i32(int v)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+
+// The compact work queue whose chunk fills one wave of T = p.fill_blocks
+// blocks [PKV, Methodology 1 "Compact work queue", "Row-local bounds"; the
+// fill rule is this library's], derived by each block for itself from the
+// device lengths, so that no builder kernel runs before the decode: the
+// same items, in the same (row, KV head, chunk) order, as
+// pkv_build_work_queue at the chunk C that pkv_select_policy's fill rule
+// picks.  C is the smallest chunk (pages) with
+//   count(C) = H_kv * sum_i max(1, ceil(pages_i / C)) <= T,
+// or pages_max when one item per (row, KV head) already exceeds T.  Since
+// ceil(x) lies in [x, x + 1), C lies in [ceil(H_kv * U / T),
+// ceil(H_kv * U / (T - H_kv * B))] (U = sum_i pages_i); every thread tests
+// one candidate of that range at a time, so the search takes one round
+// whenever the range holds no more candidates than the block has threads.
+// Then a prefix sum over the rows' chunk counts places block b's item.
+// Called by every thread of the block (it has block-wide barriers); `sm`
+// holds 3 * B + 5 int32 of shared memory that nothing else uses meanwhile.
+// speculative: lengths read through L2 before the dependency wait, for the
+// L2 prefetch only; no error is recorded.
+template <int NTHREADS>
+__device__ FillItem fill_queue_item(const Params &p, int32_t *sm, bool speculative)
+{
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int B = p.B;
+    int32_t *pages = sm;            // [B]
+    int32_t *lens = sm + B;         // [B] (clamped)
+    int32_t *rs = sm + 2 * B;       // [B + 1]: items of one KV head before row i
+    int32_t *red = sm + 3 * B + 1;  // [4]: pages_max, sum of pages, best candidate (two rounds' slots)
+    const int64_t cap = (int64_t)p.max_pages * kPage;
+    __syncthreads();  // every thread is done with sm
+    if (tid == 0) {
+        red[0] = 0;
+        red[1] = 0;
+        red[2] = INT_MAX;
+        red[3] = INT_MAX;
+    }
+    __syncthreads();
+    int lmax = 0, lsum = 0;
+    for (int i = tid; i < B; i += NTHREADS) {
+        int N = speculative ? ld_l2_only(p.seq_lens + i) : __ldg(p.seq_lens + i);
+        if (N < 0 || N > cap) {
+            if (!speculative)
+                atomicOr(p.ws_error, kErrSeqLen);
+            N = N < 0 ? 0 : (int)cap;
+        }
+        const int pg = (N + kPage - 1) / kPage;
+        lens[i] = N;
+        pages[i] = pg;
+        lmax = max(lmax, pg);
+        lsum += pg;
+    }
+    lmax = warp_max_i32(lmax);
+    lsum = warp_sum_i32(lsum);
+    if (lane == 0 && (lmax > 0 || lsum > 0)) {
+        atomicMax(&red[0], lmax);
+        atomicAdd(&red[1], lsum);
+    }
+    __syncthreads();
+    const int pmax = red[0];
+    const int64_t U = red[1];
+    const int64_t T = p.fill_blocks;
+    const int64_t HB = (int64_t)p.H_kv * B;
+    int64_t C;
+    if (pmax == 0) {
+        C = 1;  // every row is empty: one empty item per (row, KV head)
+    } else if (HB > T) {
+        C = pmax;
+    } else {
+        int64_t lo = (p.H_kv * U + T - 1) / T;
+        int64_t hi = HB < T ? (p.H_kv * U + (T - HB) - 1) / (T - HB) : pmax;
+        lo = lo < 1 ? 1 : (lo > pmax ? pmax : lo);
+        hi = hi > pmax ? pmax : (hi < lo ? lo : hi);
+        // hi satisfies the rule (count(hi) <= T); find the smallest that does
+        for (int round = 0; lo < hi; ++round) {
+            const int64_t step = (hi - lo + NTHREADS) / NTHREADS;
+            const int64_t c = lo + (int64_t)tid * step;
+            int32_t *best = red + 2 + (round & 1);
+            if (c < hi) {
+                const uint32_t cu = (uint32_t)c;
+                int64_t n = 0;
+                for (int i = 0; i < B && n * p.H_kv <= T; ++i) {
+                    const uint32_t k = ((uint32_t)pages[i] + cu - 1) / cu;
+                    n += k > 1 ? k : 1;
+                }
+                if (n * p.H_kv <= T)
+                    atomicMin(best, (int)c);
+            }
+            if (tid == 0)
+                red[2 + ((round + 1) & 1)] = INT_MAX;  // the next round's slot
+            __syncthreads();
+            const int64_t b = *best < hi ? *best : hi;
+            lo = b - step + 1 > lo ? b - step + 1 : lo;
+            hi = b;
+            __syncthreads();  // every thread has read this round's slot
+        }
+        C = lo;
+    }
+    // one KV head's item offsets per row (one warp scans the rows)
+    if (tid < 32) {
+        int carry = 0;
+        for (int base = 0; base < B; base += 32) {
+            const int i = base + lane;
+            int cnt = 0;
+            if (i < B) {
+                const int k = (int)(((int64_t)pages[i] + C - 1) / C);
+                cnt = k > 1 ? k : 1;
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int add = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off)
+                    incl += add;
+            }
+            if (i < B)
+                rs[i] = carry + incl - cnt;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0)
+            rs[B] = carry;
+    }
+    fence_proxy_async_smem();  // these generic writes precede later TMA writes into the ring
+    __syncthreads();
+    FillItem f;
+    f.valid = false;
+    f.row = f.h = f.tb = f.te = f.slot0 = f.len = 0;
+    f.nslots = 1;
+    const int64_t b = blockIdx.x;
+    if (b >= (int64_t)rs[B] * p.H_kv)
+        return f;  // past the queue: nothing to do for this block
+    int lo = 0, hi = B - 1;  // the last row whose items start at or before b
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)rs[mid] * p.H_kv <= b)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const int i = lo;
+    const int cnt = rs[i + 1] - rs[i];
+    const int64_t j = b - (int64_t)rs[i] * p.H_kv;
+    const int h = (int)(j / cnt);
+    const int c = (int)(j % cnt);
+    const int N = lens[i];
+    const int64_t span = C * kPage;
+    f.row = i;
+    f.h = h;
+    f.len = N;
+    f.tb = N > 0 ? (int)(c * span) : 0;
+    f.te = N > 0 ? (int)((c + 1) * span < N ? (c + 1) * span : N) : 0;
+    f.slot0 = (int)((int64_t)rs[i] * p.H_kv + (int64_t)h * cnt);
+    f.nslots = cnt;
+    f.valid = true;
+    return f;
+}
+
 // One block = one work item (row, KV head, token range) for all G query heads.
 // The deep-ring variants (two blocks per SM at most, by shared memory) tell
 // the compiler so.  With that hint the D = 128, G <= 8 variants come out at
@@ -995,10 +1198,21 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     int4 *spec_item = reinterpret_cast<int4 *>(smem + C::kMiscOff + 32);
     if (tid == 0)
         *spec_item = make_int4(-1, 0, 0, 0);
+    int32_t *fill_scratch = reinterpret_cast<int32_t *>(smem);  // the idle ring, before any page copy
     if (!p.pdl_early) {
         __syncthreads();
-        if (warp == NW && (int)blockIdx.x < p.prefetch_blocks)
+        const bool warm = (int)blockIdx.x < p.prefetch_blocks;
+        if (p.mode == PKV_WORK_QUEUE && p.device_fill) {
+            if (warm) {
+                const FillItem g = fill_queue_item<C::kThreads>(p, fill_scratch, true);
+                if (g.valid && tid == 0)
+                    *spec_item = make_int4(g.row, g.h, g.tb, g.te);
+                if (g.valid && warp == NW)
+                    l2_prefetch_range<D>(p, lane, g.row, g.h, g.tb / kPage, (g.te + kPage - 1) / kPage);
+            }
+        } else if (warp == NW && warm) {
             l2_prefetch_first_pages<D>(p, lane, row_cap, spec_item);
+        }
         __syncthreads();
         grid_dependency_wait();
     }
@@ -1011,7 +1225,40 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     int e_first = 0;
     bool hit = false;  // the guessed work item was the real one
     int row_len = -1;  // the row's length where known (for the early dependency gate)
-    if (p.mode == PKV_WORK_QUEUE) {
+    if (p.mode == PKV_WORK_QUEUE && p.device_fill) {
+        // the block's own item, derived from the device lengths; the
+        // table entries at the guessed item's first page go out first
+        const int4 guess = p.pdl_early ? make_int4(-1, 0, 0, 0) : *spec_item;
+        int g_entry = 0;
+        if (guess.x >= 0 && warp == NW) {
+            const int idx = guess.z / kPage + lane;
+            if (idx < p.max_pages)
+                g_entry = __ldg(p.block_table + (int64_t)guess.x * p.max_pages + idx);
+        }
+        const FillItem f = fill_queue_item<C::kThreads>(p, fill_scratch, false);
+        if (!f.valid)
+            return;
+        hit = guess.x == f.row && guess.y == f.h && guess.z == f.tb && guess.w == f.te;
+        row = f.row;
+        h = f.h;
+        tb = f.tb;
+        te = f.te;
+        slot0 = f.slot0;
+        nslots = f.nslots;
+        my_slot = blockIdx.x;
+        e_first = g_entry;
+        if (slot0 + nslots > p.n_items) {
+            if (tid == 0)
+                atomicOr(p.ws_error, kErrItem);
+            return;
+        }
+        if (warp == NW) {
+            const int idx = tb / kPage + lane;
+            if (!hit && idx < p.max_pages)
+                e_first = __ldg(p.block_table + (int64_t)row * p.max_pages + idx);
+            row_len = f.len;
+        }
+    } else if (p.mode == PKV_WORK_QUEUE) {
         // a queue built on the device may hold fewer items than the grid has
         // blocks (the buffer holds one per block); the item, the item count
         // and the loads at the guessed item's addresses go out at once
@@ -2383,9 +2630,21 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         return PKV_ERR_INVALID;
     if (pl.mode == PKV_SPLIT_S && (pl.num_splits < 1 || pl.chunk_pages < 1))
         return PKV_ERR_INVALID;
-    if ((pl.mode == PKV_WORK_QUEUE || pl.mode == PKV_BALANCED) &&
-        (!items || !indptr || n_items < (int64_t)s.B * s.H_kv))
+    const bool device_fill = (pl.flags & PKV_FLAG_DEVICE_FILL) != 0;
+    if (device_fill) {
+        // each block derives its item: the grid must hold the longest queue the fill rule allows
+        if (pl.mode != PKV_WORK_QUEUE || (pl.flags & PKV_FLAG_SEPARATE_MERGE) || s.B > kFillMaxRows)
+            return PKV_ERR_UNSUPPORTED;
+        if (pl.num_splits < 1 || pl.chunk_pages != 0)
+            return PKV_ERR_INVALID;
+        if ((int64_t)s.B * s.max_pages_per_seq * s.H_kv > INT32_MAX)
+            return PKV_ERR_UNSUPPORTED;
+        if (n_items < std::max<int64_t>(pl.num_splits, (int64_t)s.B * s.H_kv))
+            return PKV_ERR_INVALID;
+    } else if ((pl.mode == PKV_WORK_QUEUE || pl.mode == PKV_BALANCED) &&
+               (!items || !indptr || n_items < (int64_t)s.B * s.H_kv)) {
         return PKV_ERR_INVALID;
+    }
     if (pl.mode == PKV_BALANCED && pl.num_splits < 1)
         return PKV_ERR_INVALID;
     if ((pl.flags & PKV_FLAG_CLUSTER_MERGE) && (pl.mode != PKV_SPLIT_S || pl.num_splits > 16))
@@ -2449,6 +2708,8 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.separate_merge = (pl.flags & PKV_FLAG_SEPARATE_MERGE) ? 1 : 0;
     prm.pdl_early = (pl.flags & PKV_FLAG_PDL_EARLY) && !(pl.flags & PKV_FLAG_NO_PDL) ? 1 : 0;
     prm.n_items = n_items;
+    prm.device_fill = device_fill ? 1 : 0;
+    prm.fill_blocks = device_fill ? pl.num_splits : 0;
 #ifdef PKV_TRACE
     static std::atomic<int32_t> trace_launches{0};
     prm.trace_epoch = trace_launches.fetch_add(1);
@@ -2734,7 +2995,10 @@ int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_ru
     const size_t pairs = (size_t)s.B * s.H_kv;
     L->n_items = 0;
     L->n_indptr = 0;
-    if (L->plan.mode == PKV_WORK_QUEUE) {
+    if (L->plan.mode == PKV_WORK_QUEUE && (L->plan.flags & PKV_FLAG_DEVICE_FILL)) {
+        // no queue travels: the blocks derive their items; the grid holds the longest queue
+        L->n_items = (int32_t)std::max<int64_t>(L->plan.num_splits, (int64_t)pairs);
+    } else if (L->plan.mode == PKV_WORK_QUEUE) {
         rc = pkv_work_queue_size(lens, shape, L->plan.chunk_pages, &L->n_items);
         L->n_indptr = (int32_t)pairs + 1;
     } else if (L->plan.mode == PKV_BALANCED) {
@@ -2757,7 +3021,7 @@ int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_ru
     };
     L->q_off = L->q_inline ? take(L->q_bytes) : 0;
     L->lens_off = take((size_t)s.B * 4);
-    L->items_off = take((size_t)L->n_items * sizeof(pkv_work_item));
+    L->items_off = take(L->n_indptr > 0 ? (size_t)L->n_items * sizeof(pkv_work_item) : 0);
     L->indptr_off = take((size_t)L->n_indptr * 4);
     L->bt_off = L->bt_inline ? take(L->bt_bytes) : 0;
     L->counters_off = take(ws.m_off - ws.counters_off);
@@ -2876,7 +3140,7 @@ int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, c
     pkv_work_item *h_items = reinterpret_cast<pkv_work_item *>(hst + L.items_off);
     int32_t *h_indptr = reinterpret_cast<int32_t *>(hst + L.indptr_off);
     int32_t n = 0;
-    if (L.plan.mode == PKV_WORK_QUEUE)
+    if (L.plan.mode == PKV_WORK_QUEUE && !(L.plan.flags & PKV_FLAG_DEVICE_FILL))
         rc = pkv_build_work_queue(seq_lens_host, shape, L.plan.chunk_pages, h_items, L.n_items, h_indptr, &n);
     else if (L.plan.mode == PKV_BALANCED)
         rc = pkv_build_balanced_queue(seq_lens_host, shape, L.plan.num_splits, h_items, L.n_items, h_indptr, &n);

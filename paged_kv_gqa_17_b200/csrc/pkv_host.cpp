@@ -59,6 +59,8 @@ int check_rules(const pkv_policy_rule *rules, int32_t n)
             return PKV_ERR_INVALID;
         if (r.mode == PKV_WORK_QUEUE && (r.chunk_pages < 0 || (r.chunk_pages == 0 && r.num_splits < 1)))
             return PKV_ERR_INVALID;
+        if ((r.flags & PKV_FLAG_DEVICE_FILL) && (r.mode != PKV_WORK_QUEUE || r.chunk_pages != 0))
+            return PKV_ERR_INVALID;
     }
     return PKV_OK;
 }
@@ -162,6 +164,10 @@ int pkv_select_policy(const int32_t *seq_lens_host, const pkv_shape *shape,
     }
     if (chosen->mode == PKV_BALANCED) {
         *plan = {PKV_BALANCED, chosen->num_splits, 0, chosen->flags};
+        return PKV_OK;
+    }
+    if (chosen->flags & PKV_FLAG_DEVICE_FILL) {  // the chunk is found on the device, per step
+        *plan = {PKV_WORK_QUEUE, chosen->num_splits, 0, chosen->flags};
         return PKV_OK;
     }
     const int64_t C = chosen->mode == PKV_SPLIT_S ? ceil_div(pages_max, chosen->num_splits)
@@ -381,12 +387,22 @@ int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, cons
         break;
     }
     case PKV_WORK_QUEUE: {
-        if (C < 1)
+        const bool device_fill = (plan->flags & PKV_FLAG_DEVICE_FILL) != 0;
+        int64_t Cq = C;
+        if (device_fill) {  // the chunk the blocks find on the device for these lengths
+            if (S < 1 || C != 0)
+                return PKV_ERR_INVALID;
+            int64_t pages_max = 0;
+            for (int64_t i = 0; i < B; ++i)
+                pages_max = std::max<int64_t>(pages_max, ceil_div(seq_lens_host[i], P));
+            Cq = pages_max == 0 ? 1 : fill_chunk(seq_lens_host, *shape, pages_max, S);
+        }
+        if (Cq < 1)
             return PKV_ERR_INVALID;
         out.launches = 1 + separate;
         int64_t items = 0, multi = 0;
         for (int64_t i = 0; i < B; ++i) {
-            const int64_t k = std::max<int64_t>(1, ceil_div(ceil_div(seq_lens_host[i], P), C));
+            const int64_t k = std::max<int64_t>(1, ceil_div(ceil_div(seq_lens_host[i], P), Cq));
             items += k;
             if (k > 1)
                 multi += k;
@@ -394,7 +410,7 @@ int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, cons
         out.work_items = H_kv * items;
         out.empty_items = H_kv * zero_rows;
         out.merge_state_bytes = 2 * H_kv * multi * state;
-        out.queue_bytes = 16 * out.work_items + 4 * (B * H_kv + 1);
+        out.queue_bytes = device_fill ? 0 : 16 * out.work_items + 4 * (B * H_kv + 1);
         break;
     }
     case PKV_BALANCED: {
@@ -435,6 +451,192 @@ int pkv_workspace_bytes(const pkv_shape *shape, const pkv_plan *plan, int32_t n_
     if (plan->mode == PKV_SPLIT_S && plan->num_splits < 1)
         return PKV_ERR_INVALID;
     *bytes = ws_layout(*shape, *plan, n_items).total;
+    return PKV_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Prefix-sharing work queue ["Chapter 8 - Next-generation KV cache management"
+// (actionbridge.io), 8.1 reference-counted block sharing and 8.3 prefix
+// caches: rows whose block tables start with the same physical pages; PKV,
+// Methodology 1 "Compact work queue", "Row-local bounds"].
+
+namespace pkv {
+namespace {
+
+// Sharing groups of a batch: rows with at least one full page grouped by
+// their first physical page (the lowest row leads); a group's shared length
+// is the number of leading table entries every member has in common with
+// the leader, counting only pages that are full in every member.  Groups of
+// one row, or with no shared page, are dropped.  group_of[i] = the group of
+// row i or -1; shared[g] = its length in pages; rows[g] = its rows, ascending.
+struct PrefixGroups {
+    std::vector<int32_t> group_of;
+    std::vector<int64_t> shared;
+    std::vector<std::vector<int32_t>> rows;
+};
+
+PrefixGroups prefix_groups(const int32_t *lens, const int32_t *bt, const pkv_shape &s)
+{
+    const int64_t P = s.page_size, W = s.max_pages_per_seq;
+    PrefixGroups g;
+    g.group_of.assign((size_t)s.B, -1);
+    std::vector<std::pair<int32_t, int32_t>> firsts;  // (first page, row) of rows with a full page
+    for (int32_t i = 0; i < s.B; ++i)
+        if (lens[i] >= P && W > 0)
+            firsts.push_back({bt[(int64_t)i * W], i});
+    std::stable_sort(firsts.begin(), firsts.end(),
+                     [](const std::pair<int32_t, int32_t> &a, const std::pair<int32_t, int32_t> &b) {
+                         return a.first < b.first;
+                     });
+    std::vector<std::vector<int32_t>> cand;
+    for (size_t k = 0; k < firsts.size();) {
+        size_t e = k;
+        std::vector<int32_t> rows;
+        while (e < firsts.size() && firsts[e].first == firsts[k].first)
+            rows.push_back(firsts[e++].second);
+        if (rows.size() >= 2)
+            cand.push_back(rows);  // rows ascending (stable sort of ascending rows)
+        k = e;
+    }
+    // groups in the order of their leading row
+    std::sort(cand.begin(), cand.end(),
+              [](const std::vector<int32_t> &a, const std::vector<int32_t> &b) { return a[0] < b[0]; });
+    for (const std::vector<int32_t> &rows : cand) {
+        const int32_t lead = rows[0];
+        int64_t L = std::min<int64_t>(lens[lead] / P, W);
+        for (size_t m = 1; m < rows.size(); ++m) {
+            const int64_t full = std::min<int64_t>(lens[rows[m]] / P, W);
+            int64_t k = 0;
+            while (k < std::min(full, L) && bt[(int64_t)rows[m] * W + k] == bt[(int64_t)lead * W + k])
+                ++k;
+            L = std::min(L, k);
+        }
+        if (L < 1)
+            continue;
+        for (int32_t r : rows)
+            g.group_of[(size_t)r] = (int32_t)g.rows.size();
+        g.shared.push_back(L);
+        g.rows.push_back(rows);
+    }
+    return g;
+}
+
+// Walks the prefix-sharing queue: item counts per (row, head) and, for a
+// grouped row, how many of its first items are shared chunks.
+int64_t prefix_row_items(int64_t n, int64_t L, int64_t span, int64_t P, int64_t *shared_chunks)
+{
+    if (n == 0) {
+        *shared_chunks = 0;
+        return 1;
+    }
+    const int64_t sc = ceil_div(L * P, span);
+    *shared_chunks = sc;
+    return sc + ceil_div(n - L * P, span);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+int pkv_prefix_queue_size(const int32_t *seq_lens_host, const int32_t *block_table_host, const pkv_shape *shape,
+                          int32_t chunk_pages, int32_t max_members, int32_t *n_items, int32_t *n_units)
+{
+    if (!n_items || !n_units || chunk_pages < 1 || max_members < 1 || check_shape(shape) != PKV_OK)
+        return PKV_ERR_INVALID;
+    int rc = check_lens(seq_lens_host, shape->B);
+    if (rc != PKV_OK)
+        return rc;
+    if (shape->B > 0 && shape->max_pages_per_seq > 0 && !block_table_host)
+        return PKV_ERR_INVALID;
+    for (int32_t i = 0; i < shape->B; ++i)
+        if ((int64_t)seq_lens_host[i] > (int64_t)shape->max_pages_per_seq * shape->page_size)
+            return PKV_ERR_INVALID;
+    const PrefixGroups g = prefix_groups(seq_lens_host, block_table_host, *shape);
+    const int64_t P = shape->page_size, span = (int64_t)chunk_pages * P;
+    int64_t items = 0, merged = 0;
+    for (int32_t i = 0; i < shape->B; ++i) {
+        const int32_t gi = g.group_of[(size_t)i];
+        int64_t sc = 0;
+        items += shape->H_kv * prefix_row_items(seq_lens_host[i], gi >= 0 ? g.shared[(size_t)gi] : 0, span, P, &sc);
+    }
+    for (size_t k = 0; k < g.rows.size(); ++k) {
+        const int64_t m = (int64_t)g.rows[k].size();
+        merged += shape->H_kv * ceil_div(g.shared[k] * P, span) * (m - ceil_div(m, max_members));
+    }
+    if (items > INT32_MAX)
+        return PKV_ERR_CAPACITY;
+    *n_items = (int32_t)items;
+    *n_units = (int32_t)(items - merged);
+    return PKV_OK;
+}
+
+int pkv_build_prefix_queue(const int32_t *seq_lens_host, const int32_t *block_table_host, const pkv_shape *shape,
+                           int32_t chunk_pages, int32_t max_members, pkv_work_item *items, int32_t capacity,
+                           int32_t *indptr, int32_t indptr_capacity, int32_t *n_items, int32_t *n_units)
+{
+    int32_t need = 0, units = 0;
+    int rc = pkv_prefix_queue_size(seq_lens_host, block_table_host, shape, chunk_pages, max_members, &need, &units);
+    if (rc != PKV_OK)
+        return rc;
+    *n_items = need;
+    *n_units = units;
+    const int64_t pairs = (int64_t)shape->B * shape->H_kv;
+    if (capacity < need || (int64_t)indptr_capacity < pairs + 1 + units + 1 + need)
+        return PKV_ERR_CAPACITY;
+    if ((need > 0 && !items) || !indptr)
+        return PKV_ERR_INVALID;
+    const PrefixGroups g = prefix_groups(seq_lens_host, block_table_host, *shape);
+    const int64_t P = shape->page_size, span = (int64_t)chunk_pages * P, H_kv = shape->H_kv;
+    std::vector<int32_t> pos((size_t)shape->B, 0);  // a grouped row's place in its group
+    for (const std::vector<int32_t> &rows : g.rows)
+        for (size_t k = 0; k < rows.size(); ++k)
+            pos[(size_t)rows[k]] = (int32_t)k;
+    int32_t k = 0;
+    for (int32_t i = 0; i < shape->B; ++i) {
+        const int64_t n = seq_lens_host[i];
+        const int32_t gi = g.group_of[(size_t)i];
+        const int64_t L = gi >= 0 ? g.shared[(size_t)gi] : 0;
+        for (int32_t h = 0; h < shape->H_kv; ++h) {
+            indptr[(int64_t)i * H_kv + h] = k;
+            if (n == 0) {
+                items[k++] = {i, h, 0, 0};
+                continue;
+            }
+            for (int64_t b = 0; b < L * P; b += span)
+                items[k++] = {i, h, (int32_t)b, (int32_t)std::min<int64_t>(b + span, L * P)};
+            for (int64_t b = L * P; b < n; b += span)
+                items[k++] = {i, h, (int32_t)b, (int32_t)std::min<int64_t>(b + span, n)};
+        }
+    }
+    indptr[pairs] = k;
+    // units in the order of their first member: walking the items in order, a
+    // shared chunk opens its run's unit when its row starts a run of
+    // max_members rows of the group; other shared chunks ride in that unit
+    int32_t *unit_ptr = indptr + pairs + 1;
+    int32_t *unit_items = unit_ptr + units + 1;
+    int32_t u = 0, m = 0;
+    for (int32_t x = 0; x < k; ++x) {
+        const pkv_work_item &it = items[x];
+        const int32_t gi = g.group_of[(size_t)it.row];
+        const int64_t c = x - indptr[(int64_t)it.row * H_kv + it.kv_head];
+        const bool shared_chunk = gi >= 0 && it.tok_end > it.tok_begin && it.tok_begin < g.shared[(size_t)gi] * P;
+        if (!shared_chunk) {
+            unit_ptr[u++] = m;
+            unit_items[m++] = x;
+            continue;
+        }
+        const std::vector<int32_t> &rows = g.rows[(size_t)gi];
+        const int32_t p = pos[(size_t)it.row];
+        if (p % max_members != 0)
+            continue;  // rides in the unit its run's first row opened
+        unit_ptr[u++] = m;
+        for (int32_t q = p; q < (int32_t)rows.size() && q < p + max_members; ++q)
+            unit_items[m++] = indptr[(int64_t)rows[(size_t)q] * H_kv + it.kv_head] + (int32_t)c;
+    }
+    unit_ptr[u] = m;
     return PKV_OK;
 }
 

@@ -1,12 +1,14 @@
 """Device timing of decode steps (CUDA events on the launching stream).
 
-Two protocols:
+Three protocols:
   time_steady    K steps queued back to back between one pair of events,
                  consecutive steps reading different copies of the KV pool
                  (pool_copies) so that no step finds its pages in L2.  The K
                  steps are captured once in a CUDA graph and replayed, as a
                  serving loop replays its decode step, so that the host's
                  launch rate never paces the device;
+  time_interleaved  the same K steps, each after a kernel that streams
+                 through HBM (a projection's stand-in), minus that kernel alone;
   time_isolated  single cold steps, L2 flushed (Flush) before each, events
                  around the step alone.
 """
@@ -77,6 +79,62 @@ def time_steady(w, dp, K, W, torch, bd, copies, graph=True):
     if bd.workspace_status(dp) != 0:
         raise RuntimeError("device error during the timed steps")
     return a.elapsed_time(b)
+
+
+def time_interleaved(w, dp, K, W, torch, bd, copies, filler_bytes=64 << 20, lens_jitter=False):
+    """Device time (ms) of K decode steps that each follow another kernel, as
+    in a model where attention comes after a projection: every step is a
+    filler kernel streaming filler_bytes through HBM (a copy: that many bytes
+    read and as many written) then the decode step, all K captured in one CUDA
+    graph; the filler alone, captured and timed the same way, is subtracted.
+    With lens_jitter the filler also moves every row's length by one token
+    (+1, then -1 on the next step), as a serving loop's lengths change on the
+    device between steps.  Returns (decode ms for the K steps, filler ms)."""
+    lens = torch.tensor(w.seq_lens, dtype=torch.int32, device=w.q.device)
+    out = torch.empty_like(w.q)
+    src = torch.empty(filler_bytes // 2, dtype=torch.bfloat16, device=w.q.device).normal_()
+    dst = torch.empty_like(src)
+    up = torch.tensor([1 if n + 1 <= w.max_pages * w.P else 0 for n in w.seq_lens], dtype=torch.int32,
+                      device=w.q.device)
+
+    def filler(i):
+        dst.copy_(src)
+        if lens_jitter:
+            if i % 2 == 0:
+                lens.add_(up)
+            else:
+                lens.sub_(up)
+
+    def step(i):
+        k, v = copies[i % len(copies)]
+        filler(i)
+        bd.paged_decode(w.q, k, v, w.block_table, lens, w.P, w.scale, plan=dp, out=out)
+
+    def timed(body):
+        for i in range(W):
+            body(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(K):
+                body(W + i)
+        g.replay()
+        torch.cuda.synchronize()
+        st = torch.cuda.current_stream()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        g.replay()
+        b.record(st)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b)
+
+    both = timed(step)
+    alone = timed(filler)
+    if bd.workspace_status(dp) != 0:
+        raise RuntimeError("device error during the timed steps")
+    return both - alone, alone
 
 
 def time_isolated(w, dp, K, W, torch, bd, flush):

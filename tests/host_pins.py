@@ -15,6 +15,10 @@ real oracle and against copies with a planted mistake.
                       (tests/golden/launch_fanout_b8.txt)
   merge_state_closed  queue merge traffic = 2*G*(D+2)*4 * H_kv * (slots of
                       multi-chunk pairs); rectangular = the same over B*H_kv*S slots
+  prefix_queue        the queue that stages shared prefix pages once: items tile
+                      every row, units partition the items, a unit's members cover
+                      the same tokens on the same physical pages, the shared
+                      ranges are maximal, and without sharing it is the plain queue
   counters_recount    every counter of every mode, recounted from what the step
                       really moves: the bytes of the queue as built, the pages
                       the row's tokens touch (token by token), the blocks a
@@ -137,13 +141,18 @@ def policy_semantics(O):
     assert O.select_policy([1000, 5] * 2, P, rules) == (O.WORK_QUEUE, 3, 24, 1)
     # a balanced rule takes its block count as given
     assert O.select_policy([5000, 7], P, [R(0, 9, 0, O.INT32_MAX, 3, num_splits=296, flags=4)]) == (3, 296, 0, 4)
+    # a device-fill queue rule leaves the chunk to the device and carries its budget T
+    dev_fill = [R(0, 9, 0, O.INT32_MAX, O.WORK_QUEUE, num_splits=296, flags=O.FLAG_DEVICE_FILL | 4)]
+    assert O.select_policy([5000, 7], P, dev_fill) == (O.WORK_QUEUE, 296, 0, O.FLAG_DEVICE_FILL | 4)
     # no rule matches -> single kernel; empty batch and all-empty rows -> single kernel
     assert O.select_policy([10], P, rules[:1]) == (O.NO_SPLIT, 1, 0, 0)
     assert O.select_policy([], P, rules) == (O.NO_SPLIT, 1, 0, 0)
     assert O.select_policy([0, 0], P, rules) == (O.NO_SPLIT, 1, 0, 0)
     for bad in ([R(0, 9, 0, 9, 7)], [R(0, 9, 0, 9, O.SPLIT_S, num_splits=0)],
                 [R(0, 9, 0, 9, O.WORK_QUEUE, chunk_pages=-1)],
-                [R(0, 9, 0, 9, O.WORK_QUEUE, num_splits=0, chunk_pages=0)], [R(0, 9, 0, 9, 3, num_splits=0)]):
+                [R(0, 9, 0, 9, O.WORK_QUEUE, num_splits=0, chunk_pages=0)], [R(0, 9, 0, 9, 3, num_splits=0)],
+                [R(0, 9, 0, 9, O.WORK_QUEUE, num_splits=8, chunk_pages=3, flags=O.FLAG_DEVICE_FILL)],
+                [R(0, 9, 0, 9, O.SPLIT_S, num_splits=8, flags=O.FLAG_DEVICE_FILL)]):
         try:
             O.select_policy([5], P, bad)
         except ValueError:
@@ -356,6 +365,21 @@ def counters_recount(O):
             multi = sum(indptr[k + 1] - indptr[k] for k in range(B * H_kv) if indptr[k + 1] - indptr[k] > 1)
             assert c.merge_state_bytes == 2 * state * multi, what
             assert c.launches == 1 + (1 if flags & O.FLAG_SEPARATE_MERGE else 0), what
+    # A device-fill plan (2, T, 0, flags) does the work of the queue the fill rule
+    # picks on the host for the same budget, and sends no queue.
+    for lens, H_kv, P, C in itertools.chain(CASES, _random_cases(22, 20)):
+        for T in (1, 7, 37, 296):
+            host = O.select_policy(lens, P, [R(0, O.INT32_MAX, 0, O.INT32_MAX, O.WORK_QUEUE, num_splits=T)], H_kv)
+            dev = O.counters(lens, 8 * H_kv, H_kv, 64, P, (O.WORK_QUEUE, T, 0, O.FLAG_DEVICE_FILL))
+            what = ("counters_recount device fill", lens, H_kv, P, T)
+            if host[0] != O.WORK_QUEUE:  # no tokens at all: every pair has one empty item
+                assert dev.work_items == len(lens) * H_kv and dev.merge_state_bytes == 0, what
+                continue
+            ref = O.counters(lens, 8 * H_kv, H_kv, 64, P, host)
+            items, _ = O.build_work_queue(lens, H_kv, P, host[2])
+            assert dev.work_items == ref.work_items == len(items) and dev.queue_bytes == 0, what
+            assert (dev.merge_state_bytes, dev.empty_items) == (ref.merge_state_bytes, ref.empty_items), what
+            assert dev.work_items <= max(T, len(lens) * H_kv), what
     # Worked example, by hand: lens [40, 0], H_q = 4, H_kv = 2, D = 64, P = 16, T = 3.
     # Pages per pair: 3 and 0, so U = 6 and the shares are [0,2) [2,4) [4,6).
     # Pair (0,0) = pages 0..2 -> items (0,0,0,32) in block 0 and (0,0,32,40) in block 1;
@@ -378,9 +402,102 @@ def counters_recount(O):
         ("counters worked queue", c)
 
 
+def _prefix_cases(seed=31, n=40):
+    """(lens, block_table, H_kv, P, C, M): rows drawn into a few sharing groups
+    over a small pool, with shared runs of random length, short rows, empty
+    rows and rows whose last page is partial."""
+    rng = random.Random(seed)
+    fixed_bt = [[5, 6, 7, 8], [5, 6, 7, 9], [5, 6, 1, 2], [3, 4, 0, 0], [5, 6, 7, 8]]
+    yield [64, 60, 40, 20, 50], fixed_bt, 1, 16, 2, 2
+    yield [64, 64, 64], [[1, 2, 3, 4], [1, 2, 3, 4], [1, 2, 3, 4]], 2, 16, 1, 3
+    yield [15, 15, 33], [[1, 0, 0], [1, 0, 0], [1, 7, 2]], 1, 16, 1, 4
+    for _ in range(n):
+        B = rng.randint(1, 8)
+        P = rng.choice([8, 16])
+        maxp = rng.randint(1, 9)
+        prefixes = [[rng.randint(0, 40) for _ in range(maxp)] for _ in range(rng.randint(1, 3))]
+        lens, bt = [], []
+        for _ in range(B):
+            n = rng.choice([0, rng.randint(1, P * maxp), P * rng.randint(1, maxp)])
+            base = rng.choice(prefixes)
+            k = rng.randint(0, maxp)
+            row = base[:k] + [rng.randint(41, 80) for _ in range(maxp - k)]
+            lens.append(n)
+            bt.append(row)
+        yield lens, bt, rng.randint(1, 4), P, rng.randint(1, 4), rng.randint(1, 5)
+
+
+def prefix_queue(O):
+    for lens, bt, H_kv, P, C, M in _prefix_cases():
+        items, indptr, uptr, uitems = O.build_prefix_queue(lens, bt, H_kv, P, C, M)
+        what = ("prefix_queue", lens, bt, H_kv, P, C, M)
+        groups = O.shared_prefixes(lens, bt, P)
+        L_of = {r: L for rows, L in groups for r in rows}
+        # items tile every (row, head) in order, page aligned, and a shared row's
+        # chunks restart at its shared length
+        assert len(indptr) == len(lens) * H_kv + 1 and indptr[-1] == len(items), what
+        for i, n in enumerate(lens):
+            for h in range(H_kv):
+                pair = items[indptr[i * H_kv + h]:indptr[i * H_kv + h + 1]]
+                assert all(it[:2] == (i, h) for it in pair), what
+                if n == 0:
+                    assert pair == [(i, h, 0, 0)], what
+                    continue
+                pos, L = 0, L_of.get(i, 0)
+                for (_, _, b, e) in pair:
+                    assert b == pos and e > b and b % P == 0 and e - b <= C * P, what
+                    origin = 0 if b < L * P else L * P
+                    assert (b - origin) % (C * P) == 0 and (b >= L * P or e <= L * P), what
+                    pos = e
+                assert pos == n, what
+        # units partition the items; sizes; members share KV head, tokens and pages
+        assert uptr[0] == 0 and uptr[-1] == len(uitems) == len(items), what
+        assert sorted(uitems) == list(range(len(items))), what
+        firsts = [uitems[uptr[u]] for u in range(len(uptr) - 1)]
+        assert firsts == sorted(firsts), what
+        for u in range(len(uptr) - 1):
+            mem = [items[x] for x in uitems[uptr[u]:uptr[u + 1]]]
+            assert 1 <= len(mem) <= M, what
+            if len(mem) == 1:
+                continue
+            i0, h0, b0, e0 = mem[0]
+            assert [m[0] for m in mem] == sorted(m[0] for m in mem), what
+            for (i, h, b, e) in mem:
+                assert (h, b, e) == (h0, b0, e0) and e <= (lens[i] // P) * P, what
+                for pg in range(b // P, e // P):
+                    assert int(bt[i][pg]) == int(bt[i0][pg]), what
+        # groups: rows with a full page and a common first page; L maximal
+        for rows, L in groups:
+            assert len(rows) >= 2 and L >= 1, what
+            first = int(bt[rows[0]][0])
+            assert all(lens[r] >= P and int(bt[r][0]) == first for r in rows), what
+            assert all(int(bt[r][k]) == int(bt[rows[0]][k]) for r in rows for k in range(L)), what
+            assert any(lens[r] // P == L or (L < len(bt[r]) and int(bt[r][L]) != int(bt[rows[0]][L]))
+                       for r in rows), what
+        # completeness: two rows with a full page each and one first page share it
+        group_id = {r: g for g, (rows, _) in enumerate(groups) for r in rows}
+        for i in range(len(lens)):
+            for j in range(i + 1, len(lens)):
+                if lens[i] >= P and lens[j] >= P and int(bt[i][0]) == int(bt[j][0]):
+                    assert i in group_id and group_id.get(j) == group_id[i], what
+        # no sharing: the plain queue, one item per unit
+        distinct = [[100 + 10 * r + k for k in range(len(bt[r]))] for r in range(len(lens))]
+        items2, indptr2, uptr2, uitems2 = O.build_prefix_queue(lens, distinct, H_kv, P, C, M)
+        assert (items2, indptr2) == tuple(O.build_work_queue(lens, H_kv, P, C)), what
+        assert uitems2 == list(range(len(items2))) and uptr2 == list(range(len(items2) + 1)), what
+    # worked example: rows 0, 1, 2, 4 share first page 5; rows 2 and 4 hold 2 full
+    # pages in common with row 0, so L = 2 pages = 32 tokens
+    lens, bt = [64, 60, 40, 20, 50], [[5, 6, 7, 8], [5, 6, 7, 9], [5, 6, 1, 2], [3, 4, 0, 0], [5, 6, 7, 8]]
+    assert O.shared_prefixes(lens, bt, 16) == [([0, 1, 2, 4], 2)]
+    items, indptr, uptr, uitems = O.build_prefix_queue(lens, bt, 1, 16, 2, 2)
+    assert items == [(0, 0, 0, 32), (0, 0, 32, 64), (1, 0, 0, 32), (1, 0, 32, 60), (2, 0, 0, 32), (2, 0, 32, 40),
+                     (3, 0, 0, 20), (4, 0, 0, 32), (4, 0, 32, 50)]
+    assert uptr == [0, 2, 3, 4, 6, 7, 8, 9] and uitems == [0, 2, 1, 3, 4, 7, 5, 6, 8]
+
+
 HOST_PINS = (queue_closed_form, queue_cover, queue_bruteforce, policy_paper, policy_semantics, policy_fill,
              launch_fanout, merge_state_closed, counters_recount, balanced_shares, balanced_cover,
-             balanced_bruteforce)
+             balanced_bruteforce, prefix_queue)
 
 
 def run_all(O):

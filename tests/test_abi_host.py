@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from oracle import oracle as O
 from paged_kv_gqa_17_b200 import binding as bd
@@ -178,6 +179,7 @@ def test_host_pins_hold_for_the_c_planner(L):
 
     class Adapter:
         NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED, FLAG_SEPARATE_MERGE, INT32_MAX = 0, 1, 2, 3, 1, 2**31 - 1
+        FLAG_DEVICE_FILL = 32
         Rule = O.Rule
         load_rules = staticmethod(O.load_rules)
 
@@ -198,6 +200,21 @@ def test_host_pins_hold_for_the_c_planner(L):
             ptr = indptr.tolist()
             pairs = len(lens) * H_kv
             return [tuple(x) for x in items.tolist()], ptr[:pairs + 1], ptr[pairs + 1:]
+
+        shared_prefixes = staticmethod(O.shared_prefixes)
+
+        @staticmethod
+        def build_prefix_queue(lens, bt, H_kv, P, C, M):
+            if C < 1 or M < 1:
+                raise ValueError
+            width = max([len(r) for r in bt] + [1])
+            table = torch.tensor([list(r) + [0] * (width - len(r)) for r in bt] or [[0]], dtype=torch.int32)
+            shape = bd.make_shape(len(lens), H_kv, H_kv, 64, P, width, 1)
+            items, indptr, n_units = bd.build_prefix_queue(lens, table, shape, C, M)
+            pairs = len(lens) * H_kv
+            ptr = indptr.tolist()
+            return ([tuple(x) for x in items.tolist()], ptr[:pairs + 1], ptr[pairs + 1:pairs + 2 + n_units],
+                    ptr[pairs + 2 + n_units:])
 
         @staticmethod
         def select_policy(lens, P, rules, H_kv=1):
@@ -249,3 +266,17 @@ def test_device_queue_builder_host_checks(L):
     assert L.pkv_build_fill_queue_device(None, ctypes.byref(shape), 296, None, 296, None, None, None) == -1
     assert L.pkv_build_fill_queue_device(None, ctypes.byref(big), 296, None, 1 << 20, None, None, None) == -2
     assert L.pkv_build_fill_queue_device(None, ctypes.byref(empty), 296, None, 0, None, None, None) == 0
+
+
+def test_prefix_queue_matches_oracle_bit_for_bit(L):
+    """pkv_build_prefix_queue against the oracle's plain-Python builder on
+    the seeded sharing cases: items, pair offsets, unit offsets and members."""
+    for lens, bt, H_kv, P, C, M in host_pins._prefix_cases(seed=41, n=60):
+        width = max(len(r) for r in bt)
+        table = torch.tensor([list(r) for r in bt], dtype=torch.int32)
+        shape = bd.make_shape(len(lens), H_kv, H_kv, 64, P, width, 1)
+        items, indptr, n_units = bd.build_prefix_queue(lens, table, shape, C, M)
+        o_items, o_indptr, o_uptr, o_uitems = O.build_prefix_queue(lens, bt, H_kv, P, C, M)
+        assert [tuple(x) for x in items.tolist()] == o_items, (lens, bt, H_kv, P, C, M)
+        assert indptr.tolist() == o_indptr + o_uptr + o_uitems, (lens, bt, H_kv, P, C, M)
+        assert n_units == len(o_uptr) - 1

@@ -160,12 +160,17 @@ def test_fill_builder_matches_policy_and_host_queue_bit_exactly():
         assert int(ws[:4].view(torch.int32)[0]) == 0
 
 
-@pytest.mark.parametrize("T,flags", [(37, 0), (296, 4), (5, 1)])
-def test_decode_with_device_fill_queue_matches_oracle(T, flags):
+@pytest.mark.parametrize("T,flags,fused", [(37, 0, False), (296, 4, False), (5, 1, False), (37, 0, True),
+                                           (296, 4, True), (5, 0, True)])
+def test_decode_with_device_fill_queue_matches_oracle(T, flags, fused):
+    """The fill queue from the builder kernel, or derived by every decode
+    block itself (PKV_FLAG_DEVICE_FILL): the oracle's answer, and the same
+    bits as the host-built queue at the policy's chunk."""
     w = to_device(W.make_custom([3000, 77, 1999, 16, 0, 1], 32, 8, 128, seed=142, poison=True))
     shape = bd.shape_of(w.q, w.k_pool, w.block_table)
     plan = bd.select_policy(w.seq_lens, shape, [rule(2, T, 0, flags)])
-    dp = bd.plan_decode(w.seq_lens, shape, "cuda", plan=plan, device_queue=True, fill_blocks=T)
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", plan=plan, device_queue=True, fill_blocks=T, device_fill=fused)
+    assert bool(dp.plan.flags & bd.FLAG_DEVICE_FILL) == fused and (dp.items is None) == fused
     lens = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
     out = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp)
     torch.cuda.synchronize()
@@ -176,12 +181,13 @@ def test_decode_with_device_fill_queue_matches_oracle(T, flags):
     assert torch.equal(out, ref)  # same queue, same kernels: the same bits
 
 
-def test_graph_replay_of_the_fill_queue_follows_device_lengths():
+@pytest.mark.parametrize("fused", [False, True])
+def test_graph_replay_of_the_fill_queue_follows_device_lengths(fused):
     full = [2500, 900, 40, 1300]
     w = to_device(W.make_custom(full, 16, 4, 128, seed=143, poison=False))
     shape = bd.shape_of(w.q, w.k_pool, w.block_table)
     plan = bd.select_policy(full, shape, [rule(2, 148, 0, 4)])
-    dp = bd.plan_decode(full, shape, "cuda", plan=plan, device_queue=True, fill_blocks=148)
+    dp = bd.plan_decode(full, shape, "cuda", plan=plan, device_queue=True, fill_blocks=148, device_fill=fused)
     lens = torch.tensor(full, dtype=torch.int32, device="cuda")
     out = torch.empty_like(w.q)
     s = torch.cuda.Stream()
@@ -232,3 +238,49 @@ def test_device_queue_request_passes_queue_free_plans_through():
         w.seq_lens = list(step_lens)
         assert_close(out.float().cpu().double().numpy(), oracle_full(w), f"split-S replay {step_lens}")
     del g
+
+
+def test_device_fill_derives_the_host_queue_bit_for_bit():
+    """Random batches (B up to 70, all-empty rows, single-token rows, rows at
+    the table's capacity), H_kv 1..8, budgets from 1 to past the item count:
+    every block's self-derived item gives the same bits as the host-built
+    fill queue, and the error word stays clean."""
+    rng = np.random.default_rng(23)
+    cases = [([12129, 621, 1118, 1452, 2891, 1419, 518, 3174], 8, 296), ([32768], 8, 296), ([1], 1, 296),
+             ([0, 0, 5], 2, 7), ([16] * 5, 8, 7), ([40000] * 33, 2, 296), ([5000, 0, 1, 16, 17], 2, 1)]
+    for _ in range(14):
+        B = int(rng.integers(1, 71))
+        lens = [int(x) for x in rng.choice([0, 1, 15, 16, 17, 300, 5000, 20000], B)]
+        cases.append((lens, int(rng.choice([1, 2, 4, 8])), int(rng.choice([1, 3, 37, 148, 296, 444, 5000]))))
+    for lens, H_kv, T in cases:
+        w = to_device(W.make_custom(lens, 4 * H_kv, H_kv, 64, seed=145 + len(lens), poison=True))
+        shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+        lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        fused = bd.plan_decode(lens, shape, "cuda", plan=bd.Plan(2, T, 0, bd.FLAG_DEVICE_FILL))
+        host_plan = bd.select_policy(lens, shape, [rule(2, T, 0, 0)])
+        host = bd.plan_decode(lens, shape, "cuda", plan=host_plan)
+        a = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens_d, 16, w.scale, plan=fused)
+        b = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens_d, 16, w.scale, plan=host)
+        torch.cuda.synchronize()
+        assert bd.workspace_status(fused) == 0 and bd.workspace_status(host) == 0, (lens, H_kv, T)
+        assert torch.equal(a, b), (lens, H_kv, T, host_plan.tuple())
+        if host_plan.mode == bd.WORK_QUEUE:
+            assert fused.counters["work_items"] == host.counters["work_items"] and fused.counters["queue_bytes"] == 0
+
+
+def test_device_fill_flags_bad_lengths_and_clamps():
+    """A length past the table's capacity is clamped and reported, like the
+    other paths; the output equals the host queue's for the clamped lengths."""
+    w = to_device(W.make_custom([100, 64, 40], 8, 2, 64, seed=146))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    cap = shape.max_pages_per_seq * 16
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", plan=bd.Plan(2, 37, 0, bd.FLAG_DEVICE_FILL))
+    bad = torch.tensor([100, cap + 9, -4], dtype=torch.int32, device="cuda")
+    out = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, bad, 16, w.scale, plan=dp)
+    assert bd.workspace_status(dp) & 2
+    clamped = [100, cap, 0]
+    host = bd.plan_decode(clamped, shape, "cuda", plan=bd.select_policy(clamped, shape, [rule(2, 37, 0, 0)]))
+    ref = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table,
+                          torch.tensor(clamped, dtype=torch.int32, device="cuda"), 16, w.scale, plan=host)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)

@@ -50,8 +50,8 @@ PY_MUTANTS = {
     "balanced item not clipped to row": ("min((y - u) * P, n)", "(y - u) * P"),
     "fill rule allows one item too many": ("if fill_items(lens, H_kv, P, c) <= chosen.num_splits:",
                                            "if fill_items(lens, H_kv, P, c) <= chosen.num_splits + 1:"),
-    "queue bytes miss the last pair offset": ("qbytes = 16 * work + 4 * (B * H_kv + 1)\n",
-                                              "qbytes = 16 * work + 4 * B * H_kv\n"),
+    "queue bytes miss the last pair offset": ("else 16 * work + 4 * (B * H_kv + 1)\n",
+                                              "else 16 * work + 4 * B * H_kv\n"),
     "balanced queue bytes miss the block offsets": (" + 4 * (B * H_kv + 1) + 4 * (S + 1)", " + 4 * (B * H_kv + 1)"),
     "streamed bytes count valid tokens only": ("kv_streamed = sum(pages) * P * H_kv", "kv_streamed = sum(lens) * H_kv"),
     "balanced merge counts single-slot pairs": ("        merge = 2 * sum(k for k in per_pair if k > 1) * state",
@@ -60,6 +60,18 @@ PY_MUTANTS = {
     "no-split empty rows not per head": ("work = B * H_kv\n        empty = H_kv * sum(",
                                          "work = B * H_kv\n        empty = sum("),
     "no-split work counts rows": ("        work = B * H_kv\n", "        work = B\n"),
+    "device-fill counters count the queue bytes": ("qbytes = 0 if device_fill else 16 * work",
+                                                   "qbytes = 16 * work"),
+    "device-fill plan carries a chunk": ("        return (WORK_QUEUE, chosen.num_splits, 0, chosen.flags)\n",
+                                         "        return (WORK_QUEUE, chosen.num_splits, 1, chosen.flags)\n"),
+    "prefix shares the leader's partial last page": ("        L = lens[lead] // P\n",
+                                                     "        L = -(-lens[lead] // P)\n"),
+    "prefix counts a member's partial page": ("            while k < min(full, L) and", "            while k < L and"),
+    "prefix groups rows without a full page": ("        if n >= P:\n            by_first", "        if n >= 1:\n            by_first"),
+    "prefix tail chunks restart at zero": ("                t = L * P\n                while t < n:",
+                                           "                t = 0\n                while t < n:"),
+    "prefix units exceed the member cap": ("for k in range(0, len(members), max_members):\n            units.append(members[k:k + max_members])",
+                                           "for k in range(0, len(members), max_members + 1):\n            units.append(members[k:k + max_members + 1])"),
     "fill rule ignores heads": ("    return H_kv * sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)",
                                 "    return sum(max(1, _ceil_div(_ceil_div(int(n), P), C)) for n in seq_lens)"),
 }
