@@ -88,6 +88,11 @@ typedef enum {
                                      run as one thread-block cluster and merge their states through
                                      distributed shared memory (no partial states in the workspace,
                                      no merge launch); other modes return PKV_ERR_UNSUPPORTED */
+#define PKV_FLAG_SHARED_PREFIX 64 /* WORK_QUEUE only, plan {2, U, C, flags}: items / indptr hold the
+                                     prefix-sharing queue of pkv_build_prefix_queue at chunk C and U is its
+                                     unit count: one block per unit stages the unit's shared pages once
+                                     for all its members.  n_items = the item count.  Not with
+                                     PKV_FLAG_DEVICE_FILL or PKV_FLAG_PDL_EARLY (PKV_ERR_UNSUPPORTED) */
 #define PKV_FLAG_DEVICE_FILL 32   /* WORK_QUEUE only, plan {2, T, 0, flags}: no queue is passed; every
                                      block derives its own item of the compact queue whose chunk fills
                                      one wave of T blocks (the fill rule of pkv_select_policy) from the
@@ -124,6 +129,7 @@ typedef struct {
  *   SPLIT_S:     {1, S', C, flags}  C = ceil(pages_max / S), S' = ceil(pages_max / C)
  *   WORK_QUEUE:  {2, S', C, flags}  C from the rule,        S' = ceil(pages_max / C)
  *                {2, T, 0, flags}   with PKV_FLAG_DEVICE_FILL: the fill budget T, C found on the device
+ *                {2, U, C, flags}   with PKV_FLAG_SHARED_PREFIX: U units of the prefix-sharing queue
  *   BALANCED:    {3, T, 0, flags}   T blocks from the rule's num_splits
  * where pages_max = ceil(N_max / P).  S' is the most chunks any row needs. */
 typedef struct {
@@ -440,7 +446,12 @@ PKV_API int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape 
  * counters and error word host->device in ONE copy, run pkv_paged_decode,
  * move the error word and out device->host in ONE copy and synchronize
  * `stream`.  q, block_table and out larger than 64 KiB each get a copy of
- * their own instead of travelling through the staging buffer.  q_host,
+ * their own instead of travelling through the staging buffer.  When out_host
+ * and host_staging are page-locked (mapped into the device's address space,
+ * as all page-locked memory is under unified addressing) the kernels write
+ * out straight into out_host and report device errors as flag words in
+ * host_staging, so the step moves its result without a device->host copy;
+ * pageable buffers take the packed device->host copy.  q_host,
  * block_table_host, seq_lens_host, out_host are host pointers with the
  * layouts of pkv_paged_decode; k_pool / v_pool are device pools (the cache
  * stays resident on the device).  device_buffer must be 256-byte aligned

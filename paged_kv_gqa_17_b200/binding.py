@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(HERE, "libpkv.so")
 NO_SPLIT, SPLIT_S, WORK_QUEUE, BALANCED = 0, 1, 2, 3
 FLAG_SEPARATE_MERGE, FLAG_NO_PDL, FLAG_DEEP_RING, FLAG_CLUSTER_MERGE, FLAG_PDL_EARLY = 1, 2, 4, 8, 16
 FLAG_DEVICE_FILL = 32
+FLAG_SHARED_PREFIX = 64
 FILL_MAX_ROWS = 1024  # rows a device-fill plan can plan for on the device
 INT32_MAX = 2**31 - 1
 _MODE_NAMES = {"NO_SPLIT": NO_SPLIT, "SPLIT_S": SPLIT_S, "WORK_QUEUE": WORK_QUEUE, "BALANCED": BALANCED}
@@ -452,10 +453,39 @@ class DecodePlan:
     fill_blocks: int = 0  # device queue of a WORK_QUEUE plan: the wave it fills
 
 
+def prefix_counters(seq_lens_host, shape: Shape, items: torch.Tensor, indptr: torch.Tensor, n_units: int,
+                    flags: int = 0) -> dict:
+    """Workload counters of a prefix-sharing plan, counted from its queue: one
+    block per unit, a unit's pages streamed once for all its members."""
+    lens = [int(n) for n in (seq_lens_host.tolist() if isinstance(seq_lens_host, torch.Tensor) else seq_lens_host)]
+    B, H_kv, D, P = shape.B, shape.H_kv, shape.head_dim, shape.page_size
+    G = shape.H_q // H_kv
+    pairs = B * H_kv
+    ptr = indptr.tolist()
+    it = items.tolist()
+    uptr = ptr[pairs + 1:pairs + 2 + n_units]
+    uitems = ptr[pairs + 2 + n_units:]
+    per_pair = [ptr[k + 1] - ptr[k] for k in range(pairs)]
+    streamed = 0
+    for u in range(n_units):
+        _, _, tb, te = it[uitems[uptr[u]]]
+        streamed += (-(-te // P) - tb // P) if te > tb else 0
+    return {"launches": 1 + (1 if flags & FLAG_SEPARATE_MERGE else 0), "work_items": n_units,
+            "empty_items": H_kv * sum(1 for n in lens if n == 0),
+            "merge_state_bytes": 2 * sum(k for k in per_pair if k > 1) * G * (D + 2) * 4,
+            "kv_bytes": sum(lens) * H_kv * 2 * D * 2, "kv_bytes_streamed": streamed * P * 2 * D * 2,
+            "q_bytes": B * shape.H_q * D * 2, "out_bytes": B * shape.H_q * D * 2,
+            "queue_bytes": 16 * len(it) + 4 * len(ptr), "bucket_launches": 2 * len({n for n in lens if n > 0})}
+
+
 def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[Plan] = None,
                 device_queue: bool = False, fill_blocks: int = 296,
-                device_fill: Optional[bool] = None) -> DecodePlan:
+                device_fill: Optional[bool] = None, shared_prefix_table=None) -> DecodePlan:
     """Host planning for one batch: policy (unless `plan` is given), queue, workspace.
+
+    shared_prefix_table (the host block table) asks for the queue that stages
+    the prefix pages rows share once for several rows (pkv_build_prefix_queue
+    at the plan's chunk; PKV_FLAG_SHARED_PREFIX); a NO_SPLIT plan stays as is.
 
     device_queue=True leaves the queue to the GPU, rebuilt from the device
     lengths by every paged_decode call (so one plan, or one captured CUDA
@@ -469,6 +499,22 @@ def plan_decode(seq_lens_host, shape: Shape, device, rules=None, plan: Optional[
     to those they were planned for (SPLIT_S: S' chunks of C pages)."""
     if plan is None:
         plan = select_policy(seq_lens_host, shape, rules)
+    if shared_prefix_table is not None and plan.mode != NO_SPLIT or (plan.flags & FLAG_SHARED_PREFIX):
+        # the prefix-sharing queue at the plan's chunk (a queue-free plan's whole rows otherwise)
+        if shared_prefix_table is None:
+            raise ValueError("a shared-prefix plan needs the host block table (shared_prefix_table)")
+        lens = [int(n) for n in (seq_lens_host.tolist() if isinstance(seq_lens_host, torch.Tensor)
+                                 else seq_lens_host)]
+        pages_max = max([-(-n // shape.page_size) for n in lens] + [1])
+        C = plan.chunk_pages if plan.mode in (SPLIT_S, WORK_QUEUE) and plan.chunk_pages > 0 else pages_max
+        members = max(1, 16 // (shape.H_q // shape.H_kv))
+        items_h, indptr_h, n_units = build_prefix_queue(lens, shared_prefix_table, shape, C, members)
+        flags = (plan.flags | FLAG_SHARED_PREFIX) & ~(FLAG_DEVICE_FILL | FLAG_PDL_EARLY | FLAG_CLUSTER_MERGE)
+        pplan = Plan(WORK_QUEUE, n_units, C, flags)
+        n_items = int(items_h.shape[0])
+        ws = torch.zeros(workspace_bytes(shape, pplan, n_items), dtype=torch.uint8, device=device)
+        return DecodePlan(shape, pplan, items_h.to(device), indptr_h.to(device), n_items, ws,
+                          prefix_counters(lens, shape, items_h, indptr_h, n_units, flags))
     if plan.mode == WORK_QUEUE and plan.flags & FLAG_DEVICE_FILL:
         device_queue, device_fill, fill_blocks = True, True, plan.num_splits
     if device_queue and plan.mode == WORK_QUEUE:
@@ -607,6 +653,7 @@ class HostDecoder:
         self._plan_ref = ctypes.byref(self._plan)
         self._bufs = (0, 0, 0, 0)
         self._checked = ()  # weak references to the tensors (and the shape) of the last checked call
+        self._args = None   # the argument tuple of the last call with the checked tensors, its scale, no rules
 
     def ensure(self, seq_lens_host, shape: Shape, rules=None):
         L = lib()
@@ -620,6 +667,7 @@ class HostDecoder:
         if self.host.numel() < hb.value:
             self.host = torch.zeros(hb.value, dtype=torch.uint8).pin_memory()
         self._bufs = (self.dev.data_ptr(), self.dev.numel(), self.host.data_ptr(), self.host.numel())
+        self._args = None
 
     def __call__(self, q_host: torch.Tensor, block_table_host: torch.Tensor, seq_lens_host: torch.Tensor,
                  out_host: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, scale: float, shape: Shape,
@@ -634,11 +682,21 @@ class HostDecoder:
                              self.dev.get_device())
             self._checked = tuple(weakref.ref(t) for t in (q_host, block_table_host, seq_lens_host, out_host,
                                                             k_pool, v_pool)) + (shape,)
+            self._args = None
+        elif rules is None and stream is None and timing is None and self._args is not None and \
+                self._args[6] == scale:
+            # the same checked tensors as the last call: its argument tuple holds
+            rc = self._fn(*self._args)
+            if rc != 0:
+                raise PkvError(rc, "pkv_decode_host")
+            return Plan.from_buffer_copy(self._plan)
         arr, n = rules_array(rules) if rules is not None else (None, 0)
         dev, dev_n, host, host_n = self._bufs
         args = (q_host.data_ptr(), block_table_host.data_ptr(), seq_lens_host.data_ptr(), out_host.data_ptr(),
                 k_pool.data_ptr(), v_pool.data_ptr(), float(scale), ctypes.byref(shape), arr, n, dev, dev_n,
                 host, host_n, self._stream if stream is None else _stream_ptr(stream), self._plan_ref)
+        if rules is None and stream is None:
+            self._args = args
         rc = self._fn(*args) if timing is None else self._fn_timed(*args, ctypes.byref(timing))
         if rc != 0:
             raise PkvError(rc, "pkv_decode_host")

@@ -85,6 +85,7 @@ struct __align__(64) Params {
     float *ws_l;
     float *ws_acc;
     uint32_t *ws_counters;
+    uint32_t *ws_flags;  // per slot: its partial state is written (set by its block, cleared by the merger)
     uint32_t *ws_error;
     float scale_log2;  // scale * log2(e): logits are kept in the log2 domain
     int32_t B, H_q, H_kv, G, max_pages, num_pool_pages;
@@ -92,12 +93,25 @@ struct __align__(64) Params {
     int32_t pdl_early;  // may read lengths, table and KV pages (but a row's last) before the dependency wait
     int32_t n_items;
     int32_t prefetch_blocks;  // blocks below this index warm L2 before the wait (the grid's first wave)
+    uint32_t *host_err;       // or NULL: per error bit k, a flag word host_err[k] in mapped host memory
+    int32_t n_units;          // prefix-sharing queue: units (the grid); their offsets follow the pair offsets
     int32_t device_fill;      // WORK_QUEUE: every block derives its own item from the device lengths
     int32_t fill_blocks;      // ... of the queue whose chunk fills one wave of this many blocks
 #ifdef PKV_TRACE
     int32_t trace_epoch;
 #endif
 };
+
+// Record an error bit the kernel met on device data: in the workspace's error
+// word and, for a call whose caller reads the result straight from host
+// memory, as a plain store of 1 into that bit's own flag word there (one word
+// per bit, so no read-modify-write crosses the bus).
+__device__ __forceinline__ void raise_error(const Params &p, uint32_t bit)
+{
+    atomicOr(p.ws_error, bit);
+    if (p.host_err)
+        *reinterpret_cast<volatile uint32_t *>(p.host_err + (__ffs(bit) - 1)) = 1u;
+}
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -163,8 +177,10 @@ __device__ unsigned long long g_pkv_trace_buf[2][kTraceBlocks][16];
 #endif
 
 // Wait for phase `parity` of an mbarrier, giving up after kWaitLimitNs (or
-// kWaitLimitIters polls) with the timeout bit set in the error word.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err, uint64_t limit_ns = kWaitLimitNs)
+// kWaitLimitIters polls) with the timeout bit set in the error word (and,
+// when host_flags is not NULL, the timeout's flag word set in host memory).
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err, uint64_t limit_ns = kWaitLimitNs,
+                                       uint32_t *host_flags = nullptr)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -176,6 +192,8 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *
             break;
     }
     atomicOr(err, kErrTimeout);
+    if (host_flags)
+        *reinterpret_cast<volatile uint32_t *>(host_flags) = 1u;  // bit 0: timeout
     return false;
 }
 
@@ -233,6 +251,50 @@ __device__ __forceinline__ uint32_t ticket_acq_rel(uint32_t *ctr)
     uint32_t prev;
     asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr) : "memory");
     return prev;
+}
+
+// The split kernel's ticket, taken as soon as a block's pages are done: a
+// relaxed increment, since the states travel under their own flags.
+__device__ __forceinline__ uint32_t ticket_relaxed(uint32_t *ctr)
+{
+    uint32_t prev;
+    asm volatile("atom.add.relaxed.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr) : "memory");
+    return prev;
+}
+
+// A slot's "state written" flag: set with release (after the block's state
+// stores, made visible to the setting thread by a barrier), read with acquire.
+__device__ __forceinline__ void flag_release(uint32_t *f)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(1u) : "memory");
+}
+
+__device__ __forceinline__ uint32_t flag_acquire(const uint32_t *f)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+// Wait until a slot's flag is set, then clear it for the next call.  The
+// block that sets it has already taken its ticket, so it is running and
+// sets the flag within a few microseconds; the wait still gives up after
+// kWaitLimitNs with the timeout bit set.
+__device__ __noinline__ bool wait_flag(uint32_t *f, uint32_t *err, uint32_t *host_flags)
+{
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 0; i < kWaitLimitIters; ++i) {
+        if (flag_acquire(f)) {
+            *f = 0u;
+            return true;
+        }
+        if ((i & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs)
+            break;
+    }
+    atomicOr(err, kErrTimeout);
+    if (host_flags)
+        *reinterpret_cast<volatile uint32_t *>(host_flags) = 1u;
+    return false;
 }
 
 __device__ __forceinline__ void fence_proxy_async_global()
@@ -443,7 +505,8 @@ struct Cfg {
     static constexpr int kRingBytes = 2 * NST * kStageBytes;
     static constexpr int kBarOff = ((kRingBytes > kCombineBytes ? kRingBytes : kCombineBytes) + 63) / 64 * 64;
     static constexpr int kMiscOff = kBarOff + 2 * NST * 8;  // int flag, merge mbarriers at +8, +16, a guessed item at +32
-    static constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + slack to align the base to 1024
+    static constexpr int kFillResOff = kMiscOff + 64;       // a block's self-derived work item (8 int32)
+    static constexpr int kSmemBytes = kMiscOff + 96 + 1024;  // + slack to align the base to 1024
     static constexpr int kMaxMergeTasks = (kGP * (D / 4) + kThreads - 1) / kThreads;
     // cluster merge: this block's final state [m: 16][l: 16][acc: kGP][D] in the idle ring
     static constexpr int kClusterOff = (kCombineBytes + 127) / 128 * 128;
@@ -457,6 +520,7 @@ struct Cfg {
 #ifndef PKV_ISSUE_LANES
 #define PKV_ISSUE_LANES 4
 #endif
+
 
 // Producer: copy the K and V blocks of cnt consecutive pages of one KV head
 // into the ring, page j's physical id held by lane j of `e`; pages get ring
@@ -482,7 +546,7 @@ __device__ __forceinline__ bool issue_pages(const Params &p, int lane, int e, in
             const int g = gp + j;
             const int st = g % NST;
             const int k = g / NST;
-            if (k > 0 && !mbar_wait(bar_empty + 8 * st, (k - 1) & 1, p.ws_error))
+            if (k > 0 && !mbar_wait(bar_empty + 8 * st, (k - 1) & 1, p.ws_error, kWaitLimitNs, p.host_err))
                 my_ok = false;
             if (my_ok) {
                 const uint32_t fb = bar_full + 8 * st;
@@ -756,7 +820,7 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
     for (int k = 0; k < C::kMaxMergeTasks; ++k)
         O[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int ch = 0; ch < nch; ++ch) {
-        mbar_wait(mbar0 + 8 * (ch & 1), (uses[ch & 1] + (ch >> 1)) & 1, p.ws_error);
+        mbar_wait(mbar0 + 8 * (ch & 1), (uses[ch & 1] + (ch >> 1)) & 1, p.ws_error, kWaitLimitNs, p.host_err);
         const float *st = reinterpret_cast<const float *>(smem + wbytes + (ch & 1) * half);
         const int first = ch * hs;
         const int cnt = min(hs, n - first);
@@ -1000,149 +1064,192 @@ __device__ __forceinline__ int warp_max_i32(int v)
 //   count(C) = H_kv * sum_i max(1, ceil(pages_i / C)) <= T,
 // or pages_max when one item per (row, KV head) already exceeds T.  Since
 // ceil(x) lies in [x, x + 1), C lies in [ceil(H_kv * U / T),
-// ceil(H_kv * U / (T - H_kv * B))] (U = sum_i pages_i); every thread tests
-// one candidate of that range at a time, so the search takes one round
-// whenever the range holds no more candidates than the block has threads.
-// Then a prefix sum over the rows' chunk counts places block b's item.
-// Called by every thread of the block (it has block-wide barriers); `sm`
-// holds 3 * B + 5 int32 of shared memory that nothing else uses meanwhile.
+// ceil(H_kv * U / (T - H_kv * B))] (U = sum_i pages_i): the 32 lanes of
+// warp 0 test 32 candidates of that range at a time, so the search takes one
+// round whenever the range holds at most 32 chunk sizes (it does when the
+// wave is large against B * H_kv).  Then a prefix sum over the rows' chunk
+// counts places block b's item.  Warp 0 does the work in 32-bit arithmetic
+// (the host checks H_kv * B * max_pages < 2^31): up to 32 rows in registers
+// (lane i holds row i, shuffles carry the rest), more through `sm`, 3 * B + 1
+// int32 of the idle ring.  The item reaches the block through `res` (8
+// int32 outside the ring): called by every thread (one block barrier).
 // speculative: lengths read through L2 before the dependency wait, for the
 // L2 prefetch only; no error is recorded.
+__device__ __forceinline__ uint32_t fill_row_len(const Params &p, int i, bool speculative)
+{
+    const uint32_t cap = (uint32_t)p.max_pages * kPage;
+    const int n = speculative ? ld_l2_only(p.seq_lens + i) : __ldg(p.seq_lens + i);
+    if (n >= 0 && (uint32_t)n <= cap)
+        return (uint32_t)n;
+    if (!speculative)
+        raise_error(p, kErrSeqLen);
+    return n < 0 ? 0u : cap;
+}
+
+// The smallest chunk in [lo, hi] that satisfies the fill rule (hi does),
+// given count(c) (items of one KV head at chunk c) for the lane's candidate;
+// called by a whole warp, every lane calling count() in step.
+template <typename Count>
+__device__ __forceinline__ uint32_t fill_search(uint32_t lo, uint32_t hi, uint32_t limit, int lane, Count count)
+{
+    while (lo < hi) {
+        const uint32_t step = (hi - lo + 32) / 32;
+        const uint32_t c = lo + (uint32_t)lane * step;
+        const uint32_t n = count(c < hi ? c : hi);  // every lane counts: count() may shuffle
+        const bool ok = c < hi && n <= limit;
+        const uint32_t hits = __ballot_sync(0xffffffffu, ok);
+        const uint32_t b = hits ? lo + (uint32_t)(__ffs(hits) - 1) * step : hi;
+        lo = b + 1 > lo + step ? b + 1 - step : lo;
+        hi = b;
+    }
+    return lo;
+}
+
 template <int NTHREADS>
-__device__ FillItem fill_queue_item(const Params &p, int32_t *sm, bool speculative)
+__device__ __noinline__ FillItem fill_queue_item(const Params &p, int32_t *sm, int32_t *res, bool speculative)
 {
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int B = p.B;
-    int32_t *pages = sm;            // [B]
-    int32_t *lens = sm + B;         // [B] (clamped)
-    int32_t *rs = sm + 2 * B;       // [B + 1]: items of one KV head before row i
-    int32_t *red = sm + 3 * B + 1;  // [4]: pages_max, sum of pages, best candidate (two rounds' slots)
-    const int64_t cap = (int64_t)p.max_pages * kPage;
-    __syncthreads();  // every thread is done with sm
-    if (tid == 0) {
-        red[0] = 0;
-        red[1] = 0;
-        red[2] = INT_MAX;
-        red[3] = INT_MAX;
-    }
-    __syncthreads();
-    int lmax = 0, lsum = 0;
-    for (int i = tid; i < B; i += NTHREADS) {
-        int N = speculative ? ld_l2_only(p.seq_lens + i) : __ldg(p.seq_lens + i);
-        if (N < 0 || N > cap) {
-            if (!speculative)
-                atomicOr(p.ws_error, kErrSeqLen);
-            N = N < 0 ? 0 : (int)cap;
-        }
-        const int pg = (N + kPage - 1) / kPage;
-        lens[i] = N;
-        pages[i] = pg;
-        lmax = max(lmax, pg);
-        lsum += pg;
-    }
-    lmax = warp_max_i32(lmax);
-    lsum = warp_sum_i32(lsum);
-    if (lane == 0 && (lmax > 0 || lsum > 0)) {
-        atomicMax(&red[0], lmax);
-        atomicAdd(&red[1], lsum);
-    }
-    __syncthreads();
-    const int pmax = red[0];
-    const int64_t U = red[1];
-    const int64_t T = p.fill_blocks;
-    const int64_t HB = (int64_t)p.H_kv * B;
-    int64_t C;
-    if (pmax == 0) {
-        C = 1;  // every row is empty: one empty item per (row, KV head)
-    } else if (HB > T) {
-        C = pmax;
-    } else {
-        int64_t lo = (p.H_kv * U + T - 1) / T;
-        int64_t hi = HB < T ? (p.H_kv * U + (T - HB) - 1) / (T - HB) : pmax;
-        lo = lo < 1 ? 1 : (lo > pmax ? pmax : lo);
-        hi = hi > pmax ? pmax : (hi < lo ? lo : hi);
-        // hi satisfies the rule (count(hi) <= T); find the smallest that does
-        for (int round = 0; lo < hi; ++round) {
-            const int64_t step = (hi - lo + NTHREADS) / NTHREADS;
-            const int64_t c = lo + (int64_t)tid * step;
-            int32_t *best = red + 2 + (round & 1);
-            if (c < hi) {
-                const uint32_t cu = (uint32_t)c;
-                int64_t n = 0;
-                for (int i = 0; i < B && n * p.H_kv <= T; ++i) {
-                    const uint32_t k = ((uint32_t)pages[i] + cu - 1) / cu;
-                    n += k > 1 ? k : 1;
-                }
-                if (n * p.H_kv <= T)
-                    atomicMin(best, (int)c);
-            }
-            if (tid == 0)
-                red[2 + ((round + 1) & 1)] = INT_MAX;  // the next round's slot
-            __syncthreads();
-            const int64_t b = *best < hi ? *best : hi;
-            lo = b - step + 1 > lo ? b - step + 1 : lo;
-            hi = b;
-            __syncthreads();  // every thread has read this round's slot
-        }
-        C = lo;
-    }
-    // one KV head's item offsets per row (one warp scans the rows)
     if (tid < 32) {
-        int carry = 0;
-        for (int base = 0; base < B; base += 32) {
-            const int i = base + lane;
-            int cnt = 0;
-            if (i < B) {
-                const int k = (int)(((int64_t)pages[i] + C - 1) / C);
+        const uint32_t T = (uint32_t)p.fill_blocks;
+        const uint32_t H = (uint32_t)p.H_kv;
+        const uint32_t HB = H * (uint32_t)B;
+        const uint32_t b = blockIdx.x;
+        uint32_t pmax = 0, U = 0;
+        uint32_t my_len = 0, my_pg = 0;  // row `lane` (B <= 32)
+        if (B <= 32) {
+            if (lane < B) {
+                my_len = fill_row_len(p, lane, speculative);
+                my_pg = (my_len + kPage - 1) / kPage;
+            }
+            pmax = my_pg;
+            U = my_pg;
+        } else {
+            for (int i = lane; i < B; i += 32) {
+                const uint32_t N = fill_row_len(p, i, speculative);
+                const uint32_t pg = (N + kPage - 1) / kPage;
+                sm[B + i] = (int32_t)N;
+                sm[i] = (int32_t)pg;
+                pmax = max(pmax, pg);
+                U += pg;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            pmax = max(pmax, __shfl_xor_sync(0xffffffffu, pmax, off));
+            U += __shfl_xor_sync(0xffffffffu, U, off);
+        }
+        __syncwarp();
+        // items of one head at chunk c
+        auto count = [&](uint32_t c) {
+            uint32_t n = 0;
+            for (int i = 0; i < B; ++i) {
+                const uint32_t pg = B <= 32 ? __shfl_sync(0xffffffffu, my_pg, i) : (uint32_t)sm[i];
+                const uint32_t k = (pg + c - 1) / c;
+                n += k > 1 ? k : 1;
+            }
+            return n;
+        };
+        uint32_t C;
+        if (pmax == 0) {
+            C = 1;  // every row is empty: one empty item per (row, KV head)
+        } else if (HB > T) {
+            C = pmax;
+        } else {
+            uint32_t lo = (H * U + T - 1) / T;
+            uint32_t hi = HB < T ? (H * U + (T - HB) - 1) / (T - HB) : pmax;
+            lo = lo < 1 ? 1 : (lo > pmax ? pmax : lo);
+            hi = hi > pmax ? pmax : (hi < lo ? lo : hi);
+            C = fill_search(lo, hi, T / H, lane, count);  // count(c) * H <= T  <=>  count(c) <= T / H
+        }
+        int row = -1;
+        uint32_t row_start = 0, row_cnt = 1, row_len = 0;
+        if (B <= 32) {
+            // one KV head's item offset of row `lane`, then the row whose items hold b
+            uint32_t cnt = 0;
+            if (lane < B) {
+                const uint32_t k = (my_pg + C - 1) / C;
                 cnt = k > 1 ? k : 1;
             }
-            int incl = cnt;
+            uint32_t incl = cnt;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                const int add = __shfl_up_sync(0xffffffffu, incl, off);
+                const uint32_t add = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off)
                     incl += add;
             }
-            if (i < B)
-                rs[i] = carry + incl - cnt;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
+            const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+            const uint32_t start = incl - cnt;
+            if (b < total * H) {
+                row = __popc(__ballot_sync(0xffffffffu, lane < B && start * H <= b)) - 1;
+                row_start = __shfl_sync(0xffffffffu, start, row);
+                row_cnt = __shfl_sync(0xffffffffu, cnt, row);
+                row_len = __shfl_sync(0xffffffffu, my_len, row);
+            }
+        } else {
+            int32_t *rs = sm + 2 * B;  // [B + 1]: items of one KV head before row i
+            uint32_t carry = 0;
+            for (int base = 0; base < B; base += 32) {
+                const int i = base + lane;
+                uint32_t cnt = 0;
+                if (i < B) {
+                    const uint32_t k = ((uint32_t)sm[i] + C - 1) / C;
+                    cnt = k > 1 ? k : 1;
+                }
+                uint32_t incl = cnt;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t add = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off)
+                        incl += add;
+                }
+                if (i < B)
+                    rs[i] = (int32_t)(carry + incl - cnt);
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0)
+                rs[B] = (int32_t)carry;
+            __syncwarp();
+            if (b < carry * H) {
+                int below = 0;
+                for (int base = 0; base < B; base += 32) {
+                    const int i = base + lane;
+                    below += __popc(__ballot_sync(0xffffffffu, i < B && (uint32_t)rs[i] * H <= b));
+                }
+                row = below - 1;
+                row_start = (uint32_t)rs[row];
+                row_cnt = (uint32_t)(rs[row + 1] - rs[row]);
+                row_len = (uint32_t)sm[B + row];
+            }
+            fence_proxy_async_smem();  // these generic writes precede later TMA writes into the ring
         }
-        if (lane == 0)
-            rs[B] = carry;
+        if (lane == 0) {
+            res[0] = row;
+            if (row >= 0) {
+                const uint32_t j = b - row_start * H;
+                const uint32_t h = j / row_cnt, c = j - h * row_cnt;
+                const uint32_t span = C * kPage;
+                res[1] = (int32_t)h;
+                res[2] = row_len > 0 ? (int32_t)(c * span) : 0;
+                res[3] = row_len > 0 ? (int32_t)((c + 1) * span < row_len ? (c + 1) * span : row_len) : 0;
+                res[4] = (int32_t)(row_start * H + h * row_cnt);
+                res[5] = (int32_t)row_cnt;
+                res[6] = (int32_t)row_len;
+            }
+        }
     }
-    fence_proxy_async_smem();  // these generic writes precede later TMA writes into the ring
     __syncthreads();
     FillItem f;
-    f.valid = false;
-    f.row = f.h = f.tb = f.te = f.slot0 = f.len = 0;
-    f.nslots = 1;
-    const int64_t b = blockIdx.x;
-    if (b >= (int64_t)rs[B] * p.H_kv)
-        return f;  // past the queue: nothing to do for this block
-    int lo = 0, hi = B - 1;  // the last row whose items start at or before b
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((int64_t)rs[mid] * p.H_kv <= b)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    const int i = lo;
-    const int cnt = rs[i + 1] - rs[i];
-    const int64_t j = b - (int64_t)rs[i] * p.H_kv;
-    const int h = (int)(j / cnt);
-    const int c = (int)(j % cnt);
-    const int N = lens[i];
-    const int64_t span = C * kPage;
-    f.row = i;
-    f.h = h;
-    f.len = N;
-    f.tb = N > 0 ? (int)(c * span) : 0;
-    f.te = N > 0 ? (int)((c + 1) * span < N ? (c + 1) * span : N) : 0;
-    f.slot0 = (int)((int64_t)rs[i] * p.H_kv + (int64_t)h * cnt);
-    f.nslots = cnt;
-    f.valid = true;
+    f.row = res[0];
+    f.valid = f.row >= 0;
+    f.h = res[1];
+    f.tb = res[2];
+    f.te = res[3];
+    f.slot0 = res[4];
+    f.nslots = res[5];
+    f.len = res[6];
+    __syncthreads();  // every thread has read res before it is written again
     return f;
 }
 
@@ -1199,12 +1306,13 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     if (tid == 0)
         *spec_item = make_int4(-1, 0, 0, 0);
     int32_t *fill_scratch = reinterpret_cast<int32_t *>(smem);  // the idle ring, before any page copy
+    int32_t *fill_res = reinterpret_cast<int32_t *>(smem + C::kFillResOff);
     if (!p.pdl_early) {
         __syncthreads();
         const bool warm = (int)blockIdx.x < p.prefetch_blocks;
         if (p.mode == PKV_WORK_QUEUE && p.device_fill) {
             if (warm) {
-                const FillItem g = fill_queue_item<C::kThreads>(p, fill_scratch, true);
+                const FillItem g = fill_queue_item<C::kThreads>(p, fill_scratch, fill_res, true);
                 if (g.valid && tid == 0)
                     *spec_item = make_int4(g.row, g.h, g.tb, g.te);
                 if (g.valid && warp == NW)
@@ -1215,6 +1323,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         }
         __syncthreads();
         grid_dependency_wait();
+        PKV_TRACE_POINT(13);
     }
 
     // ---- which (row, KV head, token range) this block owns ----
@@ -1235,7 +1344,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
             if (idx < p.max_pages)
                 g_entry = __ldg(p.block_table + (int64_t)guess.x * p.max_pages + idx);
         }
-        const FillItem f = fill_queue_item<C::kThreads>(p, fill_scratch, false);
+        const FillItem f = fill_queue_item<C::kThreads>(p, fill_scratch, fill_res, false);
+        PKV_TRACE_POINT(14);
         if (!f.valid)
             return;
         hit = guess.x == f.row && guess.y == f.h && guess.z == f.tb && guess.w == f.te;
@@ -1249,7 +1359,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         e_first = g_entry;
         if (slot0 + nslots > p.n_items) {
             if (tid == 0)
-                atomicOr(p.ws_error, kErrItem);
+                raise_error(p, kErrItem);
             return;
         }
         if (warp == NW) {
@@ -1294,7 +1404,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         }
         if (!ok) {
             if (tid == 0)
-                atomicOr(p.ws_error, kErrItem);
+                raise_error(p, kErrItem);
             return;
         }
         if (warp == NW) {
@@ -1318,14 +1428,14 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         int N = __ldg(p.seq_lens + row);
         if (N < 0 || N > row_cap) {
             if (tid == 0)
-                atomicOr(p.ws_error, kErrSeqLen);
+                raise_error(p, kErrSeqLen);
             N = N < 0 ? 0 : (int)row_cap;
         }
         row_len = N;
         if (p.mode == PKV_SPLIT_S) {
             const int64_t span = (int64_t)p.chunk_pages * kPage;
             if (c == 0 && tid == 0 && (int64_t)S * span < N)
-                atomicOr(p.ws_error, kErrItem);  // the plan's S * C pages do not cover this row
+                raise_error(p, kErrItem);  // the plan's S * C pages do not cover this row
             const int64_t b = (int64_t)c * span;
             tb = (int)(b < N ? b : N);
             te = (int)(b < N ? (b + span < N ? b + span : N) : N);  // empty chunk: tb == te
@@ -1391,7 +1501,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
             e_next = base + 32 + lane < npages ? __ldg(bt + base + 32 + lane) : 0;
             const bool bad = base + lane < npages && (e < 0 || e >= p.num_pool_pages);
             if (__any_sync(0xffffffffu, bad) && lane == 0)
-                atomicOr(p.ws_error, kErrPageId);
+                raise_error(p, kErrPageId);
             if (bad)
                 e = 0;  // read a real page instead; the error bit reports the bad entry
             const int cnt = npages - base < 32 ? npages - base : 32;
@@ -1451,7 +1561,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
 #ifdef PKV_TRACE
             const long long tw0 = clock64();
 #endif
-            const bool ready = mbar_wait(bar_full + 8 * s, (pidx / NST) & 1, p.ws_error);
+            const bool ready = mbar_wait(bar_full + 8 * s, (pidx / NST) & 1, p.ws_error, kWaitLimitNs, p.host_err);
 #ifdef PKV_TRACE
             cons_wait += clock64() - tw0;
 #endif
@@ -1485,6 +1595,12 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     grid_launch_dependents();  // the next kernel may start its prologue
     __syncthreads();
     PKV_TRACE_POINT(3);
+    // A split (row, KV head): the idle producer thread takes the pair's ticket
+    // now, so that its round trip overlaps the combine; the state then travels
+    // under its slot's flag (set with release once stored, see below).
+    const bool merges = !CL && nslots > 1 && !p.separate_merge;
+    if (merges && warp == NW && lane == 0)
+        misc[0] = ticket_relaxed(p.ws_counters + pair) == (uint32_t)(nslots - 1);
     float *cb_o = reinterpret_cast<float *>(smem);
     float *cb_m = cb_o + NW * C::kGP * C::kOStride;
     float *cb_l = cb_m + NW * C::kGP;
@@ -1506,11 +1622,17 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
                 }
             }
     }
-    __syncthreads();
+    constexpr int kConsumers = NW * 32;
+    if (merges) {
+        named_barrier(1, kConsumers);  // the consumer warps only: the producer thread may still wait on its ticket
+    } else {
+        __syncthreads();
+    }
 
     constexpr int D4 = D / 4;
     const int G = p.G;
-    for (int e = tid; e < G * D4; e += C::kThreads) {
+    const int combiners = merges ? kConsumers : C::kThreads;
+    for (int e = tid; e < G * D4 && tid < combiners; e += combiners) {
         const int g = e / D4;
         const int d4 = (e % D4) * 4;
         float M = -INFINITY;
@@ -1588,14 +1710,18 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         cluster_sync_all();  // peers may still be reading this block's state
     }
     // ---- the last block of a split (row, KV head) merges its states ----
-    if (!CL && nslots > 1 && !p.separate_merge) {
-        __syncthreads();
-        if (tid == 0) {
-            const uint32_t prev = ticket_acq_rel(p.ws_counters + pair);
-            misc[0] = prev == (uint32_t)(nslots - 1);
-        }
-        __syncthreads();
-        if (misc[0]) {
+    if (merges) {
+        __syncthreads();  // this block's state is stored; misc[0] holds the ticket's verdict
+        if (!misc[0]) {
+            if (tid == 0)
+                flag_release(p.ws_flags + my_slot);
+        } else {
+            // every other block of the pair has its ticket, so it is running and
+            // sets its flag once its state is stored
+            for (int t = tid; t < nslots; t += C::kThreads)
+                if (slot0 + t != my_slot)
+                    wait_flag(p.ws_flags + slot0 + t, p.ws_error, p.host_err);
+            __syncthreads();
             uint32_t uses[2] = {0, 0};
             merge_pair_last_block<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid,
                                                   uses);
@@ -1605,6 +1731,299 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         }
     }
     PKV_TRACE_POINT(12);
+}
+
+// ---------------------------------------------------------------------------
+// Prefix-sharing grid (PKV_FLAG_SHARED_PREFIX): one block per unit of the
+// prefix-sharing queue.  A unit's members are items of up to 16 / G rows
+// that cover the same tokens of the same KV head on the same physical pages
+// (a prefix their block tables share ["Chapter 8 - Next-generation KV cache
+// management", 8.1 and 8.3]): each page is staged once and the tensor-core
+// tile carries the G query heads of every member (16 columns, two n = 8
+// tiles), so the shared K/V bytes cross HBM once per unit instead of once per
+// row.  Each member's partial state goes to its own slot (its item), and the
+// last block to finish a member's (row, KV head) merges that pair as in the
+// plain queue.  Units of one member are plain work items.
+
+constexpr int kMaxMembers = 16;
+constexpr int kPrefixSmemExtra = (8 * kMaxMembers + 16) * 4;  // member table of a unit
+
+// The prefix grid's counterpart of l2_prefetch_first_pages: the unit's first
+// member, read speculatively through L2 before the dependency wait.
+template <int D>
+__device__ __forceinline__ void l2_prefetch_unit(const Params &p, int lane, int64_t row_cap)
+{
+#if PKV_L2_PREFETCH_PAGES > 0
+    const int32_t *unit_ptr = p.indptr + p.B * p.H_kv + 1;
+    const int32_t *unit_items = unit_ptr + p.n_units + 1;
+    const int u0 = ld_l2_only(unit_ptr + blockIdx.x);
+    if (u0 < 0 || u0 >= p.n_items)
+        return;
+    const int x = ld_l2_only(unit_items + u0);
+    if (x < 0 || x >= p.n_items)
+        return;
+    const int4 it = ld_l2_only(p.items + x);
+    if (!(it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w && it.w <= row_cap))
+        return;
+    l2_prefetch_range<D>(p, lane, it.x, it.y, it.z / kPage, (it.w + kPage - 1) / kPage);
+#endif
+}
+
+template <int D, int NW, int NST>
+__global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) prefix_kernel(const __grid_constant__ Params p)
+{
+    constexpr int NT = 2;  // 16 query columns: the G heads of up to 16 / G members
+    using C = Cfg<D, NT, NW, NST>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // the members' table past the misc area (kPrefixSmemExtra bytes; no static shared memory, so the
+    // dynamic size may use everything an SM offers a block)
+    int *s_row = reinterpret_cast<int *>(smem + C::kMiscOff + 96);
+    int *s_item = s_row + kMaxMembers, *s_slot0 = s_item + kMaxMembers, *s_nslots = s_slot0 + kMaxMembers;
+    int *s_h = s_nslots + kMaxMembers, *s_tb = s_h + kMaxMembers, *s_te = s_tb + kMaxMembers;
+    int *s_last = s_te + kMaxMembers;
+    volatile int &s_bad = s_last[kMaxMembers];
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t k_ring = sbase;
+    const uint32_t v_ring = sbase + NST * C::kStageBytes;
+    const uint32_t bar_full = sbase + C::kBarOff;
+    const uint32_t bar_empty = bar_full + NST * 8;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t row_cap = (int64_t)p.max_pages * kPage;
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(sbase + C::kMiscOff + 8, 1);
+        mbar_init(sbase + C::kMiscOff + 16, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+        s_bad = 0;
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+    }
+    __syncthreads();
+    if (warp == NW && (int)blockIdx.x < p.prefetch_blocks)
+        l2_prefetch_unit<D>(p, lane, row_cap);
+    __syncthreads();
+    grid_dependency_wait();
+
+    // ---- the unit's members: same KV head, same tokens, own rows and slots ----
+    const int pairs = p.B * p.H_kv;
+    const int32_t *unit_ptr = p.indptr + pairs + 1;
+    const int32_t *unit_items = unit_ptr + p.n_units + 1;
+    const int u0 = __ldg(unit_ptr + blockIdx.x);
+    const int k = __ldg(unit_ptr + blockIdx.x + 1) - u0;
+    const int G = p.G;
+    if (u0 < 0 || k < 1 || k > kMaxMembers || k * G > 8 * NT || u0 + k > p.n_items) {
+        if (tid == 0)
+            raise_error(p, kErrItem);
+        return;
+    }
+    if (tid < k) {
+        const int x = __ldg(unit_items + u0 + tid);
+        bool ok = x >= 0 && x < p.n_items;
+        const int4 it = ok ? __ldg(p.items + x) : make_int4(-1, 0, 0, 0);
+        ok = ok && it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w &&
+             it.w <= row_cap && (it.z % kPage) == 0;
+        int slot0 = 0, nslots = 0;
+        if (ok) {
+            const int pair = it.x * p.H_kv + it.y;
+            slot0 = __ldg(p.indptr + pair);
+            nslots = __ldg(p.indptr + pair + 1) - slot0;
+            ok = nslots >= 1 && slot0 >= 0 && x >= slot0 && x < slot0 + nslots && slot0 + nslots <= p.n_items;
+        }
+        s_row[tid] = it.x;
+        s_item[tid] = x;
+        s_h[tid] = it.y;
+        s_tb[tid] = it.z;
+        s_te[tid] = it.w;
+        s_slot0[tid] = slot0;
+        s_nslots[tid] = nslots;
+        if (!ok)
+            s_bad = 1;
+    }
+    __syncthreads();
+    if (tid < k && (s_h[tid] != s_h[0] || s_tb[tid] != s_tb[0] || s_te[tid] != s_te[0]))
+        s_bad = 1;
+    __syncthreads();
+    if (s_bad) {
+        if (tid == 0)
+            raise_error(p, kErrItem);
+        return;
+    }
+    const int h = s_h[0];
+    const int tb = s_tb[0];
+    const int te = s_te[0];
+    const int row0 = s_row[0];
+    const int pg0 = tb / kPage;
+    const int npages = te > tb ? (te + kPage - 1) / kPage - pg0 : 0;
+
+    float m_run[NT][2], l_run[NT][2];
+    float o[D / 16][NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        m_run[nt][0] = m_run[nt][1] = -INFINITY;
+        l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+            o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    }
+    const int r = lane >> 2;
+    const int c4 = lane & 3;
+
+    if (warp == NW) {
+        // ================= producer: the first member's table (the pages are shared) =================
+        const int32_t *bt = p.block_table + (int64_t)row0 * p.max_pages + pg0;
+        const uint64_t policy = evict_first_policy();
+        int e_next = lane < npages ? __ldg(bt + lane) : 0;
+        bool ok = true;
+        int gp = 0;
+        for (int base = 0; base < npages && ok; base += 32) {
+            int e = e_next;
+            e_next = base + 32 + lane < npages ? __ldg(bt + base + 32 + lane) : 0;
+            const bool bad = base + lane < npages && (e < 0 || e >= p.num_pool_pages);
+            if (__any_sync(0xffffffffu, bad) && lane == 0)
+                raise_error(p, kErrPageId);
+            if (bad)
+                e = 0;
+            const int cnt = npages - base < 32 ? npages - base : 32;
+            ok = issue_pages<D, NST>(p, lane, e, cnt, gp, h, k_ring, v_ring, bar_full, bar_empty, policy);
+        }
+    } else {
+        // ================= consumers: column j = member (j / G), head (j % G) =================
+        uint32_t qf[D / 16][NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int j = nt * 8 + r;
+            const int m = j / G;
+            const bool live = m < k;
+            const __nv_bfloat16 *qb =
+                p.q + ((int64_t)(live ? s_row[m] : 0) * p.H_q + (int64_t)h * G + (live ? j % G : 0)) * D;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t lo = 0, hi = 0;
+                if (live) {
+                    const uint32_t *src = reinterpret_cast<const uint32_t *>(qb + ks * 16 + 2 * c4);
+                    lo = __ldg(src);
+                    hi = __ldg(src + 4);
+                }
+                qf[ks][nt][0] = lo;
+                qf[ks][nt][1] = hi;
+            }
+        }
+        const int mi = lane >> 3;
+        const int ri = lane & 7;
+        const uint32_t k_off = (uint32_t)((8 * (mi & 1) + ri) * 128);
+        const int k_hi = mi >> 1;
+        const uint32_t v_off = (uint32_t)((8 * (mi >> 1) + ri) * 128);
+        const int v_hi = mi & 1;
+        const float sl2 = p.scale_log2;
+        for (int pidx = warp; pidx < npages; pidx += NW) {
+            const int s = pidx % NST;
+            const bool ready = mbar_wait(bar_full + 8 * s, (pidx / NST) & 1, p.ws_error, kWaitLimitNs, p.host_err);
+            if (!__all_sync(0xffffffffu, ready))
+                break;
+            const int tok0 = (pg0 + pidx) * kPage;
+            const int nvalid = te - tok0 < kPage ? te - tok0 : kPage;
+            attend_page<D, NT>(smem, sbase, k_ring + s * C::kStageBytes, v_ring + s * C::kStageBytes,
+                               bar_empty + 8 * s, nvalid, lane, r, ri, k_off, k_hi, v_off, v_hi, sl2, qf, m_run,
+                               l_run, o);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int sh = 4; sh < 32; sh <<= 1)
+                    l_run[nt][j] += __shfl_xor_sync(0xffffffffu, l_run[nt][j], sh);
+    }
+
+    // ---- combine the warps' states per column; each member's to its own slot ----
+    grid_launch_dependents();
+    __syncthreads();
+    float *cb_o = reinterpret_cast<float *>(smem);
+    float *cb_m = cb_o + NW * C::kGP * C::kOStride;
+    float *cb_l = cb_m + NW * C::kGP;
+    if (warp < NW) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int g = nt * 8 + 2 * c4 + j;
+                float *dst = cb_o + (warp * C::kGP + g) * C::kOStride;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    dst[mt * 16 + r] = o[mt][nt][j];
+                    dst[mt * 16 + r + 8] = o[mt][nt][2 + j];
+                }
+                if (r == 0) {
+                    cb_m[warp * C::kGP + g] = m_run[nt][j];
+                    cb_l[warp * C::kGP + g] = l_run[nt][j];
+                }
+            }
+    }
+    __syncthreads();
+    constexpr int D4 = D / 4;
+    for (int e = tid; e < k * G * D4; e += C::kThreads) {
+        const int col = e / D4;
+        const int d4 = (e % D4) * 4;
+        const int m = col / G;
+        const int g = col % G;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            M = fmaxf(M, cb_m[w * C::kGP + col]);
+        float L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float mw = cb_m[w * C::kGP + col];
+            if (mw == -INFINITY)
+                continue;
+            const float sc = exp2_approx(mw - M);
+            L = fmaf(cb_l[w * C::kGP + col], sc, L);
+            O = fma4(*reinterpret_cast<const float4 *>(cb_o + (w * C::kGP + col) * C::kOStride + d4), sc, O);
+        }
+        if (s_nslots[m] == 1) {
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            store_bf16x4(p.out + ((int64_t)s_row[m] * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+        } else {
+            const int64_t idx = (int64_t)s_item[m] * G + g;
+            *reinterpret_cast<float4 *>(p.ws_acc + idx * D + d4) = O;
+            if (d4 == 0) {
+                p.ws_m[idx] = M;
+                p.ws_l[idx] = L;
+            }
+        }
+    }
+    if (p.separate_merge)
+        return;
+    // ---- tickets: the last block of a member's (row, KV head) merges it ----
+    __syncthreads();
+    if (tid < k) {
+        s_last[tid] = 0;
+        if (s_nslots[tid] > 1) {
+            const uint32_t prev = ticket_acq_rel(p.ws_counters + s_row[tid] * p.H_kv + h);
+            s_last[tid] = prev == (uint32_t)(s_nslots[tid] - 1);
+        }
+    }
+    __syncthreads();
+    uint32_t uses[2] = {0, 0};
+    for (int m = 0; m < k; ++m) {
+        if (!s_last[m])
+            continue;
+        merge_pair_last_block<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, s_row[m], h, s_slot0[m], s_nslots[m],
+                                              tid, uses);
+        if (tid == 0)
+            p.ws_counters[s_row[m] * p.H_kv + h] = 0u;  // ready for the next call
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1722,7 +2141,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
     const int it1 = __ldg(block_ptr + blockIdx.x + 1);
     if (it0 < 0 || it1 < it0 || it1 > p.n_items) {
         if (tid == 0)
-            atomicOr(p.ws_error, kErrItem);
+            raise_error(p, kErrItem);
         return;
     }
     __syncthreads();  // the barriers' initialisation is visible to all warps
@@ -1738,13 +2157,13 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
             const int4 item = __ldg(p.items + it);
             int pg0, np;
             if (!item_pages(p, item, pg0, np) && lane == 0)
-                atomicOr(p.ws_error, kErrItem);
+                raise_error(p, kErrItem);
             const int32_t *bt = p.block_table + (int64_t)item.x * p.max_pages + pg0;
             for (int base = 0; base < np && ok; base += 32) {
                 int e = base + lane < np ? __ldg(bt + base + lane) : 0;
                 const bool bad = base + lane < np && (e < 0 || e >= p.num_pool_pages);
                 if (__any_sync(0xffffffffu, bad) && lane == 0)
-                    atomicOr(p.ws_error, kErrPageId);
+                    raise_error(p, kErrPageId);
                 if (bad)
                     e = 0;
                 const int cnt = np - base < 32 ? np - base : 32;
@@ -1797,7 +2216,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
             // this warp's pages of the item: global page index gp with gp % NW == warp
             for (int gp = gp_base + ((warp - gp_base % NW) + NW) % NW; alive && gp < gp_base + np; gp += NW) {
                 const int s = gp % NST;
-                const bool ready = mbar_wait(bar_full + 8 * s, (gp / NST) & 1, p.ws_error);
+                const bool ready = mbar_wait(bar_full + 8 * s, (gp / NST) & 1, p.ws_error, kWaitLimitNs, p.host_err);
                 if (!__all_sync(0xffffffffu, ready)) {
                     alive = false;
                     break;
@@ -1840,7 +2259,7 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
             const bool slot_ok = item_ok && nslots >= 1 && slot0 >= 0 && it >= slot0 && it < slot0 + nslots &&
                                  slot0 + nslots <= p.n_items;
             if (!slot_ok && item_ok && tid == 0)
-                atomicOr(p.ws_error, kErrItem);
+                raise_error(p, kErrItem);
             if (slot_ok) {
                 for (int e = tid; e < G * D4; e += kConsumers) {
                     const int g = e / D4;
@@ -1941,7 +2360,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
         nslots = __ldg(p.indptr + pair + 1) - slot0;
         if (slot0 < 0 || nslots < 0 || slot0 + nslots > p.n_items) {
             if (threadIdx.x == 0)
-                atomicOr(p.ws_error, kErrItem);
+                raise_error(p, kErrItem);
             return;
         }
     }
@@ -2575,6 +2994,31 @@ cudaError_t launch_balanced_nst(int D, int NT, const Params &prm, int64_t grid, 
     return NT == 1 ? launch_balanced<64, 1, NST>(prm, grid, st, pdl) : launch_balanced<64, 2, NST>(prm, grid, st, pdl);
 }
 
+template <int D, int NST>
+cudaError_t launch_prefix(const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+{
+    using C = Cfg<D, 2, kNW, NST>;
+    static std::atomic<uint64_t> configured{0};
+    auto kernel = prefix_kernel<D, kNW, NST>;
+    cudaError_t e = set_smem(kernel, kMaxDynSmem, configured);
+    if (e != cudaSuccess)
+        return e;
+    static std::atomic<uint64_t> occ_cache[64] = {};
+    const Occupancy o = occupancy(kernel, C::kThreads, C::kSmemBytes + kPrefixSmemExtra, occ_cache);
+    Params q = prm;
+    q.prefetch_blocks = o.per_sm * o.sms;
+    e = launch_ex(kernel, (unsigned)grid, C::kThreads, spread_smem(o, C::kSmemBytes + kPrefixSmemExtra, grid), st,
+                  pdl, q);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_prefix_any(int D, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+{
+    if (D == 128)
+        return deep ? launch_prefix<128, kNSTDeep>(prm, grid, st, pdl) : launch_prefix<128, kNST>(prm, grid, st, pdl);
+    return deep ? launch_prefix<64, kNSTDeep>(prm, grid, st, pdl) : launch_prefix<64, kNST>(prm, grid, st, pdl);
+}
+
 cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl,
                              unsigned cluster)
 {
@@ -2606,7 +3050,9 @@ int check_fast_path(const pkv_shape &s)
 struct WsPtrs {
     uint32_t *error;
     uint32_t *counters;
+    uint32_t *flags;
     float *m, *l, *acc;
+    uint32_t *host_err = nullptr;  // flag words in mapped host memory (pkv_decode_host), or NULL
 };
 
 // Internal entry shared by pkv_paged_decode, pkv_paged_decode_noalloc and
@@ -2631,7 +3077,14 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     if (pl.mode == PKV_SPLIT_S && (pl.num_splits < 1 || pl.chunk_pages < 1))
         return PKV_ERR_INVALID;
     const bool device_fill = (pl.flags & PKV_FLAG_DEVICE_FILL) != 0;
-    if (device_fill) {
+    const bool shared_prefix = (pl.flags & PKV_FLAG_SHARED_PREFIX) != 0;
+    if (shared_prefix) {
+        // the prefix-sharing queue: num_splits carries the unit count (the grid)
+        if (pl.mode != PKV_WORK_QUEUE || device_fill || (pl.flags & PKV_FLAG_PDL_EARLY))
+            return PKV_ERR_UNSUPPORTED;
+        if (!items || !indptr || n_items < (int64_t)s.B * s.H_kv || pl.num_splits < 1 || pl.num_splits > n_items)
+            return PKV_ERR_INVALID;
+    } else if (device_fill) {
         // each block derives its item: the grid must hold the longest queue the fill rule allows
         if (pl.mode != PKV_WORK_QUEUE || (pl.flags & PKV_FLAG_SEPARATE_MERGE) || s.B > kFillMaxRows)
             return PKV_ERR_UNSUPPORTED;
@@ -2673,6 +3126,7 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         uint8_t *wsb = static_cast<uint8_t *>(workspace);
         wp.error = reinterpret_cast<uint32_t *>(wsb + ws.error_off);
         wp.counters = reinterpret_cast<uint32_t *>(wsb + ws.counters_off);
+        wp.flags = reinterpret_cast<uint32_t *>(wsb + ws.flags_off);
         wp.m = reinterpret_cast<float *>(wsb + ws.m_off);
         wp.l = reinterpret_cast<float *>(wsb + ws.l_off);
         wp.acc = reinterpret_cast<float *>(wsb + ws.acc_off);
@@ -2691,7 +3145,9 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.items = reinterpret_cast<const int4 *>(items);
     prm.indptr = indptr;
     prm.ws_error = wp.error;
+    prm.host_err = wp.host_err;
     prm.ws_counters = wp.counters;
+    prm.ws_flags = wp.flags;
     prm.ws_m = wp.m;
     prm.ws_l = wp.l;
     prm.ws_acc = wp.acc;
@@ -2709,6 +3165,7 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.pdl_early = (pl.flags & PKV_FLAG_PDL_EARLY) && !(pl.flags & PKV_FLAG_NO_PDL) ? 1 : 0;
     prm.n_items = n_items;
     prm.device_fill = device_fill ? 1 : 0;
+    prm.n_units = shared_prefix ? pl.num_splits : 0;
     prm.fill_blocks = device_fill ? pl.num_splits : 0;
 #ifdef PKV_TRACE
     static std::atomic<int32_t> trace_launches{0};
@@ -2718,8 +3175,8 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     const int64_t pairs = (int64_t)s.B * s.H_kv;
     const int64_t grid = pl.mode == PKV_NO_SPLIT ? pairs
                          : pl.mode == PKV_SPLIT_S ? pairs * pl.num_splits
-                         : pl.mode == PKV_BALANCED ? (int64_t)pl.num_splits
-                                                   : n_items;
+                         : pl.mode == PKV_BALANCED || shared_prefix ? (int64_t)pl.num_splits
+                                                                     : n_items;
     if (grid > INT32_MAX || pairs > INT32_MAX)
         return PKV_ERR_UNSUPPORTED;
     const int NT = prm.G <= 8 ? 1 : 2;
@@ -2733,6 +3190,8 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     if (pl.mode == PKV_BALANCED)
         le = deep ? launch_balanced_nst<PKV_NST_BAL_DEEP>(s.head_dim, NT, prm, grid, st, pdl)
                   : launch_balanced_nst<PKV_NST_BAL>(s.head_dim, NT, prm, grid, st, pdl);
+    else if (shared_prefix)
+        le = launch_prefix_any(s.head_dim, deep, prm, grid, st, pdl);
     else
         le = launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl, cluster);
     if (le != cudaSuccess)
@@ -2961,10 +3420,24 @@ struct HostLayout {
     int32_t n_items = 0, n_indptr = 0;
     bool q_inline, bt_inline, out_inline;
     size_t q_bytes, bt_bytes;
-    size_t q_off, lens_off, items_off, indptr_off, bt_off, counters_off, err_off, out_off, m_off, l_off, acc_off;
+    size_t q_off, lens_off, items_off, indptr_off, bt_off, counters_off, flags_off, err_off, out_off, m_off, l_off,
+        acc_off;
     size_t up_bytes, down_bytes, dev_total;
     size_t h_down_off, host_total;
 };
+
+// The device address of host memory the GPU can reach (page-locked and
+// mapped, as every page-locked allocation is under unified addressing), or
+// NULL for any other pointer.
+void *device_view(const void *host)
+{
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+        cudaGetLastError();  // an unregistered pointer is not an error here
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
 
 // Four timing events per device for pkv_decode_host_timed, made on first use.
 cudaEvent_t *timing_events()
@@ -3024,7 +3497,8 @@ int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_ru
     L->items_off = take(L->n_indptr > 0 ? (size_t)L->n_items * sizeof(pkv_work_item) : 0);
     L->indptr_off = take((size_t)L->n_indptr * 4);
     L->bt_off = L->bt_inline ? take(L->bt_bytes) : 0;
-    L->counters_off = take(ws.m_off - ws.counters_off);
+    L->counters_off = take(ws.m_off - ws.counters_off);  // the counters, then the flags
+    L->flags_off = L->counters_off + (ws.flags_off - ws.counters_off);
     L->err_off = take(kWsAlign);
     L->up_bytes = L->err_off + 16;
     L->out_off = take(L->q_bytes);
@@ -3130,6 +3604,16 @@ int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *dev = static_cast<uint8_t *>(device_buffer);
     uint8_t *hst = static_cast<uint8_t *>(host_staging);
+    // When out_host and the staging buffer are page-locked, the kernels write
+    // out straight into out_host and report errors as flag words in the
+    // staging buffer: the result needs no device->host copy.
+    void *out_dev = device_view(out_host);
+    uint8_t *stage_dev = out_dev ? static_cast<uint8_t *>(device_view(hst)) : nullptr;
+    const bool direct = out_dev && stage_dev && aligned(out_dev, 16);
+    volatile uint32_t *h_flags = reinterpret_cast<volatile uint32_t *>(hst + L.h_down_off);
+    if (direct)
+        for (int k = 0; k < 4; ++k)
+            h_flags[k] = 0u;
     // upload image: inputs, queue, zeroed counters and error word
     if (L.q_inline)
         std::memcpy(hst + L.q_off, q_host, L.q_bytes);
@@ -3159,29 +3643,39 @@ int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, c
     if (!ok)
         return PKV_ERR_CUDA;
     const WsPtrs wp{reinterpret_cast<uint32_t *>(dev + L.err_off), reinterpret_cast<uint32_t *>(dev + L.counters_off),
-                    reinterpret_cast<float *>(dev + L.m_off), reinterpret_cast<float *>(dev + L.l_off),
-                    reinterpret_cast<float *>(dev + L.acc_off)};
+                    reinterpret_cast<uint32_t *>(dev + L.flags_off), reinterpret_cast<float *>(dev + L.m_off),
+                    reinterpret_cast<float *>(dev + L.l_off),
+                    reinterpret_cast<float *>(dev + L.acc_off),
+                    direct ? reinterpret_cast<uint32_t *>(stage_dev + L.h_down_off) : nullptr};
     rc = paged_decode_impl(dev + L.q_off, k_pool, v_pool, reinterpret_cast<const int32_t *>(dev + L.bt_off),
-                           reinterpret_cast<const int32_t *>(dev + L.lens_off), s.page_size, scale, dev + L.out_off,
-                           shape, &L.plan, reinterpret_cast<const pkv_work_item *>(dev + L.items_off),
+                           reinterpret_cast<const int32_t *>(dev + L.lens_off), s.page_size, scale,
+                           direct ? out_dev : dev + L.out_off, shape, &L.plan,
+                           reinterpret_cast<const pkv_work_item *>(dev + L.items_off),
                            reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, nullptr, 0, st, &wp);
     if (rc != PKV_OK)
         return rc;
     ok = !ev || cudaEventRecord(ev[2], st) == cudaSuccess;
     uint8_t *h_down = hst + L.h_down_off;
-    ok = ok && cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
-    if (ok && !L.out_inline)
-        ok = cudaMemcpyAsync(out_host, dev + L.out_off, L.q_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    if (!direct) {
+        ok = ok && cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+        if (ok && !L.out_inline)
+            ok = cudaMemcpyAsync(out_host, dev + L.out_off, L.q_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    }
     if (ok && ev)
         ok = cudaEventRecord(ev[3], st) == cudaSuccess;
     const clock::time_point t2 = clock::now();
     if (!ok || cudaStreamSynchronize(st) != cudaSuccess)
         return PKV_ERR_CUDA;
     const clock::time_point t3 = clock::now();
-    if (L.out_inline)
-        std::memcpy(out_host, h_down + (L.out_off - L.err_off), L.q_bytes);
-    uint32_t err;
-    std::memcpy(&err, h_down, 4);
+    uint32_t err = 0;
+    if (direct) {
+        for (int k = 0; k < 4; ++k)
+            err |= h_flags[k] ? (1u << k) : 0u;
+    } else {
+        if (L.out_inline)
+            std::memcpy(out_host, h_down + (L.out_off - L.err_off), L.q_bytes);
+        std::memcpy(&err, h_down, 4);
+    }
     if (timing) {
         const clock::time_point t4 = clock::now();
         auto us = [](clock::duration d) { return std::chrono::duration<double, std::micro>(d).count(); };

@@ -61,6 +61,8 @@ int check_rules(const pkv_policy_rule *rules, int32_t n)
             return PKV_ERR_INVALID;
         if ((r.flags & PKV_FLAG_DEVICE_FILL) && (r.mode != PKV_WORK_QUEUE || r.chunk_pages != 0))
             return PKV_ERR_INVALID;
+        if (r.flags & PKV_FLAG_SHARED_PREFIX)  // needs the block table: planned by the caller
+            return PKV_ERR_INVALID;
     }
     return PKV_OK;
 }
@@ -387,6 +389,8 @@ int pkv_plan_counters(const int32_t *seq_lens_host, const pkv_shape *shape, cons
         break;
     }
     case PKV_WORK_QUEUE: {
+        if (plan->flags & PKV_FLAG_SHARED_PREFIX)  // the units depend on the block table
+            return PKV_ERR_UNSUPPORTED;
         const bool device_fill = (plan->flags & PKV_FLAG_DEVICE_FILL) != 0;
         int64_t Cq = C;
         if (device_fill) {  // the chunk the blocks find on the device for these lengths

@@ -25,9 +25,10 @@ permutation of the pool is dealt to the rows in order, so every row's pages
 are scattered.  Seeds: 20260622 calibrates the policy, 20260623 is reported.
 
 With poison=True every pool page no row uses, every slot past a row's last
-token in its tail page, and every block-table entry past a row's last page
-(pointed at a poisoned page) holds bf16 NaN, so any read outside a row's real
-tokens shows up in the output.
+token in its tail page (unless another row that shares the page reads that
+slot as one of its own tokens), and every block-table entry past a row's last
+page (pointed at a poisoned page) holds bf16 NaN, so any read outside a row's
+real tokens shows up in the output.
 """
 from __future__ import annotations
 
@@ -216,9 +217,17 @@ def _materialise(name, seed, device, poison, layout, q_scale, g, B, H_q, H_kv, D
             idx = torch.tensor(unused, dtype=torch.long, device=dev)
             k_pool[idx] = nan
             v_pool[idx] = nan
+        # a row's partial last page is poisoned past its last token unless another
+        # row reads that page further (a shared page one row ends inside)
+        covered = {}
+        for i, n in enumerate(lens):
+            for j, page in enumerate(tables[i]):
+                covered[page] = max(covered.get(page, 0), min(P, n - j * P))
         for i, n in enumerate(lens):
             if n % P and tables[i]:
                 last = tables[i][-1]
+                if covered[last] > n % P:
+                    continue
                 k_pool[last, :, n % P:, :] = nan
                 v_pool[last, :, n % P:, :] = nan
     if layout == "NHD":

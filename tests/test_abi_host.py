@@ -280,3 +280,25 @@ def test_prefix_queue_matches_oracle_bit_for_bit(L):
         assert [tuple(x) for x in items.tolist()] == o_items, (lens, bt, H_kv, P, C, M)
         assert indptr.tolist() == o_indptr + o_uptr + o_uitems, (lens, bt, H_kv, P, C, M)
         assert n_units == len(o_uptr) - 1
+
+
+def test_prefix_plan_counters_recount(L):
+    """The prefix plan's counters: one block per unit, a unit's pages once."""
+    for lens, bt, H_kv, P, C, M in host_pins._prefix_cases(seed=43, n=30):
+        if P != 16:
+            continue
+        width = max(len(r) for r in bt)
+        table = torch.tensor([list(r) for r in bt], dtype=torch.int32)
+        shape = bd.make_shape(len(lens), 4 * H_kv, H_kv, 64, P, width, 1)
+        items, indptr, n_units = bd.build_prefix_queue(lens, table, shape, C, M)
+        c = bd.prefix_counters(lens, shape, items, indptr, n_units)
+        o_items, o_indptr, o_uptr, o_uitems = O.build_prefix_queue(lens, bt, H_kv, P, C, M)
+        pages = 0
+        for u in range(len(o_uptr) - 1):
+            pages += len({(o_items[x][1], pg) for x in o_uitems[o_uptr[u]:o_uptr[u + 1]]
+                          for pg in range(o_items[x][2] // P, -(-o_items[x][3] // P))})
+        assert c["kv_bytes_streamed"] == pages * P * 2 * 64 * 2, (lens, bt, H_kv, C, M)
+        assert c["work_items"] == len(o_uptr) - 1 and c["queue_bytes"] == 16 * len(o_items) + 4 * (
+            len(o_indptr) + len(o_uptr) + len(o_uitems))
+        plain = O.counters(lens, 4 * H_kv, H_kv, 64, P, (O.WORK_QUEUE, 1, C, 0))
+        assert c["kv_bytes_streamed"] <= plain.kv_bytes_streamed

@@ -133,3 +133,27 @@ def test_host_path_empty_rows():
     w = to_device(W.make_custom([0, 0], 8, 2, 64, seed=134, poison=True))
     got, _ = host_decode(w)
     assert (got == 0).all()
+
+
+@pytest.mark.parametrize("name", ["split7", "wq16_sep", "bal37"])
+def test_pageable_out_takes_the_copy_and_matches_the_direct_path(name):
+    """Page-locked out: the kernels write the result straight into it; a
+    pageable out takes the packed device->host copy.  Same kernels, same
+    bits; a device-input error is reported on both paths."""
+    w = to_device(W.make_custom([1000, 4097, 2500, 17, 0], 32, 8, 128, seed=135, poison=True))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    q_h, bt_h, lens_h, out_pinned = host_inputs(w)
+    out_pageable = torch.full_like(out_pinned, float("nan"))
+    assert not out_pageable.is_pinned()
+    dec = bd.HostDecoder("cuda")
+    dec.ensure(lens_h, shape, [PLANS[name]])
+    dec(q_h, bt_h, lens_h, out_pinned, w.k_pool, w.v_pool, w.scale, shape, rules=[PLANS[name]])
+    dec(q_h, bt_h, lens_h, out_pageable, w.k_pool, w.v_pool, w.scale, shape, rules=[PLANS[name]])
+    assert torch.equal(out_pinned, out_pageable)
+    assert_close(out_pageable.float().double().numpy(), oracle_full(w), f"pageable/{name}")
+    bad = bt_h.clone()
+    bad[1, 3] = w.num_pages + 2
+    for out in (out_pinned, out_pageable):
+        with pytest.raises(bd.PkvError) as e:
+            dec(q_h, bad, lens_h, out, w.k_pool, w.v_pool, w.scale, shape, rules=[PLANS[name]])
+        assert e.value.status == -6
