@@ -60,7 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="long",
-                    choices=["tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf"])
+                    choices=["tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf", "long_g1",
+                             "long_g2", "long_g8", "long_g16", "prefix_small"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=None)
     ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end timing (default: --steps)")
@@ -68,6 +69,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=8.0, help="target CPU time of the cpu_baseline sample")
     ap.add_argument("--no-graph", action="store_true", help="queue the timed steps from Python, not a CUDA graph")
+    ap.add_argument("--shared-prefix", action="store_true",
+                    help="run the headline workload in the prefix-sharing plan (PKV_FLAG_SHARED_PREFIX)")
     return ap.parse_args(argv)
 
 
@@ -334,6 +337,21 @@ def device_queue_timing(w, dp, K, W, torch, bd, copies):
                     "(host queue: fixed lengths)"}
 
 
+def shared_prefix_timing(w, dp, K, W, torch, bd, copies):
+    """Steady-state µs per step of the prefix-sharing plan beside the built-in
+    one, for a workload whose rows share leading pages; None otherwise."""
+    if w.shared_rows < 2:
+        return None
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dpp = bd.plan_decode(w.seq_lens, shape, w.q.device, plan=dp.plan, shared_prefix_table=w.block_table.cpu())
+    steady = time_steady(w, dpp, K, W, torch, bd, copies) / K
+    c = dpp.counters
+    return {"plan": {"mode": "WORK_QUEUE", "units": dpp.plan.num_splits, "chunk_pages": dpp.plan.chunk_pages,
+                     "flags": dpp.plan.flags}, "items": dpp.n_items, "us_per_step": round(steady * 1e3, 2),
+            "kv_bytes_streamed": c["kv_bytes_streamed"], "built_in_kv_bytes_streamed": dp.counters["kv_bytes_streamed"],
+            "note": "shared chunks staged once per unit of up to 16/G sharing rows (PKV_FLAG_SHARED_PREFIX)"}
+
+
 def measure_workload(name, seed, device, K, W, torch, bd, W_mod, flush):
     w = W_mod.make(name, seed=seed, device=device)
     shape = bd.shape_of(w.q, w.k_pool, w.block_table)
@@ -342,9 +360,10 @@ def measure_workload(name, seed, device, K, W, torch, bd, W_mod, flush):
     steady = time_steady(w, dp, K, W, torch, bd, copies) / K
     inter, _ = time_interleaved(w, dp, K, W, torch, bd, copies)
     dq = device_queue_timing(w, dp, K, W, torch, bd, copies)
+    sp = shared_prefix_timing(w, dp, K, W, torch, bd, copies)
     del copies
     iso = time_isolated(w, dp, min(K, 50), min(W, 3), torch, bd, flush)
-    return {"w": w, "dp": dp, "ms": steady, "inter_ms": inter / K, "device_queue": dq,
+    return {"w": w, "dp": dp, "ms": steady, "inter_ms": inter / K, "device_queue": dq, "shared_prefix": sp,
             "iso_ms": statistics.median(iso), "bytes": w.algorithmic_bytes(), "bytes_unique": w.algorithmic_bytes(True)}
 
 
@@ -391,7 +410,8 @@ def run_ours(args):
     # the headline workload: warm-up, then EXACTLY K timed steps between barriers
     w = W_mod.make(args.workload, seed=seed, device=device)
     shape = bd.shape_of(w.q, w.k_pool, w.block_table)
-    dp = bd.plan_decode(w.seq_lens, shape, device)
+    dp = bd.plan_decode(w.seq_lens, shape, device,
+                        shared_prefix_table=w.block_table.cpu() if args.shared_prefix else None)
     copies = pool_copies(w, torch)
     barrier(dist, device)
     torch.cuda.synchronize()
@@ -460,7 +480,8 @@ def run_ours(args):
         "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4),
         "roofline": {
             "bound": "hbm",
-            "kernel": "split_kernel (fused merge)" if counters["launches"] == 1 else "split_kernel + merge_kernel",
+            "kernel": ("prefix_kernel" if dp.plan.flags & bd.FLAG_SHARED_PREFIX else "split_kernel") +
+                      (" (fused merge)" if counters["launches"] == 1 else " + merge_kernel"),
             "achieved": round(achieved, 2),
             "peak": peak,
             "peak_source": f"{peak_src} HBM copy bandwidth",
@@ -509,6 +530,8 @@ def run_ours(args):
                            "launches": r["dp"].counters["launches"]}
             if r["device_queue"] is not None:
                 extra[name]["device_queue"] = r["device_queue"]
+            if r["shared_prefix"] is not None:
+                extra[name]["shared_prefix"] = r["shared_prefix"]
             if r["bytes_unique"] != r["bytes"]:
                 gbu = r["bytes_unique"] / (m * 1e-3) / 1e9
                 extra[name]["GB_s_unique"] = round(gbu, 1)

@@ -85,7 +85,6 @@ struct __align__(64) Params {
     float *ws_l;
     float *ws_acc;
     uint32_t *ws_counters;
-    uint32_t *ws_flags;  // per slot: its partial state is written (set by its block, cleared by the merger)
     uint32_t *ws_error;
     float scale_log2;  // scale * log2(e): logits are kept in the log2 domain
     int32_t B, H_q, H_kv, G, max_pages, num_pool_pages;
@@ -251,50 +250,6 @@ __device__ __forceinline__ uint32_t ticket_acq_rel(uint32_t *ctr)
     uint32_t prev;
     asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr) : "memory");
     return prev;
-}
-
-// The split kernel's ticket, taken as soon as a block's pages are done: a
-// relaxed increment, since the states travel under their own flags.
-__device__ __forceinline__ uint32_t ticket_relaxed(uint32_t *ctr)
-{
-    uint32_t prev;
-    asm volatile("atom.add.relaxed.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr) : "memory");
-    return prev;
-}
-
-// A slot's "state written" flag: set with release (after the block's state
-// stores, made visible to the setting thread by a barrier), read with acquire.
-__device__ __forceinline__ void flag_release(uint32_t *f)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(1u) : "memory");
-}
-
-__device__ __forceinline__ uint32_t flag_acquire(const uint32_t *f)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
-    return v;
-}
-
-// Wait until a slot's flag is set, then clear it for the next call.  The
-// block that sets it has already taken its ticket, so it is running and
-// sets the flag within a few microseconds; the wait still gives up after
-// kWaitLimitNs with the timeout bit set.
-__device__ __noinline__ bool wait_flag(uint32_t *f, uint32_t *err, uint32_t *host_flags)
-{
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t i = 0; i < kWaitLimitIters; ++i) {
-        if (flag_acquire(f)) {
-            *f = 0u;
-            return true;
-        }
-        if ((i & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs)
-            break;
-    }
-    atomicOr(err, kErrTimeout);
-    if (host_flags)
-        *reinterpret_cast<volatile uint32_t *>(host_flags) = 1u;
-    return false;
 }
 
 __device__ __forceinline__ void fence_proxy_async_global()
@@ -1106,7 +1061,7 @@ __device__ __forceinline__ uint32_t fill_search(uint32_t lo, uint32_t hi, uint32
 }
 
 template <int NTHREADS>
-__device__ __noinline__ FillItem fill_queue_item(const Params &p, int32_t *sm, int32_t *res, bool speculative)
+__device__ __forceinline__ FillItem fill_queue_item(const Params &p, int32_t *sm, int32_t *res, bool speculative)
 {
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -1141,6 +1096,8 @@ __device__ __noinline__ FillItem fill_queue_item(const Params &p, int32_t *sm, i
             U += __shfl_xor_sync(0xffffffffu, U, off);
         }
         __syncwarp();
+        if (!speculative)
+            PKV_TRACE_POINT(15);
         // items of one head at chunk c
         auto count = [&](uint32_t c) {
             uint32_t n = 0;
@@ -1595,12 +1552,6 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     grid_launch_dependents();  // the next kernel may start its prologue
     __syncthreads();
     PKV_TRACE_POINT(3);
-    // A split (row, KV head): the idle producer thread takes the pair's ticket
-    // now, so that its round trip overlaps the combine; the state then travels
-    // under its slot's flag (set with release once stored, see below).
-    const bool merges = !CL && nslots > 1 && !p.separate_merge;
-    if (merges && warp == NW && lane == 0)
-        misc[0] = ticket_relaxed(p.ws_counters + pair) == (uint32_t)(nslots - 1);
     float *cb_o = reinterpret_cast<float *>(smem);
     float *cb_m = cb_o + NW * C::kGP * C::kOStride;
     float *cb_l = cb_m + NW * C::kGP;
@@ -1622,17 +1573,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
                 }
             }
     }
-    constexpr int kConsumers = NW * 32;
-    if (merges) {
-        named_barrier(1, kConsumers);  // the consumer warps only: the producer thread may still wait on its ticket
-    } else {
-        __syncthreads();
-    }
+    __syncthreads();
 
     constexpr int D4 = D / 4;
     const int G = p.G;
-    const int combiners = merges ? kConsumers : C::kThreads;
-    for (int e = tid; e < G * D4 && tid < combiners; e += combiners) {
+    for (int e = tid; e < G * D4; e += C::kThreads) {
         const int g = e / D4;
         const int d4 = (e % D4) * 4;
         float M = -INFINITY;
@@ -1710,18 +1655,14 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         cluster_sync_all();  // peers may still be reading this block's state
     }
     // ---- the last block of a split (row, KV head) merges its states ----
-    if (merges) {
-        __syncthreads();  // this block's state is stored; misc[0] holds the ticket's verdict
-        if (!misc[0]) {
-            if (tid == 0)
-                flag_release(p.ws_flags + my_slot);
-        } else {
-            // every other block of the pair has its ticket, so it is running and
-            // sets its flag once its state is stored
-            for (int t = tid; t < nslots; t += C::kThreads)
-                if (slot0 + t != my_slot)
-                    wait_flag(p.ws_flags + slot0 + t, p.ws_error, p.host_err);
-            __syncthreads();
+    if (!CL && nslots > 1 && !p.separate_merge) {
+        __syncthreads();
+        if (tid == 0) {
+            const uint32_t prev = ticket_acq_rel(p.ws_counters + pair);
+            misc[0] = prev == (uint32_t)(nslots - 1);
+        }
+        __syncthreads();
+        if (misc[0]) {
             uint32_t uses[2] = {0, 0};
             merge_pair_last_block<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, row, h, slot0, nslots, tid,
                                                   uses);
@@ -3050,7 +2991,6 @@ int check_fast_path(const pkv_shape &s)
 struct WsPtrs {
     uint32_t *error;
     uint32_t *counters;
-    uint32_t *flags;
     float *m, *l, *acc;
     uint32_t *host_err = nullptr;  // flag words in mapped host memory (pkv_decode_host), or NULL
 };
@@ -3126,7 +3066,6 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         uint8_t *wsb = static_cast<uint8_t *>(workspace);
         wp.error = reinterpret_cast<uint32_t *>(wsb + ws.error_off);
         wp.counters = reinterpret_cast<uint32_t *>(wsb + ws.counters_off);
-        wp.flags = reinterpret_cast<uint32_t *>(wsb + ws.flags_off);
         wp.m = reinterpret_cast<float *>(wsb + ws.m_off);
         wp.l = reinterpret_cast<float *>(wsb + ws.l_off);
         wp.acc = reinterpret_cast<float *>(wsb + ws.acc_off);
@@ -3147,7 +3086,6 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
     prm.ws_error = wp.error;
     prm.host_err = wp.host_err;
     prm.ws_counters = wp.counters;
-    prm.ws_flags = wp.flags;
     prm.ws_m = wp.m;
     prm.ws_l = wp.l;
     prm.ws_acc = wp.acc;
@@ -3420,8 +3358,7 @@ struct HostLayout {
     int32_t n_items = 0, n_indptr = 0;
     bool q_inline, bt_inline, out_inline;
     size_t q_bytes, bt_bytes;
-    size_t q_off, lens_off, items_off, indptr_off, bt_off, counters_off, flags_off, err_off, out_off, m_off, l_off,
-        acc_off;
+    size_t q_off, lens_off, items_off, indptr_off, bt_off, counters_off, err_off, out_off, m_off, l_off, acc_off;
     size_t up_bytes, down_bytes, dev_total;
     size_t h_down_off, host_total;
 };
@@ -3497,8 +3434,7 @@ int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_ru
     L->items_off = take(L->n_indptr > 0 ? (size_t)L->n_items * sizeof(pkv_work_item) : 0);
     L->indptr_off = take((size_t)L->n_indptr * 4);
     L->bt_off = L->bt_inline ? take(L->bt_bytes) : 0;
-    L->counters_off = take(ws.m_off - ws.counters_off);  // the counters, then the flags
-    L->flags_off = L->counters_off + (ws.flags_off - ws.counters_off);
+    L->counters_off = take(ws.m_off - ws.counters_off);
     L->err_off = take(kWsAlign);
     L->up_bytes = L->err_off + 16;
     L->out_off = take(L->q_bytes);
@@ -3643,8 +3579,7 @@ int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, c
     if (!ok)
         return PKV_ERR_CUDA;
     const WsPtrs wp{reinterpret_cast<uint32_t *>(dev + L.err_off), reinterpret_cast<uint32_t *>(dev + L.counters_off),
-                    reinterpret_cast<uint32_t *>(dev + L.flags_off), reinterpret_cast<float *>(dev + L.m_off),
-                    reinterpret_cast<float *>(dev + L.l_off),
+                    reinterpret_cast<float *>(dev + L.m_off), reinterpret_cast<float *>(dev + L.l_off),
                     reinterpret_cast<float *>(dev + L.acc_off),
                     direct ? reinterpret_cast<uint32_t *>(stage_dev + L.h_down_off) : nullptr};
     rc = paged_decode_impl(dev + L.q_off, k_pool, v_pool, reinterpret_cast<const int32_t *>(dev + L.bt_off),

@@ -21,13 +21,12 @@ constexpr uint32_t kErrItem = 8;
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace sections, in bytes from the workspace base.  The error word,
-// the counters and the flags are zero between calls (each call leaves them
-// so); the partial states need no initial value.
+// Workspace sections, in bytes from the workspace base.  The error word and
+// the counters are zero between calls (each call leaves them so); the
+// partial states need no initial value.
 struct WsLayout {
     size_t error_off = 0;    // uint32 error word (+ padding)
     size_t counters_off = 0; // uint32 completion counter per (row, kv head) pair
-    size_t flags_off = 0;    // uint32 "state written" flag per slot
     size_t m_off = 0;        // float m[slot][G]  (running max, log2 domain)
     size_t l_off = 0;        // float l[slot][G]
     size_t acc_off = 0;      // float acc[slot][G][D]
@@ -47,8 +46,6 @@ inline WsLayout ws_layout(const pkv_shape &s, const pkv_plan &p, int32_t n_items
     size_t off = kWsAlign;  // error word section
     w.counters_off = off;
     off += round_up((size_t)pairs * 4, kWsAlign);
-    w.flags_off = off;
-    off += round_up((size_t)w.n_slots * 4, kWsAlign);
     w.m_off = off;
     off += round_up((size_t)(w.n_slots * G) * 4, kWsAlign);
     w.l_off = off;

@@ -19,6 +19,14 @@ drawn as fp32 N(0,1) and rounded to bf16, scale = 1/sqrt(head_dim)):
   bimodal, uniform, zipf
              B=8, H_q=32, H_kv=8, D=128 traces in the style of the pages'
              study (their parameters are not published; see make())
+  long_g1, long_g2, long_g8, long_g16
+             the long context with H_q = 8, 16, 64, 128 query heads over
+             the same 8 KV heads (G = 1, 2, 8, 16): the same K/V bytes, for
+             measuring what the group size costs
+  prefix_small
+             the prefix workload's shape (B=64, G=8, 16 rows sharing a
+             128-page prefix) with lengths log-uniform in [256, 16384], small
+             enough for a profiler capture
 
 For the last three the pool holds 1.25x the pages the rows need; a random
 permutation of the pool is dealt to the rows in order, so every row's pages
@@ -42,7 +50,8 @@ SEED_CALIBRATE = 20260622
 SEED_REPORT = 20260623
 PAGE = 16
 
-NAMES = ("tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf")
+NAMES = ("tiny", "long", "crossover", "mixed", "prefix", "bimodal", "uniform", "zipf", "long_g1", "long_g2",
+         "long_g8", "long_g16", "prefix_small")
 
 
 @dataclass
@@ -113,8 +122,9 @@ def make(name: str, seed: int = SEED_REPORT, device="cpu", poison: bool = False,
         perm = torch.randperm(num_pages, generator=g)
         tables = [perm[:32].tolist()]
         shared_pages = shared_rows = 0
-    elif name == "long":
-        B, H_q, H_kv, D = 1, 32, 8, 128
+    elif name == "long" or name.startswith("long_g"):
+        B, H_kv, D = 1, 8, 128
+        H_q = H_kv * (int(name[6:]) if name.startswith("long_g") else 4)
         lens = [32768]
         num_pages = 4096
         perm = torch.randperm(num_pages, generator=g)
@@ -146,9 +156,9 @@ def make(name: str, seed: int = SEED_REPORT, device="cpu", poison: bool = False,
             jitter = (0.9 + 0.2 * torch.rand(B, generator=g, dtype=torch.float64)).tolist()
             lens = [max(1, int(32768 / (k + 1) * jitter[k])) for k in range(B)]
         return _finish(name, seed, device, poison, layout, q_scale, g, B, H_q, H_kv, D, lens)
-    elif name == "prefix":
+    elif name in ("prefix", "prefix_small"):
         B, H_q, H_kv, D = 64, 64, 8, 128
-        lens = _log_uniform(g, B, 256, 131072)
+        lens = _log_uniform(g, B, 256, 131072 if name == "prefix" else 16384)
         shared_rows, shared_pages = 16, 128
         lens = [max(n, shared_pages * PAGE + 1) if i < shared_rows else n for i, n in enumerate(lens)]
         return _finish(name, seed, device, poison, layout, q_scale, g, B, H_q, H_kv, D, lens,
