@@ -426,12 +426,15 @@ def run_ours(args):
     # the same steps with the opt-in early start (PKV_FLAG_PDL_EARLY): valid here
     # because the kernel before each step is the previous step, which writes
     # none of the lengths, table or K/V pages; reported beside the headline only
-    early_plan = bd.Plan(dp.plan.mode, dp.plan.num_splits, dp.plan.chunk_pages, dp.plan.flags | bd.FLAG_PDL_EARLY)
-    dp_early = bd.plan_decode(w.seq_lens, shape, device, plan=early_plan)
     copies = pool_copies(w, torch)
-    early_ms = time_steady(w, dp_early, args.steps, args.warmup, torch, bd, copies,
-                           graph=not args.no_graph) / args.steps
-    del dp_early
+    early_ms = None
+    if not args.shared_prefix:  # the prefix-sharing grid always waits first
+        early_plan = bd.Plan(dp.plan.mode, dp.plan.num_splits, dp.plan.chunk_pages,
+                             dp.plan.flags | bd.FLAG_PDL_EARLY)
+        dp_early = bd.plan_decode(w.seq_lens, shape, device, plan=early_plan)
+        early_ms = time_steady(w, dp_early, args.steps, args.warmup, torch, bd, copies,
+                               graph=not args.no_graph) / args.steps
+        del dp_early
     inter_k = min(args.steps, 200)
     inter_ms, filler_ms = time_interleaved(w, dp, inter_k, min(args.warmup, 5), torch, bd, copies)
     dq = device_queue_timing(w, dp, min(args.steps, 200), min(args.warmup, 5), torch, bd, copies)
@@ -458,7 +461,7 @@ def run_ours(args):
         "latency_us_p10_p90": [round(x * 1e3, 2) for x in statistics.quantiles(ms, n=10)[::8]]
         if len(ms) >= 10 else None,
         "latency_GB_s": round(w.algorithmic_bytes() / (iso_ms * 1e-3) / 1e9, 1),
-        "pdl_early": {
+        "pdl_early": None if early_ms is None else {
             "us_per_step": round(early_ms * 1e3, 3),
             "GB_s": round(w.algorithmic_bytes() / (early_ms * 1e-3) / 1e9, 2),
             "note": "same steady-state timing with PKV_FLAG_PDL_EARLY (the caller promises the preceding "

@@ -482,14 +482,17 @@ struct Cfg {
 // positions gp, gp+1, ... (stage = position % NST).  PKV_ISSUE_LANES lanes
 // issue in parallel, each waiting for its own stage to be released.
 // Returns false (after setting the error bit) when a wait timed out.
+// Pages before `start` of the batch are already in the ring (copied ahead,
+// see the split kernel's speculative start) and are skipped.
 template <int D, int NST>
 __device__ __forceinline__ bool issue_pages(const Params &p, int lane, int e, int cnt, int &gp, int head,
                                             uint32_t k_ring, uint32_t v_ring, uint32_t bar_full, uint32_t bar_empty,
-                                            uint64_t policy, int gate = INT_MAX)
+                                            uint64_t policy, int gate = INT_MAX, int start = 0)
 {
     constexpr int kStage = D * kPage * 2;
     bool ok = true;
-    for (int j0 = 0; j0 < cnt && ok; j0 += PKV_ISSUE_LANES) {
+    gp -= start;  // ring position of page j of the batch: gp + j
+    for (int j0 = start; j0 < cnt && ok; j0 += PKV_ISSUE_LANES) {
         // the page at ring position `gate` may be written by the previous
         // kernel: wait for it (whole warp) before copying it
         if (gp + j0 <= gate && gate < gp + j0 + PKV_ISSUE_LANES)
@@ -907,6 +910,41 @@ __device__ void merge_pair_last_block(const Params &p, uint8_t *smem, uint32_t m
         merge_pair_direct<D>(p, row, h, slot0, n, tid, C::kThreads);
 }
 
+// The guessed range of the block, for the L2 prefetch and the speculative
+// start: its (row, KV head), first page, page count (0: no guess) and, in
+// lane j, the block-table entry of page pg0 + j (j < PKV_L2_PREFETCH_PAGES).
+struct PageGuess {
+    int row = 0, h = 0, pg0 = 0, np = 0, e = -1;
+};
+
+// L2 prefetch of pages [pg0, pg_end) of (row, KV head h), at most
+// PKV_L2_PREFETCH_PAGES of them, one page per lane of the calling warp; the
+// block-table entries are read speculatively through L2 (see above).  With
+// `g`, the range and the entries are also kept as the block's guess.
+template <int D>
+__device__ __forceinline__ void l2_prefetch_range(const Params &p, int lane, int row, int h, int64_t pg0,
+                                                  int64_t pg_end, PageGuess *g = nullptr)
+{
+#if PKV_L2_PREFETCH_PAGES > 0
+    const int64_t j = pg0 + lane;
+    int e = -1;
+    if (lane < PKV_L2_PREFETCH_PAGES && j < pg_end && j < p.max_pages) {
+        e = ld_l2_only(p.block_table + (int64_t)row * p.max_pages + j);
+        if (e >= 0 && e < p.num_pool_pages) {
+            tma_prefetch_page_l2<D>(&p.tm_k, h, e);
+            tma_prefetch_page_l2<D>(&p.tm_v, h, e);
+        }
+    }
+    if (g) {
+        g->row = row;
+        g->h = h;
+        g->pg0 = (int)pg0;
+        g->np = pg_end > pg0 ? (int)(pg_end - pg0) : 0;
+        g->e = e;
+    }
+#endif
+}
+
 // Before its dependency wait the split kernel may read nothing that the
 // kernel before it might still be writing.  What it may do is warm L2: the
 // producer warp reads its range (work item or row length) and the first
@@ -925,14 +963,16 @@ __device__ void merge_pair_last_block(const Params &p, uint8_t *smem, uint32_t m
 // read after the wait equals the guess.  Every value used is read after the
 // wait; the guess only saves one round trip to L2 when it is right.
 template <int D>
-__device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lane, int64_t row_cap, int4 *spec)
+__device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lane, int64_t row_cap, int4 *spec,
+                                                        PageGuess &g)
 {
 #if PKV_L2_PREFETCH_PAGES > 0
     int row, h;
     int64_t pg0, pg_end;
     if (p.mode == PKV_WORK_QUEUE) {
         const int4 it = ld_l2_only(p.items + blockIdx.x);
-        if (!(it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w && it.w <= row_cap))
+        if (!(it.x >= 0 && it.x < p.B && it.y >= 0 && it.y < p.H_kv && it.z >= 0 && it.z <= it.w && it.w <= row_cap &&
+              (it.z % kPage) == 0))
             return;
         if (lane == 0)
             *spec = it;
@@ -954,33 +994,7 @@ __device__ __forceinline__ void l2_prefetch_first_pages(const Params &p, int lan
             pg_end = pg_end < pg0 + p.chunk_pages ? pg_end : pg0 + p.chunk_pages;
         }
     }
-    const int64_t j = pg0 + lane;
-    if (lane < PKV_L2_PREFETCH_PAGES && j < pg_end) {
-        const int e = ld_l2_only(p.block_table + (int64_t)row * p.max_pages + j);
-        if (e >= 0 && e < p.num_pool_pages) {
-            tma_prefetch_page_l2<D>(&p.tm_k, h, e);
-            tma_prefetch_page_l2<D>(&p.tm_v, h, e);
-        }
-    }
-#endif
-}
-
-// L2 prefetch of pages [pg0, pg_end) of (row, KV head h), at most
-// PKV_L2_PREFETCH_PAGES of them, one page per lane of the calling warp; the
-// block-table entries are read speculatively through L2 (see above).
-template <int D>
-__device__ __forceinline__ void l2_prefetch_range(const Params &p, int lane, int row, int h, int64_t pg0,
-                                                  int64_t pg_end)
-{
-#if PKV_L2_PREFETCH_PAGES > 0
-    const int64_t j = pg0 + lane;
-    if (lane < PKV_L2_PREFETCH_PAGES && j < pg_end && j < p.max_pages) {
-        const int e = ld_l2_only(p.block_table + (int64_t)row * p.max_pages + j);
-        if (e >= 0 && e < p.num_pool_pages) {
-            tma_prefetch_page_l2<D>(&p.tm_k, h, e);
-            tma_prefetch_page_l2<D>(&p.tm_v, h, e);
-        }
-    }
+    l2_prefetch_range<D>(p, lane, row, h, pg0, pg_end, &g);
 #endif
 }
 
@@ -1244,6 +1258,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         }
         mbar_init(sbase + C::kMiscOff + 8, 1);
         mbar_init(sbase + C::kMiscOff + 16, 1);
+        mbar_init(sbase + C::kMiscOff + 24, 1);  // the speculative start's verdict
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
@@ -1264,6 +1279,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         *spec_item = make_int4(-1, 0, 0, 0);
     int32_t *fill_scratch = reinterpret_cast<int32_t *>(smem);  // the idle ring, before any page copy
     int32_t *fill_res = reinterpret_cast<int32_t *>(smem + C::kFillResOff);
+    const uint32_t verify_bar = sbase + C::kMiscOff + 24;
+    PageGuess guess;  // the producer warp's guess of its range (np = 0: none)
+    const uint64_t policy = evict_first_policy();
+    int spec_k = 0;   // producer: pages copied ahead into ring positions 0 .. spec_k - 1
     if (!p.pdl_early) {
         __syncthreads();
         const bool warm = (int)blockIdx.x < p.prefetch_blocks;
@@ -1273,15 +1292,43 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
                 if (g.valid && tid == 0)
                     *spec_item = make_int4(g.row, g.h, g.tb, g.te);
                 if (g.valid && warp == NW)
-                    l2_prefetch_range<D>(p, lane, g.row, g.h, g.tb / kPage, (g.te + kPage - 1) / kPage);
+                    l2_prefetch_range<D>(p, lane, g.row, g.h, g.tb / kPage, (g.te + kPage - 1) / kPage, &guess);
             }
-        } else if (warp == NW && warm) {
-            l2_prefetch_first_pages<D>(p, lane, row_cap, spec_item);
+        } else if (warm && warp == NW) {
+            l2_prefetch_first_pages<D>(p, lane, row_cap, spec_item, guess);
         }
         __syncthreads();
         grid_dependency_wait();
         PKV_TRACE_POINT(13);
+        // Speculative start of the self-planned queue: copy the guessed
+        // range's first pages now, before the block has derived its real
+        // range from the lengths (≈ 1.5 µs).  The copies read K/V after the
+        // dependency wait, so only the guessed page ids can be wrong; the
+        // producer checks them against the real ones before the consumers
+        // touch the ring, and on any difference those ring positions are
+        // drained and skipped.  Only there: where the range is one round trip
+        // away (a host-built queue, split-S), copies issued this early
+        // measured slower, since they queue ahead of that round trip.  Not
+        // either when the queue has more rows than a warp holds in registers:
+        // its derivation then keeps its arrays in the ring.
+        if (warp == NW && p.mode == PKV_WORK_QUEUE && p.device_fill && p.B <= 32) {
+            int k = guess.np < PKV_L2_PREFETCH_PAGES ? guess.np : PKV_L2_PREFETCH_PAGES;
+            k = (k < NST ? k : NST) & ~(NW - 1);  // whole rounds of the consumer warps
+            const bool ok = lane >= k || (guess.e >= 0 && guess.e < p.num_pool_pages);
+            if (!__all_sync(0xffffffffu, ok))
+                k = 0;
+            spec_k = k;
+            if (k > 0) {
+                int gp = 0;
+                issue_pages<D, NST>(p, lane, guess.e, k, gp, guess.h, k_ring, v_ring, bar_full, bar_empty, policy);
+            }
+        }
     }
+    // a block that leaves before streaming first waits for its speculative copies
+    auto drain = [&]() {
+        if (warp == NW && lane < spec_k)
+            mbar_wait(bar_full + 8 * lane, 0, p.ws_error, kWaitLimitNs, p.host_err);
+    };
 
     // ---- which (row, KV head, token range) this block owns ----
     // The producer warp fetches the first 32 block-table entries of the
@@ -1303,8 +1350,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         }
         const FillItem f = fill_queue_item<C::kThreads>(p, fill_scratch, fill_res, false);
         PKV_TRACE_POINT(14);
-        if (!f.valid)
+        if (!f.valid) {
+            drain();
             return;
+        }
         hit = guess.x == f.row && guess.y == f.h && guess.z == f.tb && guess.w == f.te;
         row = f.row;
         h = f.h;
@@ -1317,6 +1366,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         if (slot0 + nslots > p.n_items) {
             if (tid == 0)
                 raise_error(p, kErrItem);
+            drain();
             return;
         }
         if (warp == NW) {
@@ -1341,8 +1391,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
             if (warp == NW && idx < p.max_pages)
                 g_entry = __ldg(p.block_table + (int64_t)guess.x * p.max_pages + idx);
         }
-        if ((int)blockIdx.x >= n_real)
+        if ((int)blockIdx.x >= n_real) {
+            drain();
             return;
+        }
         hit = guess.x >= 0 && guess.x == it.x && guess.y == it.y && guess.z == it.z && guess.w == it.w;
         row = it.x;
         h = it.y;
@@ -1362,6 +1414,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         if (!ok) {
             if (tid == 0)
                 raise_error(p, kErrItem);
+            drain();
             return;
         }
         if (warp == NW) {
@@ -1436,14 +1489,24 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     if (warp == NW) {
         // ================= producer: block table -> TMA page copies =================
         const int32_t *bt = p.block_table + (int64_t)row * p.max_pages + pg0;
-        const uint64_t policy = evict_first_policy();
+        // the speculative copies hold pages 0 .. spec_k - 1 when the guess was
+        // right (same pair, same first page, enough pages, same page ids);
+        // otherwise the pages start at ring position spec_k
+        const bool right = __all_sync(0xffffffffu, spec_k > 0 && row == guess.row && h == guess.h &&
+                                                       pg0 == guess.pg0 && npages >= spec_k &&
+                                                       (lane >= spec_k || e_first == guess.e));
+        if (lane == 0) {
+            misc[1] = spec_k | ((spec_k > 0 && !right) ? 0x100 : 0);
+            mbar_arrive(verify_bar);  // release: the verdict precedes the consumers' reads
+        }
+        const int skip = right ? spec_k : 0;  // pages already in the ring
 #ifdef PKV_TRACE
         long long prod_wait = 0;
         const long long prod_t0 = clock64();
 #endif
         int e_next = lane < npages ? e_first : 0;
         bool ok = true;
-        int gp = 0;
+        int gp = spec_k;  // the first ring position not holding a speculative copy
         // ring position of the row's last page, which the previous kernel may write
         int gate = INT_MAX;
         if (p.pdl_early) {
@@ -1465,7 +1528,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
 #ifdef PKV_TRACE
             const long long tw0 = clock64();
 #endif
-            ok = issue_pages<D, NST>(p, lane, e, cnt, gp, h, k_ring, v_ring, bar_full, bar_empty, policy, gate);
+            ok = issue_pages<D, NST>(p, lane, e, cnt, gp, h, k_ring, v_ring, bar_full, bar_empty, policy, gate,
+                                     base == 0 ? skip : 0);
 #ifdef PKV_TRACE
             prod_wait += clock64() - tw0;
 #endif
@@ -1512,13 +1576,31 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         long long cons_wait = 0;
         const long long cons_t0 = clock64();
 #endif
+        // the speculative start's verdict: on a wrong guess, release the ring
+        // positions its copies took (each once they landed) and read the pages
+        // from position `spec` on
+        int offset = 0;
+        if (!p.pdl_early && mbar_wait(verify_bar, 0, p.ws_error, kWaitLimitNs, p.host_err)) {
+            const int v = misc[1];
+            const int spec = v & 0xff;
+            if (v & 0x100) {
+                offset = spec;
+                for (int q = warp; q < spec; q += NW) {
+                    mbar_wait(bar_full + 8 * (q % NST), (q / NST) & 1, p.ws_error, kWaitLimitNs, p.host_err);
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_empty + 8 * (q % NST));
+                }
+            }
+        }
 
         for (int pidx = warp; pidx < npages; pidx += NW) {
-            const int s = pidx % NST;
+            const int qpos = pidx + offset;
+            const int s = qpos % NST;
 #ifdef PKV_TRACE
             const long long tw0 = clock64();
 #endif
-            const bool ready = mbar_wait(bar_full + 8 * s, (pidx / NST) & 1, p.ws_error, kWaitLimitNs, p.host_err);
+            const bool ready = mbar_wait(bar_full + 8 * s, (qpos / NST) & 1, p.ws_error, kWaitLimitNs, p.host_err);
 #ifdef PKV_TRACE
             cons_wait += clock64() - tw0;
 #endif

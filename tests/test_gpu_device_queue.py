@@ -284,3 +284,31 @@ def test_device_fill_flags_bad_lengths_and_clamps():
                           torch.tensor(clamped, dtype=torch.int32, device="cuda"), 16, w.scale, plan=host)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+def test_stale_guess_is_drained_and_skipped():
+    """Decode blocks start while the builder kernel before them still writes
+    the queue (programmatic dependent launch), so a block's guess of its item
+    comes from the previous step's queue.  The lengths alternate between two
+    sets with different queues: most guesses are wrong, and the pages copied
+    ahead from them must be drained and skipped.  Every step against the
+    oracle for its own lengths."""
+    sets = ([2500, 900, 40, 1300], [700, 2300, 1500, 33])
+    w = to_device(W.make_custom([max(a, b) for a, b in zip(*sets)], 16, 4, 128, seed=147, poison=False))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    plan = bd.select_policy(sets[0], shape, [rule(2, 148, 0, 4)])
+    dp = bd.plan_decode(sets[0], shape, "cuda", plan=plan, device_queue=True, fill_blocks=148, device_fill=False)
+    lens = torch.tensor(sets[0], dtype=torch.int32, device="cuda")
+    dev_sets = [torch.tensor(x, dtype=torch.int32, device="cuda") for x in sets]
+    outs = []
+    for i in range(8):
+        lens.copy_(dev_sets[i % 2])
+        outs.append(bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens, 16, w.scale, plan=dp))
+    torch.cuda.synchronize()
+    assert bd.workspace_status(dp) == 0
+    refs = []
+    for x in sets:
+        w.seq_lens = list(x)
+        refs.append(oracle_full(w))
+    for i, out in enumerate(outs):
+        assert_close(out.float().cpu().double().numpy(), refs[i % 2], f"step {i}")
