@@ -295,11 +295,13 @@ def time_e2e(w, K, W, torch, bd, flush):
         parts.append(d)
     breakdown = {k: round(statistics.median(p[k] for p in parts), 2) for k in parts[0]}
     breakdown["binding_us"] = round(breakdown["wall_us"] - sum(breakdown[k] for k in (
-        "host_plan_us", "host_enqueue_us", "host_wait_us", "host_unpack_us")), 2)
-    breakdown["note"] = ("medians over timed calls: host_* from the library's host clock (plan = policy + queue + "
-                         "staging image; enqueue = copies and launches queued; wait = cudaStreamSynchronize; unpack "
-                         "= out read from staging), dev_* from CUDA events, binding_us = Python and ctypes around "
-                         "the call")
+        "host_plan_us", "host_enqueue_us", "host_wait_us", "host_unpack_us", "host_events_us")), 2)
+    breakdown["note"] = ("medians over calls of pkv_decode_host_timed: host_* from the library's host clock (plan = "
+                         "policy + queue + staging image; enqueue = copy and launches queued; wait = "
+                         "cudaStreamSynchronize; unpack = the result read back; events = reading the events), dev_* "
+                         "from CUDA events recorded between the copy and the kernels, which cost time of their own "
+                         "and keep the kernel from starting early, so these calls run longer than the untimed ones "
+                         "of us_per_step; binding_us = Python and ctypes around the call")
     counters = bd.plan_counters(w.seq_lens, shape, plan)
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + lens_h.numel() * 4 + counters["queue_bytes"]
     d2h = out_h.numel() * 2 + 16

@@ -91,7 +91,8 @@ typedef enum {
 #define PKV_FLAG_SHARED_PREFIX 64 /* WORK_QUEUE only, plan {2, U, C, flags}: items / indptr hold the
                                      prefix-sharing queue of pkv_build_prefix_queue at chunk C and U is its
                                      unit count: one block per unit stages the unit's shared pages once
-                                     for all its members.  n_items = the item count.  Not with
+                                     for all its members (always with the 12-page ring, as if
+                                     PKV_FLAG_DEEP_RING were set).  n_items = the item count.  Not with
                                      PKV_FLAG_DEVICE_FILL or PKV_FLAG_PDL_EARLY (PKV_ERR_UNSUPPORTED) */
 #define PKV_FLAG_DEVICE_FILL 32   /* WORK_QUEUE only, plan {2, T, 0, flags}: no queue is passed; every
                                      block derives its own item of the compact queue whose chunk fills
@@ -475,7 +476,8 @@ typedef struct {
     double host_unpack_us;   /* out and the error word read back from host_staging */
     double dev_h2d_us;       /* device time of the host->device copies */
     double dev_kernel_us;    /* device time of the decode kernels */
-    double dev_d2h_us;       /* device time of the device->host copies */
+    double dev_d2h_us;       /* device time of the device->host copies (none when out is page-locked) */
+    double host_events_us;   /* reading the events back: the measurement's own cost, not the step's */
 } pkv_host_timing;
 
 /* pkv_decode_host that also reports where its time went into *timing (when

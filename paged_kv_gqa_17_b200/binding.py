@@ -77,7 +77,7 @@ class Counters(ctypes.Structure):
 class HostTiming(ctypes.Structure):
     """Where one pkv_decode_host call's time went (pkv_host_timing), in microseconds."""
     _fields_ = [(n, ctypes.c_double) for n in ("host_plan_us", "host_enqueue_us", "host_wait_us", "host_unpack_us",
-                                               "dev_h2d_us", "dev_kernel_us", "dev_d2h_us")]
+                                               "dev_h2d_us", "dev_kernel_us", "dev_d2h_us", "host_events_us")]
 
     def as_dict(self):
         return {f: float(getattr(self, f)) for f, _ in self._fields_}

@@ -3035,16 +3035,22 @@ cudaError_t launch_prefix(const Params &prm, int64_t grid, cudaStream_t st, bool
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_prefix_any(int D, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
+// The prefix grid always runs the 12-page ring: its 16-column tile needs
+// about 190 registers, and only the deep variant's launch bounds (two blocks
+// per SM) keep two blocks resident; with the 8-page ring one block per SM ran
+// a 64-row batch 1.6x slower than the split kernel.
+cudaError_t launch_prefix_any(int D, const Params &prm, int64_t grid, cudaStream_t st, bool pdl)
 {
-    if (D == 128)
-        return deep ? launch_prefix<128, kNSTDeep>(prm, grid, st, pdl) : launch_prefix<128, kNST>(prm, grid, st, pdl);
-    return deep ? launch_prefix<64, kNSTDeep>(prm, grid, st, pdl) : launch_prefix<64, kNST>(prm, grid, st, pdl);
+    return D == 128 ? launch_prefix<128, kNSTDeep>(prm, grid, st, pdl) : launch_prefix<64, kNSTDeep>(prm, grid, st, pdl);
 }
 
+// Head dim 128 with the 16-column tile (G > 8) also takes the 12-page ring
+// whatever the plan's flags say: with the 8-page ring's launch bounds it needs
+// 193 registers, which leaves one block per SM.
 cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_t grid, cudaStream_t st, bool pdl,
                              unsigned cluster)
 {
+    deep = deep || (D == 128 && NT == 2);
     if (cluster > 0)
         return deep ? launch_split_nst<kNSTDeep, true>(D, NT, prm, grid, st, pdl, cluster)
                     : launch_split_nst<kNST, true>(D, NT, prm, grid, st, pdl, cluster);
@@ -3211,7 +3217,7 @@ int paged_decode_impl(const void *q, const void *k_pool, const void *v_pool, con
         le = deep ? launch_balanced_nst<PKV_NST_BAL_DEEP>(s.head_dim, NT, prm, grid, st, pdl)
                   : launch_balanced_nst<PKV_NST_BAL>(s.head_dim, NT, prm, grid, st, pdl);
     else if (shared_prefix)
-        le = launch_prefix_any(s.head_dim, deep, prm, grid, st, pdl);
+        le = launch_prefix_any(s.head_dim, prm, grid, st, pdl);
     else
         le = launch_split_any(s.head_dim, NT, deep, prm, grid, st, pdl, cluster);
     if (le != cudaSuccess)
@@ -3707,6 +3713,7 @@ int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, c
             timing->dev_kernel_us = ms * 1e3;
         if (cudaEventElapsedTime(&ms, ev[2], ev[3]) == cudaSuccess)
             timing->dev_d2h_us = ms * 1e3;
+        timing->host_events_us = us(clock::now() - t4);
     }
     return status_from_error_word(err);
 }
