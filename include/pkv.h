@@ -491,6 +491,39 @@ PKV_API int pkv_decode_host_timed(const void *q_host, const int32_t *block_table
                                   size_t device_buffer_bytes, void *host_staging, size_t host_staging_bytes,
                                   void *stream, pkv_plan *plan_out, pkv_host_timing *timing);
 
+/* The arguments of pkv_decode_host as one parameter block, for a serving
+ * loop that issues the same call every step (same buffers, new contents):
+ * the caller fills the block once and passes its address each step, which
+ * spares a foreign-function binding the marshalling of sixteen arguments per
+ * call.  Every field means what the argument of the same name of
+ * pkv_decode_host_timed means; the block is read, never written, and the
+ * caller owns it. */
+typedef struct {
+    const void *q_host;
+    const int32_t *block_table_host;
+    const int32_t *seq_lens_host;
+    void *out_host;
+    const void *k_pool;
+    const void *v_pool;
+    float scale;
+    const pkv_shape *shape;
+    const pkv_policy_rule *rules;
+    int32_t n_rules;
+    void *device_buffer;
+    size_t device_buffer_bytes;
+    void *host_staging;
+    size_t host_staging_bytes;
+    void *stream;
+    pkv_plan *plan_out;
+    pkv_host_timing *timing; /* NULL, or where pkv_decode_host_timed reports its time */
+} pkv_host_call;
+
+/* pkv_decode_host_timed(call->q_host, ..., call->plan_out, call->timing):
+ * the same step, the same return codes; PKV_ERR_INVALID when call is NULL
+ * [PKV, Methodology 3 "Evaluation protocol": synchronized wall time
+ * including host planning]. */
+PKV_API int pkv_decode_host_call(const pkv_host_call *call);
+
 #ifdef __cplusplus
 }
 #endif

@@ -83,6 +83,14 @@ class HostTiming(ctypes.Structure):
         return {f: float(getattr(self, f)) for f, _ in self._fields_}
 
 
+class HostCall(ctypes.Structure):
+    """pkv_host_call: the arguments of pkv_decode_host as one parameter block."""
+    _fields_ = [("q_host", c_p), ("block_table_host", c_p), ("seq_lens_host", c_p), ("out_host", c_p),
+                ("k_pool", c_p), ("v_pool", c_p), ("scale", ctypes.c_float), ("shape", c_p), ("rules", c_p),
+                ("n_rules", c_i32), ("device_buffer", c_p), ("device_buffer_bytes", c_sz), ("host_staging", c_p),
+                ("host_staging_bytes", c_sz), ("stream", c_p), ("plan_out", c_p), ("timing", c_p)]
+
+
 _lib = None
 
 # (name, restype, argtypes) of every function include/pkv.h declares
@@ -116,6 +124,7 @@ SIGNATURES = [
      [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p]),
     ("pkv_decode_host_timed", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p, c_p]),
+    ("pkv_decode_host_call", ctypes.c_int, [c_p]),
 ]
 
 
@@ -649,11 +658,14 @@ class HostDecoder:
         self._stream = _stream_ptr(stream if stream is not None else torch.cuda.current_stream(self.device))
         self._fn = lib().pkv_decode_host
         self._fn_timed = lib().pkv_decode_host_timed
+        self._fn_call = lib().pkv_decode_host_call
         self._plan = Plan()
         self._plan_ref = ctypes.byref(self._plan)
         self._bufs = (0, 0, 0, 0)
         self._checked = ()  # weak references to the tensors (and the shape) of the last checked call
         self._args = None   # the argument tuple of the last call with the checked tensors, its scale, no rules
+        self._call = HostCall()  # the same arguments as a pkv_host_call block
+        self._call_ref = ctypes.byref(self._call)
 
     def ensure(self, seq_lens_host, shape: Shape, rules=None):
         L = lib()
@@ -666,8 +678,10 @@ class HostDecoder:
             self.dev = torch.zeros(db.value, dtype=torch.uint8, device=self.device)
         if self.host.numel() < hb.value:
             self.host = torch.zeros(hb.value, dtype=torch.uint8).pin_memory()
-        self._bufs = (self.dev.data_ptr(), self.dev.numel(), self.host.data_ptr(), self.host.numel())
-        self._args = None
+        bufs = (self.dev.data_ptr(), self.dev.numel(), self.host.data_ptr(), self.host.numel())
+        if bufs != self._bufs:  # the stored argument block names the old buffers
+            self._bufs = bufs
+            self._args = None
 
     def __call__(self, q_host: torch.Tensor, block_table_host: torch.Tensor, seq_lens_host: torch.Tensor,
                  out_host: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, scale: float, shape: Shape,
@@ -683,10 +697,10 @@ class HostDecoder:
             self._checked = tuple(weakref.ref(t) for t in (q_host, block_table_host, seq_lens_host, out_host,
                                                             k_pool, v_pool)) + (shape,)
             self._args = None
-        elif rules is None and stream is None and timing is None and self._args is not None and \
-                self._args[6] == scale:
-            # the same checked tensors as the last call: its argument tuple holds
-            rc = self._fn(*self._args)
+        elif rules is None and stream is None and self._args is not None and self._args[6] == scale:
+            # the same checked tensors as the last call: its parameter block holds
+            self._call.timing = None if timing is None else ctypes.addressof(timing)
+            rc = self._fn_call(self._call_ref)
             if rc != 0:
                 raise PkvError(rc, "pkv_decode_host")
             return Plan.from_buffer_copy(self._plan)
@@ -697,6 +711,12 @@ class HostDecoder:
                 host, host_n, self._stream if stream is None else _stream_ptr(stream), self._plan_ref)
         if rules is None and stream is None:
             self._args = args
+            c = self._call
+            (c.q_host, c.block_table_host, c.seq_lens_host, c.out_host, c.k_pool, c.v_pool, c.scale) = args[:7]
+            c.shape = ctypes.addressof(shape)
+            c.rules, c.n_rules = None, 0
+            (c.device_buffer, c.device_buffer_bytes, c.host_staging, c.host_staging_bytes, c.stream) = args[10:15]
+            c.plan_out = ctypes.addressof(self._plan)
         rc = self._fn(*args) if timing is None else self._fn_timed(*args, ctypes.byref(timing))
         if rc != 0:
             raise PkvError(rc, "pkv_decode_host")

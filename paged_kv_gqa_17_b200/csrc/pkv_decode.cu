@@ -3596,6 +3596,16 @@ int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const i
                                  host_staging_bytes, stream, plan_out, nullptr);
 }
 
+int pkv_decode_host_call(const pkv_host_call *c)
+{
+    if (c == nullptr)
+        return PKV_ERR_INVALID;
+    return pkv_decode_host_timed(c->q_host, c->block_table_host, c->seq_lens_host, c->out_host, c->k_pool,
+                                 c->v_pool, c->scale, c->shape, c->rules, c->n_rules, c->device_buffer,
+                                 c->device_buffer_bytes, c->host_staging, c->host_staging_bytes, c->stream,
+                                 c->plan_out, c->timing);
+}
+
 int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, const int32_t *seq_lens_host,
                           void *out_host, const void *k_pool, const void *v_pool, float scale,
                           const pkv_shape *shape, const pkv_policy_rule *rules, int32_t n_rules,

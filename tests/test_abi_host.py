@@ -302,3 +302,20 @@ def test_prefix_plan_counters_recount(L):
             len(o_indptr) + len(o_uptr) + len(o_uitems))
         plain = O.counters(lens, 4 * H_kv, H_kv, 64, P, (O.WORK_QUEUE, 1, C, 0))
         assert c["kv_bytes_streamed"] <= plain.kv_bytes_streamed
+
+
+def test_host_call_block_matches_the_header(L, tmp_path):
+    """bd.HostCall has pkv_host_call's size and field offsets (a C program
+    compiled against the header prints them), and the parameter-block entry
+    point rejects a NULL block before any CUDA call."""
+    fields = [f for f, _ in bd.HostCall._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"pkv.h\"\nint main(void) {\n"
+                   "  printf(\"%zu\", sizeof(pkv_host_call));\n"
+                   + "".join(f"  printf(\" %zu\", offsetof(pkv_host_call, {f}));\n" for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got == [ctypes.sizeof(bd.HostCall)] + [getattr(bd.HostCall, f).offset for f in fields]
+    assert L.pkv_decode_host_call(None) == -1

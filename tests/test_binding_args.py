@@ -207,6 +207,9 @@ def test_host_decoder_checks_each_new_tensor_object_once(monkeypatch):
     dec._plan = bd.Plan()
     dec._plan_ref = ctypes.byref(dec._plan)
     dec._fn = lambda *x: (calls.append(1), 0)[1]
+    dec._fn_call = lambda ref: (calls.append(1), 0)[1]             # repeated calls: the parameter block
+    dec._call = bd.HostCall()
+    dec._call_ref = ctypes.byref(dec._call)
     a, shape = _host_args()
     args = [a[k] for k in ("q_host", "block_table_host", "seq_lens_host", "out_host", "k_pool", "v_pool")]
 
@@ -217,6 +220,8 @@ def test_host_decoder_checks_each_new_tensor_object_once(monkeypatch):
     call()
     call()
     assert len(checks) == 1 and len(calls) == 3
+    assert dec._call.q_host == args[0].data_ptr() and dec._call.v_pool == args[5].data_ptr()
+    assert dec._call.scale == 0.125 and dec._call.shape == ctypes.addressof(shape)
     call(q=args[0].clone())                                           # a new q object
     assert len(checks) == 2
     call(shp=bd.shape_of(a["q_host"], a["k_pool"], a["block_table_host"]))   # a new shape object

@@ -7,6 +7,8 @@ tests.  Covers every plan family the policy can pick (the balanced one
 included), inputs that travel inside the packed copies and inputs too large
 for them (q, block table, out above 64 KiB), and buffer reuse after a call
 that the kernels reported a device-input error on."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -157,3 +159,38 @@ def test_pageable_out_takes_the_copy_and_matches_the_direct_path(name):
         with pytest.raises(bd.PkvError) as e:
             dec(q_h, bad, lens_h, out, w.k_pool, w.v_pool, w.scale, shape, rules=[PLANS[name]])
         assert e.value.status == -6
+
+
+def test_repeated_call_takes_the_parameter_block_and_sees_new_contents():
+    """A HostDecoder call with the same (checked) tensors as the last one goes
+    through pkv_decode_host_call with the stored parameter block; new
+    contents of those tensors (q, lengths, table) are what it decodes."""
+    w = to_device(W.make_custom([3000, 517, 0, 1200], 32, 8, 128, seed=131, poison=False))
+    q_h, bt_h, lens_h, out_h = host_inputs(w)
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table, w.layout)
+    dec = bd.HostDecoder(w.q.device)
+    dec.ensure(lens_h, shape)
+    dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape)
+    assert_close(out_h.float().double().numpy(), oracle_full(w), "first call")
+    assert dec._args is not None
+    calls = []
+    real = dec._fn_call
+    dec._fn_call = lambda ref: calls.append(1) or real(ref)
+    g = torch.Generator().manual_seed(7)
+    # lengths within each row's pages; step 1 swaps the tables of rows 0 and 3
+    for step, lens in enumerate(([2999, 528, 0, 1], [1200, 1, 0, 3008], [3000, 517, 0, 1200])):
+        new_q = torch.randn(w.q.shape, generator=g).to(torch.bfloat16)
+        q_h.copy_(new_q)
+        lens_h.copy_(torch.tensor(lens, dtype=torch.int32))
+        if step in (1, 2):
+            bt_h[[0, 3]] = bt_h[[3, 0]].clone()
+        dec.ensure(lens_h, shape)  # a serving loop's per-step sizing keeps the stored block
+        dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape)
+        w2 = dataclasses.replace(w, q=new_q.to(w.q.device), seq_lens=list(lens),
+                                 block_table=bt_h.to(w.q.device))
+        assert_close(out_h.float().double().numpy(), oracle_full(w2), f"step {step}")
+    assert len(calls) == 3
+    tm = bd.HostTiming()  # the timed step goes through the same block
+    dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, timing=tm)
+    assert len(calls) == 4 and tm.dev_kernel_us > 0 and tm.host_wait_us > 0
+    assert_close(out_h.float().double().numpy(), oracle_full(w2), "timed step")
