@@ -275,12 +275,14 @@ def time_e2e(w, K, W, torch, bd, flush):
         dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape)
     times = []
     plan = None
+    replays0 = bd.host_replays()
     for i in range(K):
         flush(i)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         plan = dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape)
         times.append((time.perf_counter() - t0) * 1e3)
+    replays = bd.host_replays() - replays0
     # where the time goes: the same calls once more through pkv_decode_host_timed
     # (host clock inside the library, CUDA events around the copies and kernels)
     parts = []
@@ -301,11 +303,12 @@ def time_e2e(w, K, W, torch, bd, flush):
                          "cudaStreamSynchronize; unpack = the result read back; events = reading the events), dev_* "
                          "from CUDA events recorded between the copy and the kernels, which cost time of their own "
                          "and keep the kernel from starting early, so these calls run longer than the untimed ones "
-                         "of us_per_step; binding_us = Python and ctypes around the call")
+                         "of us_per_step; timed calls queue the copy and launches themselves, never the graph the "
+                         "untimed ones replay; binding_us = Python and ctypes around the call")
     counters = bd.plan_counters(w.seq_lens, shape, plan)
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + lens_h.numel() * 4 + counters["queue_bytes"]
     d2h = out_h.numel() * 2 + 16
-    return times, h2d, d2h, out_h, breakdown
+    return times, h2d, d2h, out_h, breakdown, replays
 
 
 def fill_budget(w, bd):
@@ -347,11 +350,18 @@ def shared_prefix_timing(w, dp, K, W, torch, bd, copies):
     shape = bd.shape_of(w.q, w.k_pool, w.block_table)
     dpp = bd.plan_decode(w.seq_lens, shape, w.q.device, plan=dp.plan, shared_prefix_table=w.block_table.cpu())
     steady = time_steady(w, dpp, K, W, torch, bd, copies) / K
+    # the same chunk size as a plain work queue: the sharing's own effect
+    plain = bd.Plan(bd.WORK_QUEUE, 1, dpp.plan.chunk_pages, dpp.plan.flags & ~bd.FLAG_SHARED_PREFIX)
+    dpq = bd.plan_decode(w.seq_lens, shape, w.q.device, plan=plain)
+    steady_q = time_steady(w, dpq, K, W, torch, bd, copies) / K
     c = dpp.counters
     return {"plan": {"mode": "WORK_QUEUE", "units": dpp.plan.num_splits, "chunk_pages": dpp.plan.chunk_pages,
                      "flags": dpp.plan.flags}, "items": dpp.n_items, "us_per_step": round(steady * 1e3, 2),
+            "same_chunk_work_queue_us_per_step": round(steady_q * 1e3, 2),
             "kv_bytes_streamed": c["kv_bytes_streamed"], "built_in_kv_bytes_streamed": dp.counters["kv_bytes_streamed"],
-            "note": "shared chunks staged once per unit of up to 16/G sharing rows (PKV_FLAG_SHARED_PREFIX)"}
+            "note": "shared chunks staged once per unit of up to 16/G sharing rows (PKV_FLAG_SHARED_PREFIX); "
+                    "same_chunk_work_queue: the plain work queue with the same chunk, every row streaming its "
+                    "own pages"}
 
 
 def measure_workload(name, seed, device, K, W, torch, bd, W_mod, flush):
@@ -441,8 +451,8 @@ def run_ours(args):
     inter_ms, filler_ms = time_interleaved(w, dp, inter_k, min(args.warmup, 5), torch, bd, copies)
     dq = device_queue_timing(w, dp, min(args.steps, 200), min(args.warmup, 5), torch, bd, copies)
     del copies
-    e2e_ms, h2d, d2h, _, e2e_parts = time_e2e(w, args.e2e_steps or args.steps, min(args.warmup, 3), torch, bd,
-                                              flush)
+    e2e_ms, h2d, d2h, _, e2e_parts, e2e_replays = time_e2e(w, args.e2e_steps or args.steps, min(args.warmup, 3),
+                                                           torch, bd, flush)
     e2e_total = max_over_ranks(sum(e2e_ms), dist, device)
     e2e_bytes = sum_over_ranks(float(w.algorithmic_bytes() * len(e2e_ms)), dist, device)
 
@@ -503,7 +513,9 @@ def run_ours(args):
             "d2h_bytes_per_step": d2h,
             "note": "synchronized pkv_decode_host per step: host plan + queue, one H2D copy of "
                     "q/table/lengths/queue from pinned memory, kernels that write out (and any error flags) straight "
-                    "into the caller's pinned host buffers over the bus; KV cache resident",
+                    "into the caller's pinned host buffers over the bus; KV cache resident; from the second call "
+                    "with the same buffers and plan the copy and the launches are one replayed CUDA graph",
+            "graph_replays": e2e_replays,
             "breakdown": e2e_parts,
         },
         "gpu_launches": int(counters["launches"] * args.steps),

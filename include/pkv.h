@@ -455,7 +455,14 @@ PKV_API int pkv_decode_host_bytes(const int32_t *seq_lens_host, const pkv_shape 
  * pageable buffers take the packed device->host copy.  q_host,
  * block_table_host, seq_lens_host, out_host are host pointers with the
  * layouts of pkv_paged_decode; k_pool / v_pool are device pools (the cache
- * stays resident on the device).  device_buffer must be 256-byte aligned
+ * stays resident on the device).  An untimed call whose q, block table, out
+ * and staging all qualify for the paths above (page-locked, q and the table
+ * inside the staging image) and that needs the same copy and launches as the
+ * calling thread's previous call (same buffers, pools, scale, shape, plan and
+ * queue length; new contents are fine) is captured as a CUDA graph, and the
+ * thread's later calls with the same needs replay it: one graph launch per
+ * step instead of a copy and the kernel launches.  A step that cannot be
+ * captured runs as before.  device_buffer must be 256-byte aligned
  * (PKV_ERR_UNSUPPORTED otherwise); it needs no zeroing.  The plan used is
  * written to *plan_out when not NULL.  Returns the device error status like
  * pkv_workspace_status when the kernels ran. */
@@ -481,7 +488,8 @@ typedef struct {
 } pkv_host_timing;
 
 /* pkv_decode_host that also reports where its time went into *timing (when
- * not NULL; the events it records add a little device time of their own).
+ * not NULL; the events it records add a little device time of their own, and
+ * a timed call always queues its copy and launches itself, never a graph).
  * Arguments and return codes as pkv_decode_host [PKV, Methodology 3
  * "Evaluation protocol": synchronized wall time including host planning]. */
 PKV_API int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host,
@@ -517,6 +525,10 @@ typedef struct {
     pkv_plan *plan_out;
     pkv_host_timing *timing; /* NULL, or where pkv_decode_host_timed reports its time */
 } pkv_host_call;
+
+/* How many pkv_decode_host calls of the calling thread replayed a captured
+ * graph of their step (see pkv_decode_host). */
+PKV_API int64_t pkv_decode_host_replays(void);
 
 /* pkv_decode_host_timed(call->q_host, ..., call->plan_out, call->timing):
  * the same step, the same return codes; PKV_ERR_INVALID when call is NULL

@@ -20,7 +20,7 @@ _LAZY = {
     "load_rules", "default_rules", "decode_host", "PkvError",
     "NO_SPLIT", "SPLIT_S", "WORK_QUEUE", "BALANCED", "FLAG_SEPARATE_MERGE", "FLAG_NO_PDL", "FLAG_DEEP_RING",
     "build_balanced_queue", "paged_decode_noalloc", "shape_of", "HostDecoder", "FLAG_CLUSTER_MERGE",
-    "FLAG_PDL_EARLY", "FLAG_DEVICE_FILL", "FLAG_SHARED_PREFIX", "build_prefix_queue", "HostTiming", "HostCall",
+    "FLAG_PDL_EARLY", "FLAG_DEVICE_FILL", "FLAG_SHARED_PREFIX", "build_prefix_queue", "HostTiming", "HostCall", "host_replays",
     "noalloc_status", "balanced_queue_capacity",
     "build_balanced_queue_device", "fill_queue_capacity", "build_fill_queue_device",
 }

@@ -125,6 +125,7 @@ SIGNATURES = [
     ("pkv_decode_host_timed", ctypes.c_int,
      [c_p, c_p, c_p, c_p, c_p, c_p, ctypes.c_float, c_p, c_p, c_i32, c_p, c_sz, c_p, c_sz, c_p, c_p, c_p]),
     ("pkv_decode_host_call", ctypes.c_int, [c_p]),
+    ("pkv_decode_host_replays", ctypes.c_int64, []),
 ]
 
 
@@ -640,6 +641,11 @@ def workspace_status(plan: DecodePlan, stream=None) -> int:
     err = c_i32(0)
     L.pkv_workspace_status(plan.workspace.data_ptr(), _stream_ptr(stream), ctypes.byref(err))
     return int(err.value)
+
+
+def host_replays() -> int:
+    """How many pkv_decode_host calls of this thread replayed a captured graph of their step."""
+    return int(lib().pkv_decode_host_replays())
 
 
 class HostDecoder:

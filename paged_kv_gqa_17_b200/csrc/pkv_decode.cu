@@ -3483,6 +3483,55 @@ cudaEvent_t *timing_events()
     return events[dev];
 }
 
+// Everything the work a pkv_decode_host call enqueues depends on, apart from
+// the contents of the buffers: calls with equal keys enqueue the same copies
+// and launches with the same arguments.
+struct HostGraphKey {
+    int device;
+    const void *dev, *hst, *out_dev, *stage_dev, *k_pool, *v_pool;
+    float scale;
+    pkv_shape shape;
+    pkv_plan plan;
+    int32_t n_items;
+    size_t up_bytes;
+};
+
+// The calling thread's replayable step: a CUDA graph of the upload copy and
+// the decode launches, captured the second time in a row that a call comes
+// with the same key and replayed while the key stays the same.  A serving
+// loop with steady buffers and plan then queues one graph launch per step
+// instead of a copy and a kernel launch.
+struct HostGraph {
+    HostGraphKey key{}, last{};
+    bool have_key = false, have_last = false, failed = false;
+    cudaGraphExec_t exec = nullptr;
+    int64_t replays = 0;
+};
+
+HostGraph &host_graph()
+{
+    static thread_local HostGraph hg;
+    return hg;
+}
+
+bool same_key(const HostGraphKey &a, const HostGraphKey &b) { return std::memcmp(&a, &b, sizeof a) == 0; }
+
+// A non-blocking stream of the current device to capture on (capture only
+// records work, so its stream never runs anything).
+cudaStream_t capture_stream(int dev)
+{
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    if (dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();
+        streams[dev] = nullptr;
+    }
+    return streams[dev];
+}
+
 int host_layout(const int32_t *lens, const pkv_shape *shape, const pkv_policy_rule *rules, int32_t n_rules,
                 HostLayout *L)
 {
@@ -3596,6 +3645,8 @@ int pkv_decode_host(const void *q_host, const int32_t *block_table_host, const i
                                  host_staging_bytes, stream, plan_out, nullptr);
 }
 
+int64_t pkv_decode_host_replays(void) { return host_graph().replays; }
+
 int pkv_decode_host_call(const pkv_host_call *c)
 {
     if (c == nullptr)
@@ -3665,39 +3716,97 @@ int pkv_decode_host_timed(const void *q_host, const int32_t *block_table_host, c
     if (rc != PKV_OK)
         return rc;
     const clock::time_point t1 = clock::now();
-    bool ok = !ev || cudaEventRecord(ev[0], st) == cudaSuccess;
-    ok = ok && cudaMemcpyAsync(dev, hst, L.up_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
-    if (ok && !L.q_inline)
-        ok = cudaMemcpyAsync(dev + L.q_off, q_host, L.q_bytes, cudaMemcpyHostToDevice, st) == cudaSuccess;
-    if (ok && !L.bt_inline)
-        ok = cudaMemcpyAsync(dev + L.bt_off, block_table_host, L.bt_bytes, cudaMemcpyHostToDevice, st) ==
-             cudaSuccess;
-    if (ok && ev)
-        ok = cudaEventRecord(ev[1], st) == cudaSuccess;
-    if (!ok)
-        return PKV_ERR_CUDA;
-    const WsPtrs wp{reinterpret_cast<uint32_t *>(dev + L.err_off), reinterpret_cast<uint32_t *>(dev + L.counters_off),
-                    reinterpret_cast<float *>(dev + L.m_off), reinterpret_cast<float *>(dev + L.l_off),
-                    reinterpret_cast<float *>(dev + L.acc_off),
-                    direct ? reinterpret_cast<uint32_t *>(stage_dev + L.h_down_off) : nullptr};
-    rc = paged_decode_impl(dev + L.q_off, k_pool, v_pool, reinterpret_cast<const int32_t *>(dev + L.bt_off),
-                           reinterpret_cast<const int32_t *>(dev + L.lens_off), s.page_size, scale,
-                           direct ? out_dev : dev + L.out_off, shape, &L.plan,
-                           reinterpret_cast<const pkv_work_item *>(dev + L.items_off),
-                           reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, nullptr, 0, st, &wp);
-    if (rc != PKV_OK)
-        return rc;
-    ok = !ev || cudaEventRecord(ev[2], st) == cudaSuccess;
     uint8_t *h_down = hst + L.h_down_off;
-    if (!direct) {
-        ok = ok && cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
-        if (ok && !L.out_inline)
-            ok = cudaMemcpyAsync(out_host, dev + L.out_off, L.q_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    // The step's device work on stream `ss`, with the timing events when `evs`.
+    auto enqueue = [&](cudaStream_t ss, cudaEvent_t *evs) -> int {
+        bool ok = !evs || cudaEventRecord(evs[0], ss) == cudaSuccess;
+        ok = ok && cudaMemcpyAsync(dev, hst, L.up_bytes, cudaMemcpyHostToDevice, ss) == cudaSuccess;
+        if (ok && !L.q_inline)
+            ok = cudaMemcpyAsync(dev + L.q_off, q_host, L.q_bytes, cudaMemcpyHostToDevice, ss) == cudaSuccess;
+        if (ok && !L.bt_inline)
+            ok = cudaMemcpyAsync(dev + L.bt_off, block_table_host, L.bt_bytes, cudaMemcpyHostToDevice, ss) ==
+                 cudaSuccess;
+        if (ok && evs)
+            ok = cudaEventRecord(evs[1], ss) == cudaSuccess;
+        if (!ok)
+            return PKV_ERR_CUDA;
+        const WsPtrs wp{reinterpret_cast<uint32_t *>(dev + L.err_off),
+                        reinterpret_cast<uint32_t *>(dev + L.counters_off), reinterpret_cast<float *>(dev + L.m_off),
+                        reinterpret_cast<float *>(dev + L.l_off), reinterpret_cast<float *>(dev + L.acc_off),
+                        direct ? reinterpret_cast<uint32_t *>(stage_dev + L.h_down_off) : nullptr};
+        const int r = paged_decode_impl(dev + L.q_off, k_pool, v_pool, reinterpret_cast<const int32_t *>(dev + L.bt_off),
+                                        reinterpret_cast<const int32_t *>(dev + L.lens_off), s.page_size, scale,
+                                        direct ? out_dev : dev + L.out_off, shape, &L.plan,
+                                        reinterpret_cast<const pkv_work_item *>(dev + L.items_off),
+                                        reinterpret_cast<const int32_t *>(dev + L.indptr_off), L.n_items, nullptr, 0,
+                                        ss, &wp);
+        if (r != PKV_OK)
+            return r;
+        ok = !evs || cudaEventRecord(evs[2], ss) == cudaSuccess;
+        if (!direct) {
+            ok = ok &&
+                 cudaMemcpyAsync(h_down, dev + L.err_off, L.down_bytes, cudaMemcpyDeviceToHost, ss) == cudaSuccess;
+            if (ok && !L.out_inline)
+                ok = cudaMemcpyAsync(out_host, dev + L.out_off, L.q_bytes, cudaMemcpyDeviceToHost, ss) ==
+                     cudaSuccess;
+        }
+        if (ok && evs)
+            ok = cudaEventRecord(evs[3], ss) == cudaSuccess;
+        return ok ? PKV_OK : PKV_ERR_CUDA;
+    };
+    // Untimed calls whose whole step sits in page-locked buffers replay a
+    // graph of it once the same key has come twice in a row.
+    HostGraph &hg = host_graph();
+    HostGraphKey key;
+    std::memset(&key, 0, sizeof key);
+    const bool graphable = !ev && direct && L.q_inline && L.bt_inline && cudaGetDevice(&key.device) == cudaSuccess;
+    bool launched = false;
+    if (graphable) {
+        key.dev = dev;
+        key.hst = hst;
+        key.out_dev = out_dev;
+        key.stage_dev = stage_dev;
+        key.k_pool = k_pool;
+        key.v_pool = v_pool;
+        key.scale = scale;
+        key.shape = s;
+        key.plan = L.plan;
+        key.n_items = L.n_items;
+        key.up_bytes = L.up_bytes;
+        if (!(hg.have_key && same_key(hg.key, key)) && hg.have_last && same_key(hg.last, key)) {
+            // second call in a row with this key: capture its step
+            cudaGraphExec_t exec = nullptr;
+            cudaStream_t cs = capture_stream(key.device);
+            if (cs && cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) == cudaSuccess) {
+                const int r = enqueue(cs, nullptr);
+                cudaGraph_t graph = nullptr;
+                const bool ended = cudaStreamEndCapture(cs, &graph) == cudaSuccess;
+                if (r == PKV_OK && ended && graph && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess)
+                    exec = nullptr;
+                if (graph)
+                    cudaGraphDestroy(graph);
+            }
+            cudaGetLastError();  // a step that cannot be captured runs as before
+            if (hg.exec)
+                cudaGraphExecDestroy(hg.exec);  // freed once any launch of it in flight ends
+            hg.exec = exec;
+            hg.key = key;
+            hg.have_key = true;
+            hg.failed = exec == nullptr;
+        }
+        hg.last = key;
+        hg.have_last = true;
+        if (hg.have_key && same_key(hg.key, key) && !hg.failed) {
+            if (cudaGraphLaunch(hg.exec, st) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            launched = true;
+            ++hg.replays;
+        }
     }
-    if (ok && ev)
-        ok = cudaEventRecord(ev[3], st) == cudaSuccess;
+    if (!launched && (rc = enqueue(st, ev)) != PKV_OK)
+        return rc;
     const clock::time_point t2 = clock::now();
-    if (!ok || cudaStreamSynchronize(st) != cudaSuccess)
+    if (cudaStreamSynchronize(st) != cudaSuccess)
         return PKV_ERR_CUDA;
     const clock::time_point t3 = clock::now();
     uint32_t err = 0;

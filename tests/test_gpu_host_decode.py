@@ -194,3 +194,46 @@ def test_repeated_call_takes_the_parameter_block_and_sees_new_contents():
     dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, timing=tm)
     assert len(calls) == 4 and tm.dev_kernel_us > 0 and tm.host_wait_us > 0
     assert_close(out_h.float().double().numpy(), oracle_full(w2), "timed step")
+
+
+@pytest.mark.parametrize("name", sorted(PLANS))
+def test_repeated_steps_replay_a_captured_graph(name):
+    """The second call in a row with the same buffers and plan captures the
+    step as a CUDA graph and later calls replay it: every replayed step
+    decodes its own new q and matches the oracle, a call with other lengths
+    (another queue) runs without the graph, and a device-input error found
+    during a replay is reported like any other."""
+    w = to_device(W.make_custom([1000, 4097, 2500, 17, 0], 32, 8, 128, seed=132, poison=True))
+    q_h, bt_h, lens_h, out_h = host_inputs(w)
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table, w.layout)
+    rules = [PLANS[name]]
+    dec = bd.HostDecoder(w.q.device)
+    dec.ensure(lens_h, shape, rules)
+    g = torch.Generator().manual_seed(11)
+    before = bd.host_replays()
+    for step in range(4):
+        new_q = torch.randn(w.q.shape, generator=g).to(torch.bfloat16)
+        q_h.copy_(new_q)
+        out_h.fill_(float("nan"))
+        dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
+        w2 = dataclasses.replace(w, q=new_q.to(w.q.device))
+        assert_close(out_h.float().double().numpy(), oracle_full(w2), f"{name} step {step}")
+    assert bd.host_replays() - before == 3  # the first call runs directly, the next three replay
+    lens2 = [999, 4097, 2496, 16, 0]  # shorter only: the slots past each length are poisoned
+    lens_h.copy_(torch.tensor(lens2, dtype=torch.int32))
+    dec.ensure(lens_h, shape, rules)
+    dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
+    w3 = dataclasses.replace(w2, seq_lens=lens2)
+    assert_close(out_h.float().double().numpy(), oracle_full(w3), f"{name} other lengths")
+    lens_h.copy_(torch.tensor(w.seq_lens, dtype=torch.int32))
+    for _ in range(2):
+        dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
+    assert_close(out_h.float().double().numpy(), oracle_full(w2), f"{name} back")
+    bad = bt_h.clone()
+    bad[1, 3] = w.num_pages + 2
+    n = bd.host_replays()
+    with pytest.raises(bd.PkvError) as e:
+        dec(q_h, bad, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
+    assert e.value.status == -6 and bd.host_replays() == n + 1  # reported from a replayed step
+    dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
+    assert_close(out_h.float().double().numpy(), oracle_full(w2), f"{name} after the error")
