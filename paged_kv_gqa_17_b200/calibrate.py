@@ -15,7 +15,8 @@ on a holdout seed].  This script does the same by measurement:
      batches, G = 8 for the third).
   2. It times every candidate plan (no-split; split-S over several S with
      and without the deep ring, and with the cluster merge at S = 8 and 16;
-     the work queue over seven chunk sizes, with and without the deep ring,
+     the work queue over ten chunk sizes from 8 to 512 pages, with and
+     without the deep ring,
      and with the chunk size that fills one wave of 222 to 444 blocks; the
      balanced grid at one and two blocks per SM) as the steady-state device
      time of back-to-back steps over rotating pool copies.
@@ -28,6 +29,8 @@ on a holdout seed].  This script does the same by measurement:
 
 It writes the table as JSON (the library's build turns it into its built-in
 table) and prints a markdown report (also written to --report when given).
+With --only-b B it re-measures only the cells of B's row and replaces that
+row's rules in the existing table, keeping every other rule.
 """
 from __future__ import annotations
 
@@ -56,7 +59,7 @@ def candidates():
         out += [(1, S, 0, 0), (1, S, 0, 4)]
     for S in (8, 16):
         out.append((1, S, 0, 12))  # cluster merge, deep ring
-    for C in (8, 16, 24, 32, 48, 64, 96):
+    for C in (8, 16, 24, 32, 48, 64, 96, 128, 256, 512):
         out += [(2, 1, C, 0), (2, 1, C, 4)]
     # C chosen to fill one wave of T blocks: about 1.5, 1.8 and 2 blocks per SM with
     # the deep ring (two fit per SM), 2 and 3 per SM with the 8-page ring
@@ -107,10 +110,10 @@ def pick(times):
     return min(near, key=lambda c: (c[0], bin(c[3]).count("1"), times[c]))
 
 
-def build_rules(best):
-    """best[(bi, nj)] -> candidate; merge equal neighbours along N for each B range."""
+def build_rules(best, rows):
+    """best[(bi, nj)] -> candidate; merge equal neighbours along N for each B range in rows."""
     rules = []
-    for bi in range(len(B_REP)):
+    for bi in rows:
         nj = 0
         while nj < len(N_REP):
             c = best[(bi, nj)]
@@ -141,7 +144,10 @@ def main(argv=None):
     ap.add_argument("--report", default=None, help="also write the markdown report to this file")
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--draws", type=int, default=3, help="batches per cell (geometric mean)")
+    ap.add_argument("--only-b", type=int, default=None, choices=B_REP,
+                    help="re-measure only this representative B's row; keep the table's other rules")
     args = ap.parse_args(argv)
+    rows = [B_REP.index(args.only_b)] if args.only_b is not None else list(range(len(B_REP)))
 
     import torch
 
@@ -152,13 +158,20 @@ def main(argv=None):
     bd.lib()
     cands = candidates()
     best, calib = {}, {}
-    for bi, B in enumerate(B_REP):
+    for bi in rows:
+        B = B_REP[bi]
         for nj, n in enumerate(N_REP):
             t = measure_cell(B, n, W.SEED_CALIBRATE, args.steps, cands, torch, bd, W, bench, args.draws)
             calib[(bi, nj)] = t
             best[(bi, nj)] = pick(t)
             print(f"B={B:3d} N_max={n:6d} best {best[(bi, nj)]} {t[best[(bi, nj)]]:.2f} us", flush=True)
-    rules = build_rules(best)
+    rules = build_rules(best, rows)
+    if args.only_b is not None:
+        with open(args.out) as f:
+            old_rules = json.load(f)["rules"]
+        lo = B_EDGES[rows[0]]
+        rules = [r for r in old_rules if r["b_lo"] != lo] + rules
+        rules.sort(key=lambda r: (r["b_lo"], r["nmax_lo"]))
     doc = {
         "name": "b200_calibrated",
         "about": "Built-in policy table of libpkv.so (pkv_default_policy), written by "
@@ -173,13 +186,15 @@ def main(argv=None):
     # holdout check
     lines = ["# Policy calibration on B200", "",
              "Command: `python -m paged_kv_gqa_17_b200.calibrate" + (f" --report {args.report}" if args.report else "")
+             + (f" --only-b {args.only_b}" if args.only_b is not None else "")
              + "` (writes paged_kv_gqa_17_b200/policy_b200.json).", "",
              "Steady-state µs per decode step (CUDA-graph replay of back-to-back steps over rotating pool copies), "
              f"H_kv=8, D=128; each cell is the geometric mean over {args.draws} batches (G = 4, 4, 8). "
              "Calibration seed 20260622 picks the plan; holdout seed 20260623 (other batches) re-measures it.", "",
              "| B | N_max | chosen plan (mode, S/T, C, flags) | calib µs | holdout µs | holdout best | best µs | regret |",
              "|---|---|---|---|---|---|---|---|"]
-    for bi, B in enumerate(B_REP):
+    for bi in rows:
+        B = B_REP[bi]
         for nj, n in enumerate(N_REP):
             c = best[(bi, nj)]
             hold = measure_cell(B, n, W.SEED_REPORT, args.steps, cands, torch, bd, W, bench, args.draws)
