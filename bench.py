@@ -370,13 +370,16 @@ def measure_workload(name, seed, device, K, W, torch, bd, W_mod, flush):
     dp = bd.plan_decode(w.seq_lens, shape, device)
     copies = pool_copies(w, torch)
     steady = time_steady(w, dp, K, W, torch, bd, copies) / K
+    early_plan = bd.Plan(dp.plan.mode, dp.plan.num_splits, dp.plan.chunk_pages, dp.plan.flags | bd.FLAG_PDL_EARLY)
+    early = time_steady(w, bd.plan_decode(w.seq_lens, shape, device, plan=early_plan), K, W, torch, bd, copies) / K
     inter, _ = time_interleaved(w, dp, K, W, torch, bd, copies)
     dq = device_queue_timing(w, dp, K, W, torch, bd, copies)
     sp = shared_prefix_timing(w, dp, K, W, torch, bd, copies)
     del copies
     iso = time_isolated(w, dp, min(K, 50), min(W, 3), torch, bd, flush)
-    return {"w": w, "dp": dp, "ms": steady, "inter_ms": inter / K, "device_queue": dq, "shared_prefix": sp,
-            "iso_ms": statistics.median(iso), "bytes": w.algorithmic_bytes(), "bytes_unique": w.algorithmic_bytes(True)}
+    return {"w": w, "dp": dp, "ms": steady, "early_ms": early, "inter_ms": inter / K, "device_queue": dq,
+            "shared_prefix": sp, "iso_ms": statistics.median(iso), "bytes": w.algorithmic_bytes(),
+            "bytes_unique": w.algorithmic_bytes(True)}
 
 
 def cpu_baseline_leg(w, target_s):
@@ -542,6 +545,7 @@ def run_ours(args):
                            "us_per_step": round(m * 1e3, 2), "GB_s": round(gbs, 1),
                            "latency_us": round(r["iso_ms"] * 1e3, 2),
                            "interleaved_us_per_step": round(r["inter_ms"] * 1e3, 2),
+                           "pdl_early_us_per_step": round(r["early_ms"] * 1e3, 2),
                            "frac_of_measured": round(gbs / peak, 4),
                            "frac_of_nominal_8TBs": round(gbs / NOMINAL_HBM_GBS, 4),
                            "launches": r["dp"].counters["launches"]}

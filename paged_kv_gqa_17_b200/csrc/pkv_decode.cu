@@ -829,13 +829,18 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
     return true;
 }
 
-// Merge of a few states landed in the idle ring by per-thread async copies:
-// every thread issues the copies of its own (head g, 4 columns) tasks for all
-// n states (and the (m, l) pairs are shared out), so every load of the merge
-// is in flight at once without holding registers; then each thread merges
-// its tasks alone, in ascending slot order: M = max_s m_s, w_s = 2^(m_s - M)
-// (0 for a neutral state), L = sum w_s l_s, out = sum w_s acc_s / L.
-// Returns false when the ring cannot hold the n states.
+// Merge of a pair's states landed in the idle ring by per-thread async
+// copies: every thread issues the copies of its own (head g, 4 columns) tasks
+// for all n states (and the (m, l) pairs are shared out), so every load of the
+// merge is in flight at once without holding registers; then each thread
+// merges its tasks alone, in ascending slot order: M = max_s m_s,
+// w_s = 2^(m_s - M) (0 for a neutral state), L = sum w_s l_s,
+// out = sum w_s acc_s / L.  States too large for the ring go through
+// merge_pair_landed_passes; returns false when even that cannot hold them.
+template <int D, int NT, int NW, int NST>
+__device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *smem, int row, int h, int slot0,
+                                                      int n, int tid);
+
 template <int D, int NT, int NW, int NST>
 __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h, int slot0, int n, int tid)
 {
@@ -844,7 +849,7 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
     constexpr int D4 = D / 4;
     const int acc_bytes = n * G * D * 4;
     if (acc_bytes + 2 * n * G * 4 > C::kRingBytes)
-        return false;
+        return merge_pair_landed_passes<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid);
     float *acc_s = reinterpret_cast<float *>(smem);  // [n][G][D]
     float *m_s = acc_s + n * G * D;                  // [n][G]
     float *l_s = m_s + n * G;                        // [n][G]
@@ -893,9 +898,72 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
     return true;
 }
 
+// The landed merge in two or four passes over the columns, for states whose
+// D columns do not fit the ring at once: each pass lands D/2 or D/4 columns
+// of all n states (the m and l of all states land once, behind them) and
+// merges them as above.  A call of its own, so that the kernels' main loops
+// keep their registers.  Returns false when a quarter of the columns does
+// not fit either.
+template <int D, int NT, int NW, int NST>
+__device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *smem, int row, int h, int slot0,
+                                                      int n, int tid)
+{
+    using C = Cfg<D, NT, NW, NST>;
+    const int G = p.G;
+    const int ml_bytes = 2 * n * G * 4;
+    int parts = 2;
+    if (n * G * (D / 2) * 4 + ml_bytes > C::kRingBytes)
+        parts = 4;
+    if (n * G * (D / parts) * 4 + ml_bytes > C::kRingBytes)
+        return false;
+    const int Dp = D / parts;  // columns per pass
+    const int Dp4 = Dp / 4;
+    float *acc_s = reinterpret_cast<float *>(smem);  // [n][G][Dp]
+    float *m_s = acc_s + n * G * Dp;                 // [n][G]
+    float *l_s = m_s + n * G;                        // [n][G]
+    const uint32_t base = smem_addr(smem);
+    const float *acc_g = p.ws_acc + (int64_t)slot0 * G * D;
+    for (int part = 0; part < parts; ++part) {
+        const int c0 = part * Dp;
+        for (int e = tid; e < G * Dp4; e += C::kThreads) {
+            const int g = e / Dp4;
+            const int d4 = (e % Dp4) * 4;
+            for (int s = 0; s < n; ++s)
+                cp_async_16(base + 4 * ((s * G + g) * Dp + d4), acc_g + (int64_t)(s * G + g) * D + c0 + d4);
+        }
+        if (part == 0)
+            for (int i = tid; i < n * G; i += C::kThreads) {
+                cp_async_4(smem_addr(m_s + i), p.ws_m + (int64_t)slot0 * G + i);
+                cp_async_4(smem_addr(l_s + i), p.ws_l + (int64_t)slot0 * G + i);
+            }
+        cp_async_wait_all();
+        __syncthreads();
+        for (int e = tid; e < G * Dp4; e += C::kThreads) {
+            const int g = e / Dp4;
+            const int d4 = (e % Dp4) * 4;
+            float M = -INFINITY;
+            for (int s = 0; s < n; ++s)
+                M = fmaxf(M, m_s[s * G + g]);
+            float L = 0.f;
+            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < n; ++s) {
+                const float m = m_s[s * G + g];
+                const float w = m == -INFINITY ? 0.f : exp2_approx(m - M);
+                L = fmaf(w, l_s[s * G + g], L);
+                O = fma4(*reinterpret_cast<const float4 *>(acc_s + (s * G + g) * Dp + d4), w, O);
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + c0 + d4, scale4(O, inv));
+        }
+        __syncthreads();  // the next pass refills the ring; after the last one it is free again
+    }
+    return true;
+}
+
 // The last block's merge of a pair: through per-thread async copies into the
-// ring whenever the ring holds all n states ("landed"), else staged through
-// the ring in double-buffered bulk copies, else straight into registers.
+// ring whenever the ring holds a quarter of the columns of all n states
+// ("landed", in one, two or four passes), else staged through the ring in
+// double-buffered bulk copies, else straight into registers.
 // Timed on B200 with the step's own blocks merging: landed beat staged at 17
 // states (mixed batch, 18.3 -> 17.5 us per step) and at 32 (long context,
 // 24.2 -> 23.2 us per step).

@@ -81,6 +81,8 @@ CASES = {
     "g16_d128": ([900, 123], 32, 2, 128),
     "g6_d64": ([257, 40], 12, 2, 64),
     "g12_d128": ([600], 24, 2, 128),
+    "g8_d64": ([3000, 77], 16, 2, 64),   # 32 states of 2 KB: the D = 64 ring lands them in column passes
+    "g16_d64": ([2100], 32, 2, 64),      # 32 or more states of 4 KB: staged through the 8-page ring
 }
 
 
@@ -201,6 +203,21 @@ def test_full_size_configs_every_output(name):
     w = to_device(W.make(name, poison=True))
     got, dp = run(w)
     assert dp.plan.mode in (1, 2) and dp.plan.flags & 4, dp.plan
+    ref = oracle_full(w, threads=CORES)
+    assert_close(got, ref, f"{name} plan {dp.plan}")
+    assert rel_l2(got, ref) < 1e-2
+
+
+@pytest.mark.parametrize("name", ["long_g8", "long_g16"])
+@pytest.mark.parametrize("mode", [None, "split32"])
+def test_long_context_wide_groups_every_output(name, mode):
+    """The long context at G = 8 and 16, where a pair's 32 partial states
+    (128 and 256 KB) exceed the idle ring and the last block merges them in
+    two or four passes over the columns: every output, in the built-in plan
+    and at S = 32 without flags."""
+    w = to_device(W.make(name, poison=True))
+    got, dp = run(w, mode_rule=MODES[mode] if mode else None)
+    assert dp.plan.mode == 1 and dp.plan.num_splits == 32, dp.plan
     ref = oracle_full(w, threads=CORES)
     assert_close(got, ref, f"{name} plan {dp.plan}")
     assert rel_l2(got, ref) < 1e-2
