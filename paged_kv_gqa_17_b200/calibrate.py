@@ -138,6 +138,13 @@ def build_rules(best, rows):
     return rules
 
 
+def replace_row(old_rules, row_rules, b_lo):
+    """The table with the rules of the B range starting at b_lo replaced by
+    row_rules, ordered by (b_lo, nmax_lo)."""
+    rules = [r for r in old_rules if r["b_lo"] != b_lo] + list(row_rules)
+    return sorted(rules, key=lambda r: (r["b_lo"], r["nmax_lo"]))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--out", default=os.path.join(HERE, "policy_b200.json"))
@@ -168,10 +175,7 @@ def main(argv=None):
     rules = build_rules(best, rows)
     if args.only_b is not None:
         with open(args.out) as f:
-            old_rules = json.load(f)["rules"]
-        lo = B_EDGES[rows[0]]
-        rules = [r for r in old_rules if r["b_lo"] != lo] + rules
-        rules.sort(key=lambda r: (r["b_lo"], r["nmax_lo"]))
+            rules = replace_row(json.load(f)["rules"], rules, B_EDGES[rows[0]])
     doc = {
         "name": "b200_calibrated",
         "about": "Built-in policy table of libpkv.so (pkv_default_policy), written by "

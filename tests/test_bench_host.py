@@ -63,3 +63,28 @@ def test_recorded_traffic_follows_the_kernel_source_hash(monkeypatch):
     assert bench.recorded_traffic(name) is None
     assert bench.recorded_traffic("no-such-workload") is None
 
+
+
+def test_calibration_row_replacement_keeps_the_other_rows_and_covers_the_grid():
+    """calibrate --only-b: the re-measured row's rules replace exactly the
+    old rules of that B range; together they still cover every (B, N_max)
+    of the grid exactly once, and build_rules merges equal neighbours."""
+    import json
+
+    from paged_kv_gqa_17_b200 import calibrate as cal
+
+    old = json.load(open(os.path.join(ROOT, "paged_kv_gqa_17_b200", "policy_b200.json")))["rules"]
+    bi = cal.B_REP.index(8)
+    best = {(bi, nj): (2, 1, 48, 4) if nj < 3 else (2, 296, 0, 0) for nj in range(len(cal.N_REP))}
+    row = cal.build_rules(best, [bi])
+    assert [(r["nmax_lo"], r["nmax_hi"]) for r in row] == [(0, 16384), (16384, 2**31 - 1)]
+    assert row[0] == {"b_lo": 8, "b_hi": 16, "nmax_lo": 0, "nmax_hi": 16384, "mode": "WORK_QUEUE",
+                      "chunk_pages": 48, "flags": 4}
+    assert row[1]["num_splits"] == 296 and row[1]["chunk_pages"] == 0 and "flags" not in row[1]
+    new = cal.replace_row(old, row, cal.B_EDGES[bi])
+    assert [r for r in new if r["b_lo"] != 8] == [r for r in old if r["b_lo"] != 8]
+    assert [r for r in new if r["b_lo"] == 8] == row
+    for B in (1, 2, 3, 4, 7, 8, 15, 16, 31, 32, 64, 1000):
+        for n in (0, 1023, 1024, 5000, 16383, 16384, 70000, 2**31 - 2):
+            hits = [r for r in new if r["b_lo"] <= B < r["b_hi"] and r["nmax_lo"] <= n < r["nmax_hi"]]
+            assert len(hits) == 1, (B, n, hits)
