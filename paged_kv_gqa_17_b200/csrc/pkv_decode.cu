@@ -835,13 +835,13 @@ __device__ bool merge_pair_staged(const Params &p, uint8_t *smem, uint32_t mbar0
 // merge is in flight at once without holding registers; then each thread
 // merges its tasks alone, in ascending slot order: M = max_s m_s,
 // w_s = 2^(m_s - M) (0 for a neutral state), L = sum w_s l_s,
-// out = sum w_s acc_s / L.  States too large for the ring go through
-// merge_pair_landed_passes; returns false when even that cannot hold them.
+// out = sum w_s acc_s / L.  With kPasses, states too large for the ring go
+// through merge_pair_landed_passes; returns false when they cannot land.
 template <int D, int NT, int NW, int NST>
 __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *smem, int row, int h, int slot0,
                                                       int n, int tid);
 
-template <int D, int NT, int NW, int NST>
+template <int D, int NT, int NW, int NST, bool kPasses>
 __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h, int slot0, int n, int tid)
 {
     using C = Cfg<D, NT, NW, NST>;
@@ -849,7 +849,7 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
     constexpr int D4 = D / 4;
     const int acc_bytes = n * G * D * 4;
     if (acc_bytes + 2 * n * G * 4 > C::kRingBytes)
-        return merge_pair_landed_passes<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid);
+        return kPasses && merge_pair_landed_passes<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid);
     float *acc_s = reinterpret_cast<float *>(smem);  // [n][G][D]
     float *m_s = acc_s + n * G * D;                  // [n][G]
     float *l_s = m_s + n * G;                        // [n][G]
@@ -966,13 +966,15 @@ __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *
 // double-buffered bulk copies, else straight into registers.
 // Timed on B200 with the step's own blocks merging: landed beat staged at 17
 // states (mixed batch, 18.3 -> 17.5 us per step) and at 32 (long context,
-// 24.2 -> 23.2 us per step).
-template <int D, int NT, int NW, int NST>
+// 24.2 -> 23.2 us per step).  The balanced grid merges without the column
+// passes (kPasses false): the out-of-line call cost its main loop registers
+// (128 with spills instead of 140) and 0.7-2.9 us per step.
+template <int D, int NT, int NW, int NST, bool kPasses = true>
 __device__ void merge_pair_last_block(const Params &p, uint8_t *smem, uint32_t mbar0, int row, int h, int slot0,
                                       int n, int tid, uint32_t (&uses)[2])
 {
     using C = Cfg<D, NT, NW, NST>;
-    if (merge_pair_landed<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid))
+    if (merge_pair_landed<D, NT, NW, NST, kPasses>(p, smem, row, h, slot0, n, tid))
         return;
     if (!merge_pair_staged<D, NT, NW, NST>(p, smem, mbar0, row, h, slot0, n, tid, uses))
         merge_pair_direct<D>(p, row, h, slot0, n, tid, C::kThreads);
@@ -2418,7 +2420,8 @@ __global__ void __launch_bounds__((NW + 1) * 32) balanced_kernel(const __grid_co
     uint32_t uses[2] = {0, 0};
     for (int k = 0; k < nd; ++k) {
         const int4 d = deferred[k];
-        merge_pair_last_block<D, NT, NW, NST>(p, smem, sbase + C::kMiscOff + 8, d.x, d.y, d.z, d.w, tid, uses);
+        merge_pair_last_block<D, NT, NW, NST, false>(p, smem, sbase + C::kMiscOff + 8, d.x, d.y, d.z, d.w, tid,
+                                                     uses);
         __syncthreads();
         if (tid == 0)
             p.ws_counters[d.x * p.H_kv + d.y] = 0u;  // ready for the next call
