@@ -902,8 +902,9 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
 // D columns do not fit the ring at once: each pass lands D/2 or D/4 columns
 // of all n states (the m and l of all states land once, behind them) and
 // merges them as above.  A call of its own, so that the kernels' main loops
-// keep their registers.  Returns false when a quarter of the columns does
-// not fit either.
+// keep their registers.  Returns false (the caller stages the states instead)
+// when a quarter of the columns does not fit either, or when a pass would
+// leave most threads idle.
 template <int D, int NT, int NW, int NST>
 __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *smem, int row, int h, int slot0,
                                                       int n, int tid)
@@ -914,7 +915,12 @@ __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *
     int parts = 2;
     if (n * G * (D / 2) * 4 + ml_bytes > C::kRingBytes)
         parts = 4;
-    if (n * G * (D / parts) * 4 + ml_bytes > C::kRingBytes)
+    // Each pass merges G * D / (4 * parts) (head, 4-column) tasks, one per
+    // thread, with n dependent steps each; with fewer than 128 tasks (G = 4,
+    // or G = 8 in four passes) the staged merge, whose chunks keep all 128
+    // consumer threads busy, measured faster (long context at G = 4 with the
+    // 8-page ring: 25.2 against 26.6 us per step).
+    if (n * G * (D / parts) * 4 + ml_bytes > C::kRingBytes || G * D / (4 * parts) < 128)
         return false;
     const int Dp = D / parts;  // columns per pass
     const int Dp4 = Dp / 4;
@@ -1295,14 +1301,17 @@ __device__ __forceinline__ FillItem fill_queue_item(const Params &p, int32_t *sm
 }
 
 // One block = one work item (row, KV head, token range) for all G query heads.
-// The deep-ring variants (two blocks per SM at most, by shared memory) tell
-// the compiler so.  With that hint the D = 128, G <= 8 variants come out at
-// 128 registers, which still lets the 8-stage ones run three blocks per SM,
-// and they measured faster on B200 than the unhinted allocation (115
-// registers) at every timed configuration (long context, crossover, mixed,
-// many-wave queues).
-template <int D, int NT, int NW, int NST, bool CL>
-__global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kernel(const __grid_constant__ Params p)
+// The launch bounds say how many blocks share an SM: two for the deep ring
+// (by shared memory), three for the 8-page ring.  The three-block hint keeps
+// the 8-stage D = 128, G <= 8 variant at 128 registers; without it the
+// kernel grew to 134 registers, which fit only two blocks of five warps per
+// SM (registers are handed out per SM sub-partition), and many-wave queues
+// ran up to 25 % slower.
+// FILL: the self-planned queue (PKV_FLAG_DEVICE_FILL) and its speculative
+// start are compiled into a variant of their own: in the other variants
+// their code cost the main loop 6 registers and 0.1-0.3 us per step.
+template <int D, int NT, int NW, int NST, bool CL, bool FILL>
+__global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 3)) split_kernel(const __grid_constant__ Params p)
 {
     using C = Cfg<D, NT, NW, NST>;
     extern __shared__ uint8_t smem_raw[];
@@ -1356,7 +1365,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     if (!p.pdl_early) {
         __syncthreads();
         const bool warm = (int)blockIdx.x < p.prefetch_blocks;
-        if (p.mode == PKV_WORK_QUEUE && p.device_fill) {
+        if (FILL && p.mode == PKV_WORK_QUEUE) {
             if (warm) {
                 const FillItem g = fill_queue_item<C::kThreads>(p, fill_scratch, fill_res, true);
                 if (g.valid && tid == 0)
@@ -1381,7 +1390,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         // measured slower, since they queue ahead of that round trip.  Not
         // either when the queue has more rows than a warp holds in registers:
         // its derivation then keeps its arrays in the ring.
-        if (warp == NW && p.mode == PKV_WORK_QUEUE && p.device_fill && p.B <= 32) {
+        if (FILL && warp == NW && p.mode == PKV_WORK_QUEUE && p.B <= 32) {
             int k = guess.np < PKV_L2_PREFETCH_PAGES ? guess.np : PKV_L2_PREFETCH_PAGES;
             k = (k < NST ? k : NST) & ~(NW - 1);  // whole rounds of the consumer warps
             const bool ok = lane >= k || (guess.e >= 0 && guess.e < p.num_pool_pages);
@@ -1408,7 +1417,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
     int e_first = 0;
     bool hit = false;  // the guessed work item was the real one
     int row_len = -1;  // the row's length where known (for the early dependency gate)
-    if (p.mode == PKV_WORK_QUEUE && p.device_fill) {
+    if (FILL && p.mode == PKV_WORK_QUEUE) {
         // the block's own item, derived from the device lengths; the
         // table entries at the guessed item's first page go out first
         const int4 guess = p.pdl_early ? make_int4(-1, 0, 0, 0) : *spec_item;
@@ -1565,7 +1574,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         const bool right = __all_sync(0xffffffffu, spec_k > 0 && row == guess.row && h == guess.h &&
                                                        pg0 == guess.pg0 && npages >= spec_k &&
                                                        (lane >= spec_k || e_first == guess.e));
-        if (lane == 0) {
+        if (FILL && lane == 0) {
             misc[1] = spec_k | ((spec_k > 0 && !right) ? 0x100 : 0);
             mbar_arrive(verify_bar);  // release: the verdict precedes the consumers' reads
         }
@@ -1650,7 +1659,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, (NST >= 12 ? 2 : 1)) split_kern
         // positions its copies took (each once they landed) and read the pages
         // from position `spec` on
         int offset = 0;
-        if (!p.pdl_early && mbar_wait(verify_bar, 0, p.ws_error, kWaitLimitNs, p.host_err)) {
+        if (FILL && !p.pdl_early && mbar_wait(verify_bar, 0, p.ws_error, kWaitLimitNs, p.host_err)) {
             const int v = misc[1];
             const int spec = v & 0xff;
             if (v & 0x100) {
@@ -3013,12 +3022,12 @@ cudaError_t launch_ex(void (*kernel)(Args...), unsigned grid, unsigned block, si
     return cudaLaunchKernelEx(&cfg, kernel, prm);
 }
 
-template <int D, int NT, int NST, bool CL>
+template <int D, int NT, int NST, bool CL, bool FILL>
 cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st, bool pdl, unsigned cluster)
 {
     using C = Cfg<D, NT, kNW, NST>;
     static std::atomic<uint64_t> configured{0};
-    auto kernel = split_kernel<D, NT, kNW, NST, CL>;
+    auto kernel = split_kernel<D, NT, kNW, NST, CL, FILL>;
     cudaError_t e = set_smem(kernel, kMaxDynSmem, configured);
     if (e != cudaSuccess)
         return e;
@@ -3044,15 +3053,20 @@ cudaError_t launch_split(const Params &prm, int64_t grid, cudaStream_t st, bool 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int NST, bool CL>
+template <int NST, bool CL, bool FILL>
 cudaError_t launch_split_nst(int D, int NT, const Params &prm, int64_t grid, cudaStream_t st, bool pdl,
                              unsigned cluster)
 {
-    if (D == 128)
-        return NT == 1 ? launch_split<128, 1, NST, CL>(prm, grid, st, pdl, cluster)
-                       : launch_split<128, 2, NST, CL>(prm, grid, st, pdl, cluster);
-    return NT == 1 ? launch_split<64, 1, NST, CL>(prm, grid, st, pdl, cluster)
-                   : launch_split<64, 2, NST, CL>(prm, grid, st, pdl, cluster);
+    if (D == 128) {
+        if (NT == 1)
+            return launch_split<128, 1, NST, CL, FILL>(prm, grid, st, pdl, cluster);
+        if constexpr (NST >= 12)
+            return launch_split<128, 2, NST, CL, FILL>(prm, grid, st, pdl, cluster);
+        else
+            return cudaErrorInvalidConfiguration;  // launch_split_any gives this tile the deep ring
+    }
+    return NT == 1 ? launch_split<64, 1, NST, CL, FILL>(prm, grid, st, pdl, cluster)
+                   : launch_split<64, 2, NST, CL, FILL>(prm, grid, st, pdl, cluster);
 }
 
 #ifndef PKV_NST_BAL
@@ -3123,10 +3137,13 @@ cudaError_t launch_split_any(int D, int NT, bool deep, const Params &prm, int64_
 {
     deep = deep || (D == 128 && NT == 2);
     if (cluster > 0)
-        return deep ? launch_split_nst<kNSTDeep, true>(D, NT, prm, grid, st, pdl, cluster)
-                    : launch_split_nst<kNST, true>(D, NT, prm, grid, st, pdl, cluster);
-    return deep ? launch_split_nst<kNSTDeep, false>(D, NT, prm, grid, st, pdl, 0)
-                : launch_split_nst<kNST, false>(D, NT, prm, grid, st, pdl, 0);
+        return deep ? launch_split_nst<kNSTDeep, true, false>(D, NT, prm, grid, st, pdl, cluster)
+                    : launch_split_nst<kNST, true, false>(D, NT, prm, grid, st, pdl, cluster);
+    if (prm.device_fill)
+        return deep ? launch_split_nst<kNSTDeep, false, true>(D, NT, prm, grid, st, pdl, 0)
+                    : launch_split_nst<kNST, false, true>(D, NT, prm, grid, st, pdl, 0);
+    return deep ? launch_split_nst<kNSTDeep, false, false>(D, NT, prm, grid, st, pdl, 0)
+                : launch_split_nst<kNST, false, false>(D, NT, prm, grid, st, pdl, 0);
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
