@@ -237,6 +237,12 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src)
                  : "memory");
 }
 
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most the most recently committed group of this thread's
+// async copies is still in flight.
+__device__ __forceinline__ void cp_async_wait_but_last() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
 __device__ __forceinline__ void cp_async_wait_all()
 {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -841,6 +847,54 @@ template <int D, int NT, int NW, int NST>
 __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *smem, int row, int h, int slot0,
                                                       int n, int tid);
 
+// The merge weights of a pair's n landed states, once per head rather than
+// once per column task: warp w takes the heads g = w, w + warps, ...; for
+// each it finds M_g = max_s m_s, overwrites m_s with w_s = 2^(m_s - M_g)
+// (0 for a neutral state) and writes L_g = sum_s w_s l_s to lsum[g].
+template <int kThreads>
+__device__ __forceinline__ void merge_weights(float *m_s, const float *l_s, float *lsum, int n, int G, int tid)
+{
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int g = warp; g < G; g += kThreads / 32) {
+        float M = -INFINITY;
+        for (int s = lane; s < n; s += 32)
+            M = fmaxf(M, m_s[s * G + g]);
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1)
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+        float L = 0.f;
+        for (int s = lane; s < n; s += 32) {
+            const float m = m_s[s * G + g];
+            const float w = m == -INFINITY ? 0.f : exp2_approx(m - M);
+            m_s[s * G + g] = w;
+            L = fmaf(w, l_s[s * G + g], L);
+        }
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1)
+            L += __shfl_xor_sync(0xffffffffu, L, sh);
+        if (lane == 0)
+            lsum[g] = L;
+    }
+}
+
+// One (head g, 4 columns) task of a landed merge: sum_s w_s acc_s over the
+// n states in ascending slot order (two interleaved chains), divided by L_g.
+__device__ __forceinline__ float4 merge_task(const float *acc_s, const float *w_s, int n, int G, int g, int stride,
+                                             int d4, float L)
+{
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f), O2 = O;
+    int s = 0;
+    for (; s + 1 < n; s += 2) {
+        O = fma4(*reinterpret_cast<const float4 *>(acc_s + (s * G + g) * stride + d4), w_s[s * G + g], O);
+        O2 = fma4(*reinterpret_cast<const float4 *>(acc_s + ((s + 1) * G + g) * stride + d4), w_s[(s + 1) * G + g],
+                  O2);
+    }
+    if (s < n)
+        O = fma4(*reinterpret_cast<const float4 *>(acc_s + (s * G + g) * stride + d4), w_s[s * G + g], O);
+    O = make_float4(O.x + O2.x, O.y + O2.y, O.z + O2.z, O.w + O2.w);
+    return scale4(O, L > 0.f ? 1.f / L : 0.f);
+}
+
 template <int D, int NT, int NW, int NST, bool kPasses>
 __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h, int slot0, int n, int tid)
 {
@@ -848,13 +902,21 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
     const int G = p.G;
     constexpr int D4 = D / 4;
     const int acc_bytes = n * G * D * 4;
-    if (acc_bytes + 2 * n * G * 4 > C::kRingBytes)
+    if (acc_bytes + (2 * n * G + G) * 4 > C::kRingBytes)
         return kPasses && merge_pair_landed_passes<D, NT, NW, NST>(p, smem, row, h, slot0, n, tid);
     float *acc_s = reinterpret_cast<float *>(smem);  // [n][G][D]
-    float *m_s = acc_s + n * G * D;                  // [n][G]
+    float *m_s = acc_s + n * G * D;                  // [n][G], then the weights
     float *l_s = m_s + n * G;                        // [n][G]
+    float *lsum = l_s + n * G;                       // [G]
     const uint32_t base = smem_addr(smem);
     const float *acc_g = p.ws_acc + (int64_t)slot0 * G * D;
+    // m and l land first, the accumulators behind them: the weights are
+    // computed while the accumulators are still in flight
+    for (int i = tid; i < n * G; i += C::kThreads) {
+        cp_async_4(smem_addr(m_s + i), p.ws_m + (int64_t)slot0 * G + i);
+        cp_async_4(smem_addr(l_s + i), p.ws_l + (int64_t)slot0 * G + i);
+    }
+    cp_async_commit();
 #pragma unroll
     for (int k = 0; k < C::kMaxMergeTasks; ++k) {
         const int e = tid + k * C::kThreads;
@@ -867,10 +929,10 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
             }
         }
     }
-    for (int i = tid; i < n * G; i += C::kThreads) {
-        cp_async_4(smem_addr(m_s + i), p.ws_m + (int64_t)slot0 * G + i);
-        cp_async_4(smem_addr(l_s + i), p.ws_l + (int64_t)slot0 * G + i);
-    }
+    cp_async_commit();
+    cp_async_wait_but_last();
+    __syncthreads();
+    merge_weights<C::kThreads>(m_s, l_s, lsum, n, G, tid);
     cp_async_wait_all();
     __syncthreads();
 #pragma unroll
@@ -879,19 +941,8 @@ __device__ bool merge_pair_landed(const Params &p, uint8_t *smem, int row, int h
         if (e < G * D4) {
             const int g = e / D4;
             const int d4 = (e % D4) * 4;
-            float M = -INFINITY;
-            for (int s = 0; s < n; ++s)
-                M = fmaxf(M, m_s[s * G + g]);
-            float L = 0.f;
-            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s = 0; s < n; ++s) {
-                const float m = m_s[s * G + g];
-                const float w = m == -INFINITY ? 0.f : exp2_approx(m - M);
-                L = fmaf(w, l_s[s * G + g], L);
-                O = fma4(*reinterpret_cast<const float4 *>(acc_s + (s * G + g) * D + d4), w, O);
-            }
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4, scale4(O, inv));
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + d4,
+                         merge_task(acc_s, m_s, n, G, g, D, d4, lsum[g]));
         }
     }
     __syncthreads();  // the ring is free again once every thread has left it
@@ -911,7 +962,7 @@ __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *
 {
     using C = Cfg<D, NT, NW, NST>;
     const int G = p.G;
-    const int ml_bytes = 2 * n * G * 4;
+    const int ml_bytes = (2 * n * G + G) * 4;
     int parts = 2;
     if (n * G * (D / 2) * 4 + ml_bytes > C::kRingBytes)
         parts = 4;
@@ -925,10 +976,16 @@ __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *
     const int Dp = D / parts;  // columns per pass
     const int Dp4 = Dp / 4;
     float *acc_s = reinterpret_cast<float *>(smem);  // [n][G][Dp]
-    float *m_s = acc_s + n * G * Dp;                 // [n][G]
+    float *m_s = acc_s + n * G * Dp;                 // [n][G], then the weights
     float *l_s = m_s + n * G;                        // [n][G]
+    float *lsum = l_s + n * G;                       // [G]
     const uint32_t base = smem_addr(smem);
     const float *acc_g = p.ws_acc + (int64_t)slot0 * G * D;
+    for (int i = tid; i < n * G; i += C::kThreads) {
+        cp_async_4(smem_addr(m_s + i), p.ws_m + (int64_t)slot0 * G + i);
+        cp_async_4(smem_addr(l_s + i), p.ws_l + (int64_t)slot0 * G + i);
+    }
+    cp_async_commit();
     for (int part = 0; part < parts; ++part) {
         const int c0 = part * Dp;
         for (int e = tid; e < G * Dp4; e += C::kThreads) {
@@ -937,29 +994,19 @@ __device__ __noinline__ bool merge_pair_landed_passes(const Params &p, uint8_t *
             for (int s = 0; s < n; ++s)
                 cp_async_16(base + 4 * ((s * G + g) * Dp + d4), acc_g + (int64_t)(s * G + g) * D + c0 + d4);
         }
-        if (part == 0)
-            for (int i = tid; i < n * G; i += C::kThreads) {
-                cp_async_4(smem_addr(m_s + i), p.ws_m + (int64_t)slot0 * G + i);
-                cp_async_4(smem_addr(l_s + i), p.ws_l + (int64_t)slot0 * G + i);
-            }
+        cp_async_commit();
+        if (part == 0) {
+            cp_async_wait_but_last();
+            __syncthreads();
+            merge_weights<C::kThreads>(m_s, l_s, lsum, n, G, tid);
+        }
         cp_async_wait_all();
         __syncthreads();
         for (int e = tid; e < G * Dp4; e += C::kThreads) {
             const int g = e / Dp4;
             const int d4 = (e % Dp4) * 4;
-            float M = -INFINITY;
-            for (int s = 0; s < n; ++s)
-                M = fmaxf(M, m_s[s * G + g]);
-            float L = 0.f;
-            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s = 0; s < n; ++s) {
-                const float m = m_s[s * G + g];
-                const float w = m == -INFINITY ? 0.f : exp2_approx(m - M);
-                L = fmaf(w, l_s[s * G + g], L);
-                O = fma4(*reinterpret_cast<const float4 *>(acc_s + (s * G + g) * Dp + d4), w, O);
-            }
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + c0 + d4, scale4(O, inv));
+            store_bf16x4(p.out + ((int64_t)row * p.H_q + (int64_t)h * G + g) * D + c0 + d4,
+                         merge_task(acc_s, m_s, n, G, g, Dp, d4, lsum[g]));
         }
         __syncthreads();  // the next pass refills the ring; after the last one it is free again
     }
