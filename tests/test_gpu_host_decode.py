@@ -63,6 +63,7 @@ PLANS = {
     "bal37": rule(3, 37),
     "bal296": rule(3, 296),
     "split16_cl": rule(1, 16, 0, 8),
+    "wqfill37_dev": rule(2, 37, 0, 4 | 32),  # blocks derive their items from the uploaded lengths
 }
 
 
