@@ -2585,7 +2585,9 @@ __global__ void wait_timeout_selftest_kernel(uint32_t *err, uint64_t limit_ns)
 // item per head owned by the last block whose share starts at or before the
 // pair's position; indptr holds the pair offsets, then the block offsets.
 // One block of threads: the row page counts and the per-pair item counts are
-// each prefix-summed over the block, and each thread emits its pair's items.
+// each prefix-summed over the block, then the items are emitted one per
+// thread (each finds its pair by a binary search of the pair offsets), so a
+// pair spread over many shares no longer costs one thread a serial loop.
 
 constexpr int kBuildThreads = 256;
 constexpr int kBuildWarps = kBuildThreads / 32;
@@ -2706,6 +2708,7 @@ __global__ void __launch_bounds__(kBuildThreads)
         pair_span(q, a, n);
         return share_owner(U, T, n == 0 ? a : a + n - 1);
     };
+    // the pairs' item counts and offsets
     carry = 0;
     for (int64_t base = 0; base < pairs; base += kBuildThreads) {
         const int64_t p = base + tid;
@@ -2718,42 +2721,69 @@ __global__ void __launch_bounds__(kBuildThreads)
             cnt = n == 0 ? 1 : (span < n ? span : n);
         }
         const int64_t incl = block_inclusive_scan(cnt, scan);
-        const int64_t o = carry + incl - cnt;
-        if (p < pairs) {
-            indptr[p] = (int32_t)o;
-            const int i = (int)(p / H_kv), h = (int)(p % H_kv);
-            const int64_t N = clamped_len(i);
-            int64_t prev = p == 0 ? -1 : last_owner(p - 1);
-            int64_t x = a, idx = o;
-            for (int64_t k = 0; k < cnt; ++k, ++idx) {
-                const int64_t b = share_owner(U, T, x);
-                int4 it = make_int4(i, h, 0, 0);
-                if (n > 0) {
-                    const int64_t end = share_start(U, T, b + 1);
-                    const int64_t y = a + n < end ? a + n : end;
-                    it.z = (int)((x - a) * P);
-                    it.w = (int)((y - a) * P < N ? (y - a) * P : N);
-                    x = y;
-                }
-                if (idx < capacity)
-                    items[idx] = it;
-                else
-                    atomicOr(err, kErrItem);
-                for (int64_t c = prev + 1; c <= b; ++c)
-                    block_ptr[c] = (int32_t)idx;
-                prev = b;
-            }
-            if (p == pairs - 1) {
-                indptr[pairs] = (int32_t)(o + cnt);
-                for (int64_t c = prev + 1; c <= T; ++c)
-                    block_ptr[c] = (int32_t)(o + cnt);
-            }
-        }
+        if (p < pairs)
+            indptr[p] = (int32_t)(carry + incl - cnt);
         if (tid == kBuildThreads - 1)
             total = carry + incl;
         __syncthreads();
         carry = total;
         __syncthreads();
+    }
+    const int64_t n_items = carry;
+    if (tid == 0)
+        indptr[pairs] = (int32_t)n_items;
+    __syncthreads();  // the offsets are visible to every thread
+    // The items, one thread per item: item k of pair p covers the pair's pages
+    // [x_k, x_{k+1}) of share b_k; when every share holds a page (U >= T) the
+    // pair's owners are consecutive, b_k = b_0 + k and x_k = max(a, start(b_k)),
+    // otherwise every share holds at most one page and item k is page a + k.
+    // Each item also sets the block offsets of the shares after the previous
+    // item's owner up to its own.
+    auto item_owner = [&](int64_t a, int64_t n, int64_t k) {
+        if (n == 0)
+            return share_owner(U, T, a);
+        return U >= T ? share_owner(U, T, a) + k : share_owner(U, T, a + k);
+    };
+    for (int64_t idx = tid; idx < n_items; idx += kBuildThreads) {
+        int64_t lo = 0, hi = pairs - 1;  // the pair: the last offset <= idx (offsets rise strictly)
+        while (lo < hi) {
+            const int64_t mid = (lo + hi + 1) / 2;
+            if (indptr[mid] <= idx)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int64_t p = lo;
+        const int64_t k = idx - indptr[p];
+        int64_t a, n;
+        pair_span(p, a, n);
+        const int i = (int)(p / H_kv), h = (int)(p % H_kv);
+        const int64_t b = item_owner(a, n, k);
+        int4 it = make_int4(i, h, 0, 0);
+        if (n > 0) {
+            const int64_t N = clamped_len(i);
+            int64_t x, y;
+            if (U >= T) {
+                x = k == 0 ? a : share_start(U, T, b);
+                const int64_t end = share_start(U, T, b + 1);
+                y = a + n < end ? a + n : end;
+            } else {
+                x = a + k;
+                y = x + 1;
+            }
+            it.z = (int)((x - a) * P);
+            it.w = (int)((y - a) * P < N ? (y - a) * P : N);
+        }
+        if (idx < capacity)
+            items[idx] = it;
+        else
+            atomicOr(err, kErrItem);
+        const int64_t prev = k > 0 ? item_owner(a, n, k - 1) : (p == 0 ? -1 : last_owner(p - 1));
+        for (int64_t c = prev + 1; c <= b; ++c)
+            block_ptr[c] = (int32_t)idx;
+        if (idx == n_items - 1)
+            for (int64_t c = b + 1; c <= T; ++c)
+                block_ptr[c] = (int32_t)n_items;
     }
 }
 
