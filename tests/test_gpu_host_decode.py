@@ -238,3 +238,45 @@ def test_repeated_steps_replay_a_captured_graph(name):
     assert e.value.status == -6 and bd.host_replays() == n + 1  # reported from a replayed step
     dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape, rules=rules)
     assert_close(out_h.float().double().numpy(), oracle_full(w2), f"{name} after the error")
+
+
+def test_two_threads_each_replay_their_own_step():
+    """Two host threads, each with its own HostDecoder and stream, call the
+    host path concurrently (the binding releases the interpreter lock during
+    the call): each thread keeps its own captured graph and every output
+    matches the oracle for that thread's q."""
+    import threading
+
+    w = to_device(W.make_custom([2500, 700, 33], 32, 8, 128, seed=133, poison=True))
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table, w.layout)
+    results, errors = {}, []
+
+    def worker(tag, seed):
+        try:
+            st = torch.cuda.Stream()
+            q_h, bt_h, lens_h, out_h = host_inputs(w)
+            dec = bd.HostDecoder(w.q.device, stream=st)
+            dec.ensure(lens_h, shape)
+            g = torch.Generator().manual_seed(seed)
+            before = bd.host_replays()
+            outs = []
+            for _ in range(6):
+                q = torch.randn(w.q.shape, generator=g).to(torch.bfloat16)
+                q_h.copy_(q)
+                dec(q_h, bt_h, lens_h, out_h, w.k_pool, w.v_pool, w.scale, shape)
+                outs.append((q, out_h.clone()))
+            results[tag] = (outs, bd.host_replays() - before)
+        except Exception as e:  # reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(t, 50 + t)) for t in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for tag, (outs, replays) in results.items():
+        assert replays == 5, (tag, replays)  # per thread: one direct call, then replays
+        for q, out in outs[::2]:
+            w2 = dataclasses.replace(w, q=q.to(w.q.device))
+            assert_close(out.float().double().numpy(), oracle_full(w2), f"thread {tag}")
