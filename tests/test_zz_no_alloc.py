@@ -33,6 +33,7 @@ RULES = [
     bd.Rule(*ANY, 3, 24, 0, 0),   # balanced grid: several items per block, deferred merges
     bd.Rule(*ANY, 1, 8, 0, 8),    # split-S as clusters merging over distributed shared memory
     bd.Rule(*ANY, 3, 37, 0, 4),   # balanced grid, deep ring
+    bd.Rule(*ANY, 2, 37, 0, 36),  # self-planned queue: the blocks derive their items from the lengths
 ]
 
 
