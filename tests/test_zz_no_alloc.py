@@ -34,6 +34,7 @@ RULES = [
     bd.Rule(*ANY, 1, 8, 0, 8),    # split-S as clusters merging over distributed shared memory
     bd.Rule(*ANY, 3, 37, 0, 4),   # balanced grid, deep ring
     bd.Rule(*ANY, 2, 37, 0, 36),  # self-planned queue: the blocks derive their items from the lengths
+    bd.Rule(*ANY, 1, 16, 0, 20),  # split-S with the early start (the kernel before writes only outputs)
 ]
 
 
@@ -82,6 +83,26 @@ def test_noalloc_matches_workspace_entry_point(L, lens, H_q, H_kv, D):
         assert bd.noalloc_status() == 0, f"device error after the no-alloc calls, plan {dp.plan}"
         _close(first, ref, f"first call, plan {dp.plan}")
         _close(second, ref, f"second call, plan {dp.plan}")
+
+
+def test_noalloc_prefix_sharing_plan(L):
+    """The prefix-sharing grid through the no-alloc entry point: rows that
+    share leading pages, the same outputs as the workspace entry point."""
+    w = to_device(W.make_custom([1200, 1100, 900, 40, 2000], 32, 8, 128, seed=303, poison=True, shared_rows=3,
+                                shared_pages=32))
+    lens_dev = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
+    shape = bd.shape_of(w.q, w.k_pool, w.block_table)
+    dp = bd.plan_decode(w.seq_lens, shape, "cuda", rules=[bd.Rule(*ANY, 2, 1, 16, 4)],
+                        shared_prefix_table=w.block_table.cpu())
+    assert dp.plan.flags & bd.FLAG_SHARED_PREFIX and dp.n_items > dp.plan.num_splits  # some units share
+    ref = bd.paged_decode(w.q, w.k_pool, w.v_pool, w.block_table, lens_dev, w.P, w.scale, plan=dp)
+    torch.cuda.synchronize()
+    assert bd.workspace_status(dp) == 0
+    for call in ("first", "second"):
+        got = _noalloc(L, w, dp, lens_dev)
+        torch.cuda.synchronize()
+        assert bd.noalloc_status() == 0
+        _close(got, ref, f"{call} call, prefix-sharing plan")
 
 
 def test_noalloc_rejects_plans_larger_than_its_scratch(L):
